@@ -1,0 +1,455 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+* brute-force recomputation of stable slots on tiny inputs, and the HT row
+  order recomputed with a library stable sort;
+* hand-worked examples under tests/golden/ (routing, balanced plans, an FP8
+  block, a combine);
+* the OCP E4M3 code table and torch's float8_e4m3fn / bfloat16 converters
+  over every finite bf16 value and a set of scales;
+* plan invariants over many random count vectors (every load is floor or
+  ceil of L/R when no slot overflow is flagged, at most S replicas per rank,
+  pieces cover each expert exactly once, the layout is a permutation);
+* closed forms: identity expert with weights summing to 1 returns x
+  bit-exactly; the fp32 combine stays within its error bound of the fp64 sum;
+* adjoint identities of combine/combine-backward and dispatch/
+  dispatch-backward, exact on small-integer data.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from combine_ep_dispatch_03_b200 import synth
+from conftest import golden_path
+
+
+def _kv(path):
+    rows = {}
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        key, *vals = line.split()
+        rows[key] = vals
+    return rows
+
+
+def _golden_value(tok: str) -> float:
+    if "*2^" in tok:
+        a, b = tok.split("*2^")
+        return float(a) * 2.0 ** int(b)
+    if tok.startswith("2^"):
+        return 2.0 ** int(tok[2:])
+    if tok == "-0":
+        return -0.0
+    return float(tok)
+
+
+# ------------------------------------------------------------------ formats
+
+def test_e4m3_golden_table(orc):
+    for line in open(golden_path("e4m3_ofp8_codes.txt")):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        val, code = line.split()[:2]
+        got = int(orc.e4m3_from_f32(np.array([_golden_value(val)], np.float32))[0])
+        assert got == int(code, 16), (val, hex(got), code)
+
+
+def _all_finite_bf16() -> np.ndarray:
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    f = (bits.astype(np.uint32) << 16).view(np.float32)
+    return f[np.isfinite(f)]
+
+
+def test_e4m3_matches_torch_in_range_all_bf16_times_scales(orc):
+    x = _all_finite_bf16()
+    rng = np.random.default_rng(0)
+    amaxes = np.concatenate([[448.0, 1.0, 3.5, 2.0 ** -20, 1e4], rng.lognormal(0.0, 2.0, 59)]).astype(np.float32)
+    scales = (amaxes / np.float32(448.0)).astype(np.float32)
+    for s in scales:
+        with np.errstate(over="ignore"):
+            v = (x / s).astype(np.float32)  # IEEE single division, as the method states
+        v = v[np.isfinite(v)]
+        inr = np.abs(v) <= 448.0
+        got = orc.e4m3_from_f32(v)
+        ref = torch.from_numpy(v[inr]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        np.testing.assert_array_equal(got[inr], ref)
+        # finite values beyond the format saturate to +-448
+        out = ~inr
+        np.testing.assert_array_equal(got[out], np.where(v[out] > 0, 0x7E, 0xFE).astype(np.uint8))
+
+
+def test_e4m3_decode_roundtrip(orc):
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    vals = orc.e4m3_to_f32(codes)
+    np.testing.assert_array_equal(orc.e4m3_from_f32(vals), codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    np.testing.assert_array_equal(vals, ref)
+
+
+def test_bf16_rounding_matches_torch(orc):
+    rng = np.random.default_rng(1)
+    bits = rng.integers(0, 1 << 32, size=1 << 20, dtype=np.uint64).astype(np.uint32)
+    special = np.array([0x3F808000, 0x3F818000, 0x7F7FFFFF, 0x7F7F8000, 0x00008000, 0x80018000, 0x00000001],
+                       np.uint32)
+    f = np.concatenate([bits, special]).view(np.float32)
+    f = f[~np.isnan(f)]
+    got = orc.bf16_from_f32(f)
+    ref = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, ref)
+
+
+# ------------------------------------------------------------------ routing
+
+def _brute_slots(idx: np.ndarray, E: int):
+    """O(L^2): a pair is routed if its id is in range and not repeated earlier
+    in its token; its slot counts the earlier routed pairs of its expert."""
+    T, K = idx.shape
+    flat = idx.reshape(-1)
+
+    def routed(p):
+        e = flat[p]
+        if e < 0 or e >= E:
+            return False
+        t = p // K
+        return e not in flat[t * K:p]
+
+    j = np.full(T * K, -1, np.int64)
+    for p in range(T * K):
+        if routed(p):
+            j[p] = sum(1 for q in range(p) if flat[q] == flat[p] and routed(q))
+    return j
+
+
+def test_route_golden(orc):
+    g = _kv(golden_path("route_worked.txt"))
+    idx = np.array(g["idx"], np.int32).reshape(4, 2)
+    r = orc.route(idx, E=4, R=2, mode="ht")
+    np.testing.assert_array_equal(r.cnt, np.array(g["cnt"], np.int32))
+    np.testing.assert_array_equal(r.j, np.array(g["j"], np.int32))
+    np.testing.assert_array_equal(r.dest_row, np.array(g["ht_dest"], np.int32))
+    assert r.flags == 0
+    ll = orc.route(idx, E=4, R=2, mode="ll", cap=int(g["ll_cap"][0]))
+    np.testing.assert_array_equal(ll.dest_row, np.array(g["ll_dest"], np.int32))
+    assert ll.flags == int(g["ll_flags"][0])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_route_brute_force(orc, seed):
+    rng = np.random.default_rng(seed)
+    T, K, E = int(rng.integers(1, 40)), int(rng.integers(1, 5)), int(rng.choice([4, 8, 16]))
+    idx = rng.integers(-1, E + 1, size=(T, K)).astype(np.int32)  # includes masked, bad and repeated ids
+    r = orc.route(idx, E=E, R=2 if E % 2 == 0 else 1)
+    np.testing.assert_array_equal(r.j, _brute_slots(idx, E))
+    routed = r.j >= 0
+    np.testing.assert_array_equal(r.cnt, np.bincount(idx.reshape(-1)[routed], minlength=E))
+    bad = ((idx < -1) | (idx >= E)).any()
+    assert bool(r.flags & orc.FLAG_BAD_EXPERT_ID) == bool(bad)
+
+
+@pytest.mark.parametrize("E,R,K,T", [(16, 4, 2, 128), (64, 8, 8, 300), (8, 2, 3, 77)])
+def test_route_ht_order_is_stable_sort(orc, E, R, K, T):
+    idx, _ = synth.routing(T, E, K, seed=E + T)
+    r = orc.route(idx, E=E, R=R)
+    flat = idx.numpy().reshape(-1)
+    order = np.argsort(flat, kind="stable")  # HT rows: by expert, ties in (t, k) order
+    inv = np.empty_like(order)
+    inv[order] = np.arange(order.size)
+    np.testing.assert_array_equal(r.dest_row, inv)
+    assert r.cnt.sum() == T * K  # counts sum to T*K
+    assert sorted(r.dest_row.tolist()) == list(range(T * K))  # each pair exactly once
+
+
+def test_route_ll_capacity(orc):
+    idx, _ = synth.routing(200, 8, 2, zipf_s=2.0, seed=3)
+    cap = 20
+    r = orc.route(idx, E=8, R=2, mode="ll", cap=cap)
+    j = _brute_slots(idx.numpy(), 8)
+    flat = idx.numpy().reshape(-1)
+    expect = np.where((j >= 0) & (j < cap), flat * cap + j, -1)
+    np.testing.assert_array_equal(r.dest_row, expect)
+    assert r.flags & orc.FLAG_CAPACITY
+    np.testing.assert_array_equal(r.recv_counts, np.minimum(np.bincount(flat, minlength=8), cap))
+
+
+# ------------------------------------------------------------------ plan
+
+def _golden_plans():
+    cases, cur = [], None
+    for line in open(golden_path("plan_worked.txt")):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        key, *vals = line.split()
+        if key == "case":
+            cur = {}
+        elif key == "end":
+            cases.append(cur)
+        else:
+            cur[key] = [int(v) for v in vals]
+    return cases
+
+
+def _idx_from_counts(cnt):
+    """One pair per token, tokens ordered by expert: the stable index of the
+    i-th token of expert e is i."""
+    return np.concatenate([np.full(c, e, np.int32) for e, c in enumerate(cnt)] or [np.zeros(0, np.int32)])[:, None]
+
+
+def test_plan_golden(orc):
+    for c in _golden_plans():
+        E, R, S = c["E"][0], c["R"][0], c["S"][0]
+        idx = _idx_from_counts(c["cnt"])
+        r = orc.route(idx, E=E, R=R, balanced=True, slots=S)
+        p = r.plan
+        np.testing.assert_array_equal(p["keep"], c["keep"])
+        np.testing.assert_array_equal(p["replica_expert"].reshape(-1), c["replica_expert"])
+        np.testing.assert_array_equal(p["slot_start"].reshape(-1), c["slot_start"])
+        np.testing.assert_array_equal(p["slot_len"].reshape(-1), c["slot_len"])
+        np.testing.assert_array_equal(p["rank_load"], c["rank_load"])
+        np.testing.assert_array_equal(p["rank_off"], c["rank_off"])
+        assert r.flags == c["flags"][0]
+        flat = idx.reshape(-1)
+        for e in range(E):
+            np.testing.assert_array_equal(r.dest_row[flat == e], c.get(f"rows{e}", []))
+
+
+def _plan_invariants(orc, cnt, R, S):
+    E = len(cnt)
+    g = E // R
+    idx = _idx_from_counts(cnt)
+    r = orc.route(idx, E=E, R=R, balanced=True, slots=S)
+    p = r.plan
+    L = int(np.sum(cnt))
+    q, rem = divmod(L, R)
+    load = p["rank_load"]
+    assert load.sum() == L
+    overflow = bool(r.flags & orc.FLAG_PLAN_SLOTS)
+    if not overflow:
+        np.testing.assert_array_equal(load, [q + (i < rem) for i in range(R)])
+    rep = p["replica_expert"]
+    assert ((rep >= 0).sum(axis=1) <= S).all()
+    # slots are used in order, and a rank never hosts a replica of its own expert
+    for rr in range(R):
+        used = rep[rr] >= 0
+        assert not used[np.argmin(used):].any() or used.all()
+        assert all(e // g != rr for e in rep[rr][used])
+    # pieces of every expert cover [0, cnt) exactly once, owner piece first
+    for e in range(E):
+        pieces = [(0, int(p["keep"][e]))]
+        sl = np.argwhere(rep == e)
+        pieces += [(int(p["slot_start"][a, b]), int(p["slot_len"][a, b])) for a, b in sl]
+        if p["tail_start"][e] >= 0:
+            pieces.append((int(p["tail_start"][e]), int(p["tail_len"][e])))
+        covered = sorted(x for s0, n in pieces for x in range(s0, s0 + n))
+        assert covered == list(range(int(cnt[e])))
+    # the layout is a permutation and each rank's rows sit in its region
+    assert sorted(r.dest_row.tolist()) == list(range(L))
+    return overflow
+
+
+@pytest.mark.parametrize("E,R", [(16, 4), (64, 8), (56, 8), (8, 2), (6, 3), (12, 4), (32, 8), (128, 8), (384, 16)])
+def test_plan_invariants_random_counts(orc, E, R):
+    rng = np.random.default_rng(E * 131 + R)
+    g = E // R
+    n_over = 0
+    trials = 60
+    for trial in range(trials):
+        kind = trial % 4
+        if kind == 0:
+            cnt = rng.integers(0, 50, E)
+        elif kind == 1:  # Zipf-like skew
+            w = 1.0 / np.arange(1, E + 1) ** rng.uniform(0.5, 2.0)
+            cnt = rng.multinomial(int(rng.integers(1, 4000)), w / w.sum())
+        elif kind == 2:  # all on one expert
+            cnt = np.zeros(E, np.int64)
+            cnt[rng.integers(E)] = rng.integers(1, 500)
+        else:
+            cnt = np.zeros(E, np.int64)  # empty routing, or a few sparse experts
+            if trial % 8 == 7:
+                cnt[rng.integers(E, size=3)] = rng.integers(0, 9, 3)
+        n_over += _plan_invariants(orc, cnt.astype(np.int32), R, g)
+    if g >= R:
+        assert n_over == 0  # the greedy never ran out of slots on these shapes
+
+
+def test_plan_balances_zipf_routing(orc):
+    """Imbalance sweep shape: per-rank load flat across skew under the plan."""
+    E, R, K, T = 128, 8, 8, 4096
+    for s in (0.0, 0.5, 1.0, 1.5):
+        idx, _ = synth.routing(T, E, K, zipf_s=s, seed=11)
+        r = orc.route(idx, E=E, R=R, balanced=True)
+        assert r.flags == 0
+        assert r.plan["rank_load"].max() - r.plan["rank_load"].min() <= 1
+
+
+# ------------------------------------------------------------------ dispatch
+
+def test_fp8_block_golden(orc):
+    g = _kv(golden_path("quant_combine_worked.txt"))
+    H = 256
+    x = np.zeros((1, H), np.float32)
+    for tok in g["fp8_nonzero"]:
+        i, v = tok.split(":")
+        x[0, int(i)] = float(v)
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    recv, scales, _, _ = orc.dispatch(xb, np.zeros((1, 1), np.int32), np.ones((1, 1), np.float32),
+                                      np.zeros(1, np.int32), 1, fp8=True)
+    assert scales[0, 0] == np.float32(g["fp8_scale"][0])
+    assert scales[0, 1] == np.float32(g["fp8_zero_scale"][0])  # second block is all zero
+    expect = np.zeros(H, np.uint8)
+    for tok in g["fp8_codes"]:
+        i, c = tok.split(":")
+        expect[int(i)] = int(c, 16)
+    np.testing.assert_array_equal(recv[0], expect)
+
+
+def test_fp8_dequant_error_bound(orc):
+    T, H = 64, 1024
+    x = synth.tokens_bf16(T, H, seed=5)
+    x[3, :128] = 0  # an all-zero block
+    x[4, 128:256] *= 1000.0
+    idx = np.zeros((T, 1), np.int32)
+    recv, scales, _, _ = orc.dispatch(x, idx, np.ones((T, 1), np.float32), np.arange(T, dtype=np.int32), T,
+                                      fp8=True)
+    xf = x.float().numpy().astype(np.float64)
+    sc = np.repeat(scales, 128, axis=1).astype(np.float64)
+    deq = orc.e4m3_to_f32(recv.reshape(-1)).reshape(T, H).astype(np.float64) * sc  # exact in fp64
+    amax = np.abs(xf).reshape(T, H // 128, 128).max(axis=2)
+    np.testing.assert_array_equal(scales == 0, amax == 0)
+    # |q*s - x| <= half an e4m3 step at |x|/s, times s, plus the fp32 division's
+    # half-ulp (ties such as x/s = 84 meet the first term with equality)
+    a = np.abs(xf) / np.maximum(sc, 1e-30)
+    ex = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))
+    half_step = 0.5 * 2.0 ** (ex - 3) * sc
+    assert (np.abs(deq - xf) <= half_step + a * 2.0 ** -24 * sc + 1e-300).all()
+    assert (recv.reshape(T, H)[3, :128] == 0).all()
+
+
+def test_dispatch_bf16_rows_follow_sorted_pairs(orc):
+    T, H, E, K, R = 128, 256, 16, 2, 4
+    x = synth.tokens_bf16(T, H, seed=2)
+    idx, w = synth.routing(T, E, K, seed=2)
+    r = orc.route(idx, E=E, R=R)
+    recv, _, rw, re = orc.dispatch(x, idx, w, r.dest_row, r.recv_rows)
+    order = np.argsort(idx.numpy().reshape(-1), kind="stable")
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(recv, xb[order // K])
+    np.testing.assert_array_equal(re, idx.numpy().reshape(-1)[order])
+    np.testing.assert_array_equal(rw, w.numpy().reshape(-1)[order])
+
+
+# ------------------------------------------------------------------ combine
+
+def test_combine_golden(orc):
+    g = _kv(golden_path("quant_combine_worked.txt"))
+    y = np.array([g["comb_y0"], g["comb_y1"]], np.float32)
+    yb = torch.from_numpy(y).to(torch.bfloat16)
+    w = np.array([g["comb_w"]], np.float32)
+    out = orc.combine(yb, w, np.array([0, 1], np.int32), T=1, K=2)
+    np.testing.assert_array_equal(orc.bf16_bits_to_f32(out[0]), np.array(g["comb_out"], np.float32))
+    w2 = np.array([[0.7, 0.3]], np.float32)
+    ones = torch.ones((2, 4), dtype=torch.bfloat16)
+    out2 = orc.combine(ones, w2, np.array([0, 1], np.int32), T=1, K=2)
+    assert (orc.bf16_bits_to_f32(out2) == 1.0).all()
+
+
+@pytest.mark.parametrize("mode", ["ht", "ll", "balanced"])
+def test_identity_expert_returns_x(orc, mode):
+    T, H, E, K, R = 128, 1024, 16, 2, 4
+    x = synth.tokens_bf16(T, H, seed=0)
+    idx, w = synth.routing(T, E, K, zipf_s=1.0 if mode == "balanced" else 0.0, seed=0)
+    r = orc.route(idx, E=E, R=R, mode="ll" if mode == "ll" else "ht", cap=T, balanced=mode == "balanced")
+    recv, _, _, _ = orc.dispatch(x, idx, w, r.dest_row, r.recv_rows)
+    out = orc.combine(recv, w, r.dest_row, T, K)
+    np.testing.assert_array_equal(out, x.view(torch.int16).numpy().view(np.uint16))
+
+
+def test_affine_expert_and_fp64_error_bound(orc):
+    T, H, E, K, R = 96, 512, 32, 8, 8
+    x = synth.tokens_bf16(T, H, seed=4)
+    idx, w = synth.routing(T, E, K, seed=4)
+    r = orc.route(idx, E=E, R=R)
+    recv, _, _, _ = orc.dispatch(x, idx, w, r.dest_row, r.recv_rows)
+    rt = torch.from_numpy(recv.view(np.int16)).view(torch.bfloat16)
+    y = synth.affine_expert(rt)
+    # perturb each row so the K contributions differ
+    y = (y.float() * torch.linspace(0.5, 1.5, y.shape[0])[:, None]).to(torch.bfloat16)
+    out = orc.bf16_bits_to_f32(orc.combine(y, w, r.dest_row, T, K)).reshape(T, H).astype(np.float64)
+    yf = y.float().numpy().astype(np.float64)
+    wf = w.numpy().astype(np.float64)
+    dest = r.dest_row.reshape(T, K)
+    exact = np.einsum("tk,tkh->th", wf, yf[dest])
+    absum = np.einsum("tk,tkh->th", np.abs(wf), np.abs(yf[dest]))
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact), 2.0 ** -126))) - 7)
+    bound = 0.5 * ulp + K * 2.0 ** -24 * absum * 1.01 + 2.0 ** -133
+    assert (np.abs(out - exact) <= bound + 0.5 * ulp).all()
+    # a dropped term or a wrong row would be far outside this bound
+    assert np.abs(out - exact).max() < 0.05
+
+
+def _int_bf16(rng, shape, lo=-8, hi=9):
+    return torch.from_numpy(rng.integers(lo, hi, size=shape).astype(np.float32)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("balanced", [False, True])
+def test_adjoint_identities_exact(orc, balanced):
+    rng = np.random.default_rng(7)
+    T, H, E, K, R = 40, 128, 8, 3, 4
+    idx, _ = synth.routing(T, E, K, zipf_s=1.5 if balanced else 0.0, seed=7)
+    w = torch.from_numpy(rng.choice([0.25, 0.5, -0.75, 1.0], size=(T, K)).astype(np.float32))
+    r = orc.route(idx, E=E, R=R, balanced=balanced)
+    y = _int_bf16(rng, (r.recv_rows, H))
+    g = _int_bf16(rng, (T, H))
+    x = _int_bf16(rng, (T, H))
+    f = orc.bf16_bits_to_f32
+    # <combine(y), g> == <y, combine_backward(g)>
+    cy = f(orc.combine(y, w, r.dest_row, T, K)).astype(np.float64)
+    gy = f(orc.combine_backward(g, w, r.dest_row, r.recv_rows)).astype(np.float64).reshape(r.recv_rows, H)
+    lhs = (cy.reshape(T, H) * g.float().numpy()).sum()
+    rhs = (y.float().numpy() * gy).sum()
+    assert lhs == rhs
+    # <dispatch(x), y> == <x, dispatch_backward(y)>  (dispatch_backward = unweighted combine)
+    dx, _, _, _ = orc.dispatch(x, idx, w, r.dest_row, r.recv_rows)
+    lhs2 = (f(dx).astype(np.float64).reshape(r.recv_rows, H) * y.float().numpy()).sum()
+    rhs2 = (x.float().numpy() * f(orc.combine(y, None, r.dest_row, T, K)).reshape(T, H)).sum()
+    assert lhs2 == rhs2
+
+
+# ------------------------------------------------------------------ replica reduce
+
+def test_replica_reduce_sums_exactly(orc):
+    rng = np.random.default_rng(9)
+    E, R, G = 16, 4, 1000
+    S = E // R
+    rep_exp = np.full((R, S), -1, np.int32)
+    rep_exp[1, 0] = 0
+    rep_exp[2, 0] = 0
+    rep_exp[3, 1] = 5
+    rep_exp[0, 3] = 9  # a rank may hold other ranks' experts in any slot
+    rep = rng.integers(-50, 50, size=(R, S, G)).astype(np.float32)
+    owner = rng.integers(-50, 50, size=(E, G)).astype(np.float32)
+    out = orc.replica_reduce(rep_exp, rep, owner)
+    used = rep_exp >= 0
+    for e in range(E):
+        sl = np.argwhere(rep_exp == e)
+        expect = owner[e] + sum((rep[a, b] for a, b in sl), np.zeros(G, np.float32))
+        np.testing.assert_array_equal(out[e], expect)
+    assert out.sum(dtype=np.float64) == owner.sum(dtype=np.float64) + rep[used].sum(dtype=np.float64)
+
+
+def test_replica_reduce_order_is_slot_ascending(orc):
+    # fp32 rounding makes the order visible: 2^24 + 1 - 1 differs by order
+    E, R, S, G = 2, 2, 1, 1
+    rep_exp = np.array([[-1], [0]], np.int32)
+    rep = np.array([[[0.0]], [[1.0]]], np.float32)
+    owner = np.array([[2.0 ** 24], [0.0]], np.float32)
+    out = orc.replica_reduce(rep_exp, rep, owner)
+    assert out[0, 0] == np.float32(2.0 ** 24)  # 2^24 + 1 rounds to even
+    rep_exp2 = np.array([[0], [0]], np.int32)
+    rep2 = np.array([[[1.0]], [[1.0]]], np.float32)
+    out2 = orc.replica_reduce(rep_exp2, rep2, owner)
+    assert out2[0, 0] == np.float32(2.0 ** 24)  # each +1 is lost in turn: (2^24+1)+1
