@@ -1,0 +1,540 @@
+#!/usr/bin/env python3
+"""Benchmark: MoE expert-parallel dispatch + combine on B200.
+
+One step = one pass of the hot path over one batch: ep_plan (routing
+histogram, scan, layout/plan, stable slots) + ep_dispatch + ep_combine.
+Default workload: HT prefill (T=32768, H=7168, E=256, top-8, R=8 logical ranks,
+FP8 e4m3 dispatch with per-128 scales, bf16 combine with fp32 accumulation),
+seeded synthetic routing. Every buffer is larger than L2 (126 MB), so no L2
+flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Prints ONE JSON line on rank 0. With N > 1 (torchrun), every rank runs its
+own independent EP world (weak scaling, no data-path collective); the time is
+the max over ranks of the device-timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine GB/s and tokens/s on 1 B200; % of HBM roofline vs skew"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ bytes
+
+def algorithmic_bytes(T, H, K, rows_placed, fp8):
+    """Minimum bytes each call must move (per step), by call."""
+    L = T * K
+    plan = 4 * L + 4 * L                                    # topk_idx read, dest_row written
+    payload = rows_placed * H * (1 if fp8 else 2)
+    scales = rows_placed * (H // 128) * 4 if fp8 else 0
+    dispatch = 2 * T * H + payload + scales + 12 * L + 8 * rows_placed  # x, rows, scales, idx+w+dest, recv_w+recv_expert
+    combine = 2 * rows_placed * H + 2 * T * H + 8 * L       # expert rows, out, w + dest
+    return {"plan": plan, "dispatch": dispatch, "combine": combine}
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current source of the kernel's file (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)[kernel]
+        src = os.path.join(ROOT, rec["source"])
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if sha != rec["source_sha"] or rec["workload"] != workload:
+            return None
+        return int(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+
+def dist_setup(gpus: int):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ workloads
+
+# The five workloads of the hot path (synthetic routing from combine_ep_dispatch_03_b200.synth).
+WORKLOADS = {
+    "ht_prefill": dict(T=32768, H=7168, E=256, K=8, R=8, mode="ht", cap=0, fp8=True, balanced=False, s=0.0,
+                       backward=False, G=0),
+    "ll_decode": dict(T=1024, H=7168, E=256, K=8, R=8, mode="ll", cap=1024, fp8=False, balanced=False, s=0.0,
+                      backward=False, G=0),
+    "imbalance": dict(T=32768, H=4096, E=128, K=8, R=8, mode="ht", cap=0, fp8=False, balanced=False, s=0.0,
+                      backward=False, G=0),
+    "large_train": dict(T=131072, H=7168, E=384, K=8, R=16, mode="ht", cap=0, fp8=False, balanced=True, s=1.0,
+                        backward=True, G=7168 * 256),
+    "tiny": dict(T=128, H=1024, E=16, K=2, R=4, mode="ht", cap=0, fp8=False, balanced=False, s=0.0,
+                 backward=False, G=0),
+}
+HT = WORKLOADS["ht_prefill"]
+SWEEP = WORKLOADS["imbalance"]
+
+KERNEL_OF = {"plan": "k_route_*", "combine": "k_combine", "combine_backward": "k_combine_bwd",
+             "dispatch_backward": "k_combine", "replica_reduce": "k_replica_reduce"}
+
+
+class Step:
+    """One pass of the hot path for a workload: buffers, the calls in order,
+    and the algorithmic bytes of each call."""
+
+    def __init__(self, wl: dict, dev, seed: int, host_inputs: bool = True):
+        import torch
+
+        from combine_ep_dispatch_03_b200 import ep, synth
+
+        self.wl = wl
+        T, H, E, K, R = wl["T"], wl["H"], wl["E"], wl["K"], wl["R"]
+        self.T, self.H, self.E, self.K, self.R = T, H, E, K, R
+        x = synth.tokens_bf16(T, H, seed=seed)
+        idx, w = synth.routing(T, E, K, zipf_s=wl["s"], seed=seed)
+        self.x_host = x.pin_memory() if host_inputs else x
+        self.idx_host = idx.pin_memory() if host_inputs else idx
+        self.w_host = w.pin_memory() if host_inputs else w
+        self.xd, self.idxd, self.wd = self.x_host.to(dev), self.idx_host.to(dev), self.w_host.to(dev)
+        h = ep.Ep(T, H, E, K, R, mode=wl["mode"], ll_capacity=wl["cap"], fp8=wl["fp8"], balanced=wl["balanced"],
+                  grad_elems_per_expert=wl["G"])
+        self.h = h
+        self.bufs = h.empty_recv(dev)
+        g = torch.Generator(device=dev).manual_seed(1000 + seed)
+        if wl["backward"]:
+            # identity expert: combine reads the dispatched rows (no second row buffer)
+            self.y = self.bufs["recv_x"]
+        else:
+            # the expert-FFN output stand-in, resident on the device (not timed)
+            self.y = torch.randn((h.recv_rows, H), generator=g, device=dev).to(torch.bfloat16)
+        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.calls = [("plan", lambda st: h.plan(self.idxd, st)),
+                      ("dispatch", lambda st: h.dispatch(self.xd, self.idxd, self.wd, stream=st, **self.bufs)),
+                      ("combine", lambda st: h.combine(self.y, self.wd, self.out, st))]
+        self.outputs = [self.out]
+        if wl["backward"]:
+            self.gout_host = synth.tokens_bf16(T, H, seed=seed + 5)
+            if host_inputs:
+                self.gout_host = self.gout_host.pin_memory()
+            self.gout = self.gout_host.to(dev)
+            self.gy = torch.empty((h.recv_rows, H), dtype=torch.bfloat16, device=dev)
+            self.gx = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+            self.rep = torch.randn((R, h.S, wl["G"]), generator=g, device=dev)
+            self.owner = torch.randn((E, wl["G"]), generator=g, device=dev)
+            self.calls += [
+                ("combine_backward", lambda st: h.combine_backward(self.gout, self.wd, self.gy, st)),
+                ("dispatch_backward", lambda st: h.dispatch_backward(self.gy, self.gx, st)),
+                ("replica_reduce", lambda st: h.reduce_replica_grads(self.rep, self.owner, st)),
+            ]
+            self.outputs.append(self.gx)
+        self.bytes = None
+
+    def run(self, st):
+        for _, f in self.calls:
+            f(st)
+
+    def measure_bytes(self, st):
+        """Algorithmic bytes per call, from the routing of one untimed step."""
+        self.run(st)
+        st.synchronize()  # recv_counts is written on `st`
+        T, H, K, wl = self.T, self.H, self.K, self.wl
+        L = T * K
+        placed = int(self.bufs["recv_counts"].sum().item())
+        b = algorithmic_bytes(T, H, K, placed, wl["fp8"])
+        if wl["backward"]:
+            b["combine_backward"] = 2 * T * H + 2 * placed * H + 8 * L
+            b["dispatch_backward"] = 2 * placed * H + 2 * T * H + 4 * L
+            rep, _ = self.h.get_plan(st)
+            used = [e for e in rep if e >= 0]
+            b["replica_reduce"] = 4 * wl["G"] * (len(used) + 2 * len(set(used)))
+        self.bytes = b
+        self.placed = placed
+        return b
+
+    def launches(self):
+        from combine_ep_dispatch_03_b200.ep import plan_launches
+
+        return plan_launches(self.h) + len(self.calls) - 1
+
+
+def timed(step: Step, steps, warmup, stream):
+    """Warm-up, then `steps` steps with CUDA events between the calls on the
+    launching stream. Returns (total_ms, {call: [ms per step]})."""
+    import torch
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step.run(stream)
+    torch.cuda.synchronize()
+    n = len(step.calls)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for s in range(steps):
+            ev[s][0].record(stream)
+            for i, (_, f) in enumerate(step.calls):
+                f(stream)
+                ev[s][i + 1].record(stream)
+        end.record(stream)
+    torch.cuda.synchronize()
+    per = {name: [e[i].elapsed_time(e[i + 1]) for e in ev] for i, (name, _) in enumerate(step.calls)}
+    return start.elapsed_time(end), per
+
+
+def run_native(args):
+    import torch
+
+    from combine_ep_dispatch_03_b200 import build, ep
+
+    rank, world, local = dist_setup(args.gpus)
+    if rank == 0 or local == 0:
+        build.build()
+    barrier(world)
+    ep.lib()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    stream = torch.cuda.Stream(device=dev)
+    wl = dict(WORKLOADS[args.workload])
+    if args.tokens:
+        wl["T"] = args.tokens
+    if args.zipf is not None:
+        wl["s"] = args.zipf
+    if args.balanced is not None:
+        wl["balanced"] = bool(args.balanced)
+    name = args.workload if wl == WORKLOADS[args.workload] else args.workload + "_custom"
+    seed = rank  # each rank: its own EP world (weak scaling)
+    step = Step(wl, dev, seed)
+    nbytes = step.measure_bytes(stream)
+    step_bytes = sum(nbytes.values())
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    total_ms, per = timed(step, args.steps, args.warmup, stream)
+    clocks = sampler.stop()
+    barrier(world)
+    ms_step = max_over_ranks(total_ms / args.steps, world)
+    flags = step.h.status(stream)
+
+    avg = {k: sum(v) / len(v) for k, v in per.items()}
+    peak, peak_kind = hbm_peak()
+    dom = max((k for k in avg if k != "plan"), key=lambda k: avg[k])
+    kname = KERNEL_OF.get(dom) or ("k_dispatch_fp8" if wl["fp8"] else "k_dispatch_bf16")
+    achieved = nbytes[dom] / (avg[dom] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "call": dom, "kernel": kname, "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy)",
+                "traffic": committed_traffic(kname, name), "algorithmic_bytes_per_launch": nbytes[dom]}
+
+    e2e = None if args.no_e2e else run_e2e(step, dev, stream, max(3, min(args.steps, 20)), world, step_bytes)
+    big = step.h.recv_rows * step.H * (1 if wl["fp8"] else 2)
+    result = {
+        "metric": METRIC, "value": round(world * step_bytes / (ms_step * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": name, "T": wl["T"], "H": wl["H"], "E": wl["E"], "topk": wl["K"],
+                   "logical_ranks": wl["R"], "layout": wl["mode"], "ll_capacity": wl["cap"],
+                   "balanced_plan": wl["balanced"], "zipf_s": wl["s"], "backward": wl["backward"],
+                   "payload": ("bf16 x -> fp8 e4m3 dispatch (per-128 fp32 scales)" if wl["fp8"]
+                               else "bf16 dispatch") + " -> bf16 combine (fp32 accumulation)",
+                   "l2": ("no flush: the receive buffer (%.2f GB) and the expert rows exceed L2 (126 MB)"
+                          % (big / 1e9)) if big > 2 * 126e6 else "working set partly L2-resident, no flush",
+                   "parallelism": f"{world} independent EP worlds (one per GPU), R logical ranks each"},
+        "tokens_per_s": round(world * wl["T"] / (ms_step * 1e-3), 1),
+        "rows_per_s": round(world * step.placed / (ms_step * 1e-3), 1),
+        "frac_of_hbm": round(step_bytes / (ms_step * 1e-3) / 1e9 / peak, 4),
+        "frac_of_8tbs_nominal": round(step_bytes / (ms_step * 1e-3) / 1e9 / 8000.0, 4),
+        "per_call_us": {k: round(v * 1e3, 2) for k, v in avg.items()},
+        "per_call_gbs": {k: round(nbytes[k] / (avg[k] * 1e-3) / 1e9, 1) for k in avg},
+        "bytes_per_step": step_bytes,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": step.launches() * args.steps,
+        "clocks": clocks,
+        "device_flags": flags,
+    }
+    if wl["balanced"] or wl["mode"] == "ht":
+        load = step.h.tensor(ep.T_RANK_LOAD).cpu().tolist()
+        result["rank_load_max_over_mean"] = round(max(load) / (sum(load) / len(load)), 4) if sum(load) else None
+    step.h.close()
+    del step
+    torch.cuda.empty_cache()
+    if not args.no_sweep and args.workload == "ht_prefill":
+        result["skew_sweep"] = run_sweep(dev, stream, seed, peak)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline and args.workload == "ht_prefill":
+        result["cpu_baseline"] = cpu_baseline(args.cpu_sample_tokens)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def run_e2e(step: Step, dev, stream, steps, world, step_bytes):
+    """The same step through the public API, its inputs copied from pinned
+    host memory and its results (combined tokens, and the input gradient with
+    a backward pass) read back to pinned host memory, inside the timed region."""
+    import torch
+
+    ins = [(step.x_host, step.xd), (step.idx_host, step.idxd), (step.w_host, step.wd)]
+    if step.wl["backward"]:
+        ins.append((step.gout_host, step.gout))
+    outs = [(o, torch.empty(o.shape, dtype=o.dtype).pin_memory()) for o in step.outputs]
+
+    def one():
+        for src, dst in ins:
+            dst.copy_(src, non_blocking=True)
+        step.run(stream)
+        for src, dst in outs:
+            dst.copy_(src, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            one()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(steps):
+            one()
+        e.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world)
+    h2d = sum(src.numel() * src.element_size() for src, _ in ins)
+    d2h = sum(src.numel() * src.element_size() for src, _ in outs)
+    return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": steps}
+
+
+def run_sweep(dev, stream, seed, peak, steps=10, warmup=3):
+    """Imbalance sweep: T=32768, H=4096, E=128, top-8, R=8, Zipf s, plan off/on."""
+    import torch
+
+    from combine_ep_dispatch_03_b200 import ep
+
+    rows = []
+    for balanced in (False, True):
+        for s in (0.0, 0.5, 1.0, 1.5):
+            wl = dict(SWEEP, s=s, balanced=balanced)
+            step = Step(wl, dev, seed + 11, host_inputs=False)
+            nb = step.measure_bytes(stream)
+            total, per = timed(step, steps, warmup, stream)
+            ms = total / steps
+            load = step.h.tensor(ep.T_RANK_LOAD).cpu().tolist()
+            mean = sum(load) / len(load)
+            gbs = sum(nb.values()) / (ms * 1e-3) / 1e9
+            rows.append({"zipf_s": s, "balanced": balanced, "ms": round(ms, 4), "gbs": round(gbs, 1),
+                         "frac": round(gbs / peak, 4), "load_max_over_mean": round(max(load) / mean, 4),
+                         "plan_us": round(1e3 * sum(per["plan"]) / steps, 2), "flags": step.h.status(stream)})
+            step.h.close()
+            del step
+            torch.cuda.empty_cache()
+    return rows
+
+
+def cpu_baseline(sample_tokens: int):
+    """The oracle as it stands, single-threaded on a host core, on a bounded
+    sample of the HT prefill workload: full routing of all 32768 tokens, then
+    FP8 dispatch and combine of `sample_tokens` tokens in chunks of 2048."""
+    import numpy as np
+
+    import oracle
+    from combine_ep_dispatch_03_b200 import synth
+
+    oracle.build()
+    T, H, E, K, R = HT["T"], HT["H"], HT["E"], HT["K"], HT["R"]
+    idx, w = synth.routing(T, E, K, seed=0)
+    n = min(sample_tokens, T)
+    x = synth.tokens_bf16(n, H, seed=0)
+    chunk = 2048
+    y = synth.tokens_bf16(chunk * K, H, seed=1)
+    dest = np.arange(chunk * K, dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.route(idx, E=E, R=R)
+    moved = 8 * T * K
+    for c0 in range(0, n, chunk):
+        c1 = min(n, c0 + chunk)
+        m = c1 - c0
+        oracle.dispatch(x[c0:c1], idx[c0:c1], w[c0:c1], dest[: m * K], m * K, fp8=True)
+        oracle.combine(y, w[c0:c1], dest[: m * K], m, K)
+        b = algorithmic_bytes(m, H, K, m * K, True)
+        moved += b["dispatch"] + b["combine"]
+    dt = time.perf_counter() - t0
+    return {"value": round(moved / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"ht_prefill: routing of all {T} tokens + FP8 dispatch and combine of {n} tokens"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: rank 0 only, each step a bounded
+    sample (1024 tokens) of the HT prefill workload on one host core."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from combine_ep_dispatch_03_b200 import synth
+
+    oracle.build()
+    T, H, E, K, R = HT["T"], HT["H"], HT["E"], HT["K"], HT["R"]
+    n = 1024
+    idx, w = synth.routing(T, E, K, seed=0)
+    x = synth.tokens_bf16(n, H, seed=0)
+    y = synth.tokens_bf16(n * K, H, seed=1)
+    dest = np.arange(n * K, dtype=np.int32)
+    sub_idx, sub_w = idx[:n], w[:n]
+
+    def one():
+        oracle.route(sub_idx, E=E, R=R)
+        oracle.dispatch(x, sub_idx, sub_w, dest, n * K, fp8=True)
+        oracle.combine(y, sub_w, dest, n, K)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = (time.perf_counter() - t0) / args.steps
+    b = algorithmic_bytes(n, H, K, n * K, True)
+    gbs = sum(b.values()) / dt / 1e9
+    sample = f"ht_prefill: route + FP8 dispatch + combine of {n} of {T} tokens per step"
+    print(json.dumps({
+        "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
+        "config": {"workload": workload, "T": T, "H": H, "E": E, "topk": K, "logical_ranks": R},
+        "tokens_per_s": round(n / dt, 1),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="ht_prefill")
+    ap.add_argument("--tokens", type=int, default=0, help="override T (smaller cases for profiling)")
+    ap.add_argument("--zipf", type=float, default=None, help="override the router's Zipf bias s")
+    ap.add_argument("--balanced", type=int, choices=[0, 1], default=None, help="override the balanced plan")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=24576)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,435 @@
+// data.cu -- the HBM-bound row movers: dispatch (bf16 copy or fused FP8
+// cast), combine (gather + fp32 weighted reduce), their backward twins, and
+// the replica-gradient reduce.
+//
+// NCCL EP paper (arXiv 2603.13606): dispatch(x, topk_i, topk_w, handle) ->
+// recv_x, recv_i, recv_w (Table V); FP8 quantization scales as a tensor role
+// (Table IV); combine gathers expert outputs and reduces them to the original
+// token order (Table II), per token at the receiver (Table III); the backward
+// pass reuses the forward routing state (Fig. 5). MoonEP article, para. 5:
+// gradients of duplicated experts pass through a reduce buffer and are added
+// into the owner's gradients.
+//
+// Every kernel is a streaming row mover: one CTA per token row, 16-byte
+// vector loads/stores, each input row read once and each output row written
+// once, so the bytes moved are the algorithmic bytes.
+#include <cuda_bf16.h>
+
+#include "ep_internal.cuh"
+
+namespace epb {
+namespace {
+
+__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x);
+    f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z);
+    f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+
+// round-to-nearest-even to bf16, two at a time (lo -> low half)
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint4 pack8(const float *f) {
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                      pack_bf16x2(f[6], f[7]));
+}
+
+// e4m3 with round-to-nearest-even and saturation to +-448; `lo` lands in the
+// low byte (the element at the lower address).
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ void stage_routing(const int32_t *__restrict__ dest_row, const float *__restrict__ w,
+                                              int64_t pb, int K, int *s_dest, float *s_w) {
+    if (threadIdx.x < K) {
+        s_dest[threadIdx.x] = dest_row[pb + threadIdx.x];
+        if (s_w) s_w[threadIdx.x] = w ? w[pb + threadIdx.x] : 1.0f;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// dispatch, bf16 payload: recv[dest_row[t,k]] = x[t]
+// ---------------------------------------------------------------------------
+template <int VPT>
+__global__ void __launch_bounds__(256) k_dispatch_bf16(const uint4 *__restrict__ x, const int32_t *__restrict__ idx,
+                                                       const float *__restrict__ w,
+                                                       const int32_t *__restrict__ dest_row, int K, int nvec,
+                                                       uint4 *__restrict__ recv, float *__restrict__ recv_w,
+                                                       int32_t *__restrict__ recv_expert,
+                                                       const int32_t *__restrict__ counts_src,
+                                                       int32_t *__restrict__ counts_dst, int counts_len) {
+    __shared__ int s_dest[kMaxTopk];
+    const int t = blockIdx.x;
+    const int64_t pb = (int64_t)t * K;
+    if (threadIdx.x < K) {
+        const int dr = dest_row[pb + threadIdx.x];
+        s_dest[threadIdx.x] = dr;
+        if (dr >= 0) {
+            if (recv_w) recv_w[dr] = w[pb + threadIdx.x];
+            if (recv_expert) recv_expert[dr] = idx[pb + threadIdx.x];
+        }
+    }
+    if (t == 0 && counts_dst)
+        for (int i = threadIdx.x; i < counts_len; i += blockDim.x) counts_dst[i] = counts_src[i];
+    const uint4 *src = x + (int64_t)t * nvec;
+    const int step = VPT * blockDim.x;
+    for (int c0 = 0; c0 < nvec; c0 += step) {
+        uint4 v[VPT];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int c = c0 + threadIdx.x + i * blockDim.x;
+            if (c < nvec) v[i] = __ldcs(src + c);
+        }
+        if (c0 == 0) __syncthreads();
+        for (int k = 0; k < K; ++k) {
+            const int dr = s_dest[k];
+            if (dr < 0) continue;
+            uint4 *dst = recv + (int64_t)dr * nvec;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int c = c0 + threadIdx.x + i * blockDim.x;
+                if (c < nvec) __stcs(dst + c, v[i]);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// dispatch, FP8 payload: per 128-element block b of x[t],
+//   s_b = amax_b / 448, q = e4m3(x / s_b), all-zero block -> s = 0, q = +0.
+// The cast is done once per token and its result stored K times.
+// One thread owns 16 consecutive elements (two 16-byte loads, one 16-byte
+// store); the 8 threads of a 128-block are 8 consecutive lanes.
+// ---------------------------------------------------------------------------
+template <int CPT>
+__global__ void __launch_bounds__(256) k_dispatch_fp8(const uint4 *__restrict__ x, const int32_t *__restrict__ idx,
+                                                      const float *__restrict__ w,
+                                                      const int32_t *__restrict__ dest_row, int K, int nchunk,
+                                                      uint4 *__restrict__ recv, float *__restrict__ scales,
+                                                      float *__restrict__ recv_w, int32_t *__restrict__ recv_expert,
+                                                      const int32_t *__restrict__ counts_src,
+                                                      int32_t *__restrict__ counts_dst, int counts_len) {
+    __shared__ int s_dest[kMaxTopk];
+    const int t = blockIdx.x;
+    const int64_t pb = (int64_t)t * K;
+    const int nb = nchunk >> 3; // 128-element blocks per row
+    if (threadIdx.x < K) {
+        const int dr = dest_row[pb + threadIdx.x];
+        s_dest[threadIdx.x] = dr;
+        if (dr >= 0) {
+            if (recv_w) recv_w[dr] = w[pb + threadIdx.x];
+            if (recv_expert) recv_expert[dr] = idx[pb + threadIdx.x];
+        }
+    }
+    if (t == 0 && counts_dst)
+        for (int i = threadIdx.x; i < counts_len; i += blockDim.x) counts_dst[i] = counts_src[i];
+    const uint4 *src = x + (int64_t)t * 2 * nchunk;
+    const int step = CPT * blockDim.x;
+    for (int c0 = 0; c0 < nchunk; c0 += step) {
+        uint4 a[CPT], b[CPT];
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = c0 + threadIdx.x + i * blockDim.x;
+            if (c < nchunk) {
+                a[i] = __ldcs(src + 2 * c);
+                b[i] = __ldcs(src + 2 * c + 1);
+            } else {
+                a[i] = make_uint4(0, 0, 0, 0);
+                b[i] = a[i];
+            }
+        }
+        uint4 q[CPT];
+        float sc[CPT];
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            float f[16];
+            unpack8(a[i], f);
+            unpack8(b[i], f + 8);
+            float amax = 0.0f;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) amax = fmaxf(amax, fabsf(f[u]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+            const float s = __fdiv_rn(amax, 448.0f);
+            sc[i] = s;
+            uint32_t wd[4] = {0u, 0u, 0u, 0u};
+            if (amax != 0.0f) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t lo = e4m3x2(__fdiv_rn(f[4 * u], s), __fdiv_rn(f[4 * u + 1], s));
+                    const uint32_t hi = e4m3x2(__fdiv_rn(f[4 * u + 2], s), __fdiv_rn(f[4 * u + 3], s));
+                    wd[u] = lo | (hi << 16);
+                }
+            }
+            q[i] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        }
+        if (c0 == 0) __syncthreads();
+        for (int k = 0; k < K; ++k) {
+            const int dr = s_dest[k];
+            if (dr < 0) continue;
+            uint4 *dst = recv + (int64_t)dr * nchunk;
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) {
+                const int c = c0 + threadIdx.x + i * blockDim.x;
+                if (c < nchunk) {
+                    __stcs(dst + c, q[i]);
+                    if ((c & 7) == 0) scales[(int64_t)dr * nb + (c >> 3)] = sc[i];
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// combine: out[t] = bf16(fold_k fmaf(w[t,k], y[dest_row[t,k]], acc)), k in
+// order, acc from +0; UNIT: unweighted fp32 sum (dispatch backward).
+// ---------------------------------------------------------------------------
+template <int CPT, bool UNIT>
+__global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, const float *__restrict__ w,
+                                                 const int32_t *__restrict__ dest_row, int K, int nvec,
+                                                 uint4 *__restrict__ out) {
+    __shared__ int s_dest[kMaxTopk];
+    __shared__ float s_w[kMaxTopk];
+    const int t = blockIdx.x;
+    stage_routing(dest_row, w, (int64_t)t * K, K, s_dest, s_w);
+    __syncthreads();
+    const int step = CPT * blockDim.x;
+    for (int c0 = 0; c0 < nvec; c0 += step) {
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = c0 + threadIdx.x + i * blockDim.x;
+            if (c >= nvec) continue;
+            float acc[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
+            for (int k0 = 0; k0 < K; k0 += 8) {
+                uint4 v[8];
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const int k = k0 + kk;
+                    const int dr = k < K ? s_dest[k] : -1;
+                    v[kk] = dr >= 0 ? __ldcs(y + (int64_t)dr * nvec + c) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const int k = k0 + kk;
+                    if (k >= K || s_dest[k] < 0) continue;
+                    float f[8];
+                    unpack8(v[kk], f);
+                    if (UNIT) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) acc[u] = __fadd_rn(acc[u], f[u]);
+                    } else {
+                        const float wk = s_w[k];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) acc[u] = __fmaf_rn(wk, f[u], acc[u]);
+                    }
+                }
+            }
+            __stcs(out + (int64_t)t * nvec + c, pack8(acc));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// combine backward: gy[dest_row[t,k]] = bf16(w[t,k] * g[t]) (fp32 product)
+// ---------------------------------------------------------------------------
+template <int VPT>
+__global__ void __launch_bounds__(256) k_combine_bwd(const uint4 *__restrict__ g, const float *__restrict__ w,
+                                                     const int32_t *__restrict__ dest_row, int K, int nvec,
+                                                     uint4 *__restrict__ gy) {
+    __shared__ int s_dest[kMaxTopk];
+    __shared__ float s_w[kMaxTopk];
+    const int t = blockIdx.x;
+    stage_routing(dest_row, w, (int64_t)t * K, K, s_dest, s_w);
+    const uint4 *src = g + (int64_t)t * nvec;
+    const int step = VPT * blockDim.x;
+    for (int c0 = 0; c0 < nvec; c0 += step) {
+        uint4 v[VPT];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int c = c0 + threadIdx.x + i * blockDim.x;
+            if (c < nvec) v[i] = __ldcs(src + c);
+        }
+        if (c0 == 0) __syncthreads();
+        for (int k = 0; k < K; ++k) {
+            const int dr = s_dest[k];
+            if (dr < 0) continue;
+            const float wk = s_w[k];
+            uint4 *dst = gy + (int64_t)dr * nvec;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int c = c0 + threadIdx.x + i * blockDim.x;
+                if (c >= nvec) continue;
+                float f[8];
+                unpack8(v[i], f);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) f[u] = __fmul_rn(wk, f[u]);
+                __stcs(dst + c, pack8(f));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// replica-gradient reduce: owner[e] += rep[slot] for the slots holding e,
+// ascending slot order, fp32. Persistent grid over (expert, chunk) items.
+// ---------------------------------------------------------------------------
+constexpr int kRedThreads = 256, kRedUnroll = 4;
+
+__global__ void __launch_bounds__(kRedThreads) k_replica_reduce(const float4 *__restrict__ rep,
+                                                                float4 *__restrict__ owner,
+                                                                const int32_t *__restrict__ red_experts,
+                                                                const int32_t *__restrict__ red_count,
+                                                                const int32_t *__restrict__ red_list,
+                                                                const int32_t *__restrict__ red_n, int R,
+                                                                int64_t G4) {
+    const int nred = *red_count;
+    const int64_t chunk = (int64_t)kRedThreads * kRedUnroll;
+    const int64_t per = (G4 + chunk - 1) / chunk;
+    const int64_t items = (int64_t)nred * per;
+    for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+        const int e = red_experts[it / per];
+        const int64_t base = (it % per) * chunk + threadIdx.x;
+        const int n = red_n[e];
+        const int32_t *lst = red_list + (int64_t)e * R;
+        float4 *o = owner + (int64_t)e * G4;
+        float4 acc[kRedUnroll];
+#pragma unroll
+        for (int u = 0; u < kRedUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kRedThreads;
+            acc[u] = i < G4 ? o[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int a = 0; a < n; ++a) {
+            const float4 *r = rep + (int64_t)lst[a] * G4;
+#pragma unroll
+            for (int u = 0; u < kRedUnroll; ++u) {
+                const int64_t i = base + (int64_t)u * kRedThreads;
+                if (i < G4) {
+                    const float4 v = __ldcs(r + i);
+                    acc[u].x = __fadd_rn(acc[u].x, v.x);
+                    acc[u].y = __fadd_rn(acc[u].y, v.y);
+                    acc[u].z = __fadd_rn(acc[u].z, v.z);
+                    acc[u].w = __fadd_rn(acc[u].w, v.w);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kRedUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kRedThreads;
+            if (i < G4) o[i] = acc[u];
+        }
+    }
+}
+
+// vectors per thread and threads per CTA for a row of `n` 16-byte vectors
+void pick_shape(int n, int *per_thread, int *threads) {
+    for (int v = 1; v <= 8; v <<= 1) {
+        const int th = ((n + v - 1) / v + 31) / 32 * 32;
+        if (th <= 256) {
+            *per_thread = v;
+            *threads = th < 32 ? 32 : th;
+            return;
+        }
+    }
+    *per_thread = 8;
+    *threads = 256; // rows longer than 2048 vectors loop over slabs
+}
+
+#define EPB_SWITCH_VPT(v, KERNEL, ...)                                                                               \
+    switch (v) {                                                                                                     \
+    case 1: KERNEL<1><<<grid, threads, 0, st>>>(__VA_ARGS__); break;                                                 \
+    case 2: KERNEL<2><<<grid, threads, 0, st>>>(__VA_ARGS__); break;                                                 \
+    case 4: KERNEL<4><<<grid, threads, 0, st>>>(__VA_ARGS__); break;                                                 \
+    default: KERNEL<8><<<grid, threads, 0, st>>>(__VA_ARGS__); break;                                                \
+    }
+
+} // namespace
+
+cudaError_t launch_dispatch(const Dims &d, const Workspace &ws, const void *x, const int32_t *topk_idx,
+                            const float *topk_w, void *recv_x, float *recv_scales, float *recv_w,
+                            int32_t *recv_expert, int32_t *recv_counts, cudaStream_t st) {
+    if (d.T == 0) {
+        if (recv_counts)
+            return cudaMemcpyAsync(recv_counts, ws.recv_counts, sizeof(int32_t) * d.counts_len,
+                                   cudaMemcpyDeviceToDevice, st);
+        return cudaSuccess;
+    }
+    const dim3 grid(d.T);
+    int per, threads;
+    if (d.fp8) {
+        const int nchunk = d.H / 16;
+        pick_shape(nchunk, &per, &threads);
+        EPB_SWITCH_VPT(per, k_dispatch_fp8, (const uint4 *)x, topk_idx, topk_w, ws.dest_row, d.K, nchunk,
+                       (uint4 *)recv_x, recv_scales, recv_w, recv_expert, ws.recv_counts, recv_counts,
+                       d.counts_len);
+    } else {
+        const int nvec = d.H / 8;
+        pick_shape(nvec, &per, &threads);
+        EPB_SWITCH_VPT(per, k_dispatch_bf16, (const uint4 *)x, topk_idx, topk_w, ws.dest_row, d.K, nvec,
+                       (uint4 *)recv_x, recv_w, recv_expert, ws.recv_counts, recv_counts, d.counts_len);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine_backward(const Dims &d, const Workspace &ws, const void *grad_out, const float *topk_w,
+                                    void *grad_expert_out, cudaStream_t st) {
+    if (d.T == 0) return cudaSuccess;
+    const dim3 grid(d.T);
+    const int nvec = d.H / 8;
+    int per, threads;
+    pick_shape(nvec, &per, &threads);
+    EPB_SWITCH_VPT(per, k_combine_bwd, (const uint4 *)grad_out, topk_w, ws.dest_row, d.K, nvec,
+                   (uint4 *)grad_expert_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const Dims &d, const Workspace &ws, const void *y, const float *topk_w, void *out,
+                           cudaStream_t st) {
+    if (d.T == 0) return cudaSuccess;
+    const dim3 grid(d.T);
+    const int nvec = d.H / 8;
+    int per, threads;
+    pick_shape(nvec, &per, &threads);
+    const uint4 *yy = (const uint4 *)y;
+    uint4 *oo = (uint4 *)out;
+    if (topk_w) {
+        switch (per) {
+        case 1: k_combine<1, false><<<grid, threads, 0, st>>>(yy, topk_w, ws.dest_row, d.K, nvec, oo); break;
+        case 2: k_combine<2, false><<<grid, threads, 0, st>>>(yy, topk_w, ws.dest_row, d.K, nvec, oo); break;
+        case 4: k_combine<4, false><<<grid, threads, 0, st>>>(yy, topk_w, ws.dest_row, d.K, nvec, oo); break;
+        default: k_combine<8, false><<<grid, threads, 0, st>>>(yy, topk_w, ws.dest_row, d.K, nvec, oo); break;
+        }
+    } else {
+        switch (per) {
+        case 1: k_combine<1, true><<<grid, threads, 0, st>>>(yy, nullptr, ws.dest_row, d.K, nvec, oo); break;
+        case 2: k_combine<2, true><<<grid, threads, 0, st>>>(yy, nullptr, ws.dest_row, d.K, nvec, oo); break;
+        case 4: k_combine<4, true><<<grid, threads, 0, st>>>(yy, nullptr, ws.dest_row, d.K, nvec, oo); break;
+        default: k_combine<8, true><<<grid, threads, 0, st>>>(yy, nullptr, ws.dest_row, d.K, nvec, oo); break;
+        }
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_replica_reduce(const Dims &d, const Workspace &ws, const float *rep, float *owner,
+                                  cudaStream_t st) {
+    const int64_t G4 = d.G / 4;
+    if (G4 == 0) return cudaSuccess;
+    const int grid = num_sms() * 8;
+    k_replica_reduce<<<grid, kRedThreads, 0, st>>>((const float4 *)rep, (float4 *)owner, ws.red_experts,
+                                                   ws.red_count, ws.red_list, ws.red_n, d.R, G4);
+    return cudaGetLastError();
+}
+
+} // namespace epb

@@ -1,0 +1,109 @@
+// ep_internal.cuh -- handle layout and kernel launchers shared by the .cu
+// files of libep_b200 (not part of the public ABI; see include/ep.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep.h"
+
+namespace epb {
+
+// Routing: each warp of the histogram kernel owns a "warp tile" of
+// consecutive (token, k) pairs; tiles grow with the batch so that there are
+// at most about kMaxTiles of them.
+constexpr int kMinTilePairs = 128;
+constexpr int kMaxTilePairs = 2048;
+constexpr int kMaxTiles = 1024;
+constexpr int kRouteThreads = 256;
+constexpr int kAssignPer = 4;             // pairs per thread of the assignment kernel
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kPlanThreads = 1024;
+constexpr int kMaxExperts = 4096;
+constexpr int kMaxTopk = 32;
+constexpr int kMaxRouteSmem = 200 * 1024; // dynamic shared memory cap of the routing kernels
+constexpr int kSmallMaxPairs = 1024;      // single-CTA routing up to this many pairs ...
+constexpr int kSmallMaxExperts = 512;     // ... and experts (plain layouts only)
+
+// Device workspace of a handle: the routing state one ep_plan builds and the
+// later calls of the same forward/backward pass read.
+struct Workspace {
+    int32_t *dest_row;       // [T*K]: receive-buffer row of each pair, -1 if none
+    int32_t *packed;         // [T*K]: expert | rank-in-tile << 16, 0xffff if not routed
+    int32_t *blk;            // [ntiles][E]: per-tile counts, then per-tile bases
+    uint32_t *tile_flags;    // [nhist]: status bits seen by each histogram CTA
+    int32_t *cnt;            // [E]
+    int32_t *recv_counts;    // [R*(g+S)] (HT) or [E] (LL)
+    int32_t *rank_load;      // [R]
+    int32_t *rank_off;       // [R+1]
+    int32_t *replica_expert; // [max(R*S,1)]
+    int32_t *base0;          // [E]: row of stable index 0 of each expert (piece 0)
+    int32_t *len0;           // [E]: stable indices [0, len0) live in piece 0
+    int32_t *xoff;           // [E+1]: extra pieces of expert e: [xoff[e], xoff[e+1])
+    int32_t *xstart;         // [nx_max]: first stable index of an extra piece
+    int32_t *xlen;           // [nx_max]
+    int32_t *xdst;           // [nx_max]: row of the extra piece's first index
+    int32_t *piece_start;    // [E][P]: planner scratch, pieces in creation order
+    int32_t *piece_len;      // [E][P]
+    int32_t *piece_rank;     // [E][P]: rank holding the piece
+    int32_t *piece_slot;     // [E][P]: replica slot, -2 owner tail
+    int32_t *red_list;       // [E][R]: slots (r*S+s) holding e, ascending
+    int32_t *red_n;          // [E]
+    int32_t *red_experts;    // [E]: experts with at least one replica
+    int32_t *red_count;      // [1]
+    uint32_t *flags;         // [1]: EP_FLAG_* bits of the last plan
+    unsigned long long *ticket; // [1]: CTAs of the scan kernel that have finished
+};
+
+struct Dims {
+    int T, H, E, K, R, g, S; // S = replica slots per rank (0 without a plan)
+    int mode, cap, fp8, balanced;
+    int64_t L;               // T*K pairs
+    int64_t rows;            // receive-buffer rows
+    int64_t G;               // replica-gradient elements per expert
+    int wt;                  // pairs per warp tile (a multiple of 32)
+    int ntiles, nhist;       // warp tiles, histogram CTAs
+    int nassign;             // CTAs of the slot-assignment kernel
+    int P;                   // planner scratch pieces per expert (R+1 with a plan)
+    int nx_max;              // bound on extra pieces (R*S + E with a plan, else 0)
+    int counts_len;          // recv_counts entries
+};
+
+// Sizes derived from a validated configuration; also used by the host-only
+// queries, so it allocates nothing.
+ep_status_t derive_dims(const ep_config_t *cfg, Dims *d);
+size_t workspace_bytes(const Dims &d);
+void carve_workspace(const Dims &d, void *base, Workspace *ws);
+
+// shared-memory needs of the routing kernels (host side, for validation)
+size_t route_smem_layout(const Dims &d);
+size_t route_smem_assign(const Dims &d);
+size_t route_smem_hist(const Dims &d);
+size_t route_smem_small(const Dims &d);
+bool route_use_small(const Dims &d);
+int plan_launches(const Dims &d);
+
+// ---- launchers (each returns the launch's cudaError_t) ----
+cudaError_t launch_plan(const Dims &d, const Workspace &ws, const int32_t *topk_idx, cudaStream_t st);
+cudaError_t launch_dispatch(const Dims &d, const Workspace &ws, const void *x, const int32_t *topk_idx,
+                            const float *topk_w, void *recv_x, float *recv_scales, float *recv_w,
+                            int32_t *recv_expert, int32_t *recv_counts, cudaStream_t st);
+cudaError_t launch_combine_backward(const Dims &d, const Workspace &ws, const void *grad_out, const float *topk_w,
+                                    void *grad_expert_out, cudaStream_t st);
+cudaError_t launch_combine(const Dims &d, const Workspace &ws, const void *y, const float *topk_w, void *out,
+                           cudaStream_t st);
+cudaError_t launch_replica_reduce(const Dims &d, const Workspace &ws, const float *rep, float *owner,
+                                  cudaStream_t st);
+
+int num_sms();
+
+} // namespace epb
+
+struct ep_handle {
+    ep_config_t cfg;
+    epb::Dims d;
+    epb::Workspace ws;
+    void *base;
+    int device;
+    int planned;
+};

@@ -1,0 +1,704 @@
+// route.cu -- routing for one forward pass: per-expert counts, stable slots,
+// the HT / LL layouts and the balanced-replica plan.
+//
+// NCCL EP paper (arXiv 2603.13606), Table III: HT output is "2D with token
+// counts", LL output is "3D expert-major". MoonEP article, paras. 3-5: rows go
+// straight to expert-grouped rank positions; a GPU planner replicates hot
+// experts into at most E/R prefetch slots per rank so that every rank gets a
+// predictable row count.
+//
+// Results are deterministic: positions come from counts and scans, never from
+// the order in which atomics land.
+//
+// Large batches, three kernels:
+//   k_route_hist    per warp tile of consecutive pairs: validate ids, give
+//                   each pair its rank among the tile's pairs of the same
+//                   expert (match_any), count the tile's pairs per expert
+//   k_route_scan    per expert: exclusive scan of the tile counts over tiles;
+//                   with a balanced plan, the CTA that finishes last (a
+//                   ticket counter, no waiting) builds the plan
+//   k_route_assign  per pair: stable index j = tile base + rank in tile ->
+//                   destination row through the layout tables (each CTA
+//                   computes the plain layouts' expert offsets itself)
+// Small batches without a plan, one kernel:
+//   k_route_small   one CTA does all of the above in shared memory
+#include "ep_internal.cuh"
+
+namespace epb {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallWarps = kSmallThreads / 32;
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// A pair is routed iff its id is in [0, E) and no earlier choice of the same
+// token picked that id. -1 is a masked choice (no flag). s_ids starts at a
+// token boundary, so the earlier choices of pair p are s_ids[p-k .. p-1].
+__device__ __forceinline__ int classify(const int32_t *s_ids, int p, int k, int E, uint32_t &fl) {
+    const int e = s_ids[p];
+    if (e == -1) return -1;
+    if (e < 0 || e >= E) {
+        fl |= EP_FLAG_BAD_EXPERT_ID;
+        return -1;
+    }
+    for (int k2 = 1; k2 <= k; ++k2) {
+        if (s_ids[p - k2] == e) {
+            fl |= EP_FLAG_DUP_EXPERT_ID;
+            return -1;
+        }
+    }
+    return e;
+}
+
+__device__ __forceinline__ void load_ids(const int32_t *__restrict__ idx, int64_t p0, int np, int32_t *s_ids) {
+    for (int i = threadIdx.x; i < np; i += blockDim.x) s_ids[i] = __ldg(idx + p0 + i);
+}
+
+__device__ __forceinline__ uint32_t block_or(uint32_t v, uint32_t *s_acc) {
+    v = __reduce_or_sync(kFull, v);
+    if ((threadIdx.x & 31) == 0 && v) atomicOr(s_acc, v);
+    return v;
+}
+
+// Exclusive scan of a[0..n) in shared memory by the whole block; returns the
+// total. s_warp needs 33 ints. Every thread of the block must call it.
+__device__ int block_exscan(int32_t *a, int n, int32_t *s_warp) {
+    const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, w = tid >> 5;
+    const int per = (n + nth - 1) / nth;
+    const int lo = min(n, tid * per), hi = min(n, lo + per);
+    int sum = 0;
+    for (int i = lo; i < hi; ++i) sum += a[i];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        const int nw = nth >> 5;
+        const int v = lane < nw ? s_warp[lane] : 0;
+        int inc = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(kFull, inc, o);
+            if (lane >= o) inc += u;
+        }
+        if (lane < nw) s_warp[lane] = inc - v;
+        if (lane == 31) s_warp[32] = inc;
+    }
+    __syncthreads();
+    int run = s_warp[w] + incl - sum;
+    for (int i = lo; i < hi; ++i) {
+        const int v = a[i];
+        a[i] = run;
+        run += v;
+    }
+    const int total = s_warp[32];
+    __syncthreads();
+    return total;
+}
+
+// One warp walks pairs [lo, hi) of s_ids in (token, k) order, 32 at a time,
+// adding the routed pairs of each expert to its own counters my[e].
+__device__ __forceinline__ void warp_count(const int32_t *s_ids, int lo, int hi, int K, int E, int32_t *my,
+                                           uint32_t &fl) {
+    const int lane = threadIdx.x & 31;
+    for (int base = lo; base < hi; base += 32) {
+        const int p = base + lane;
+        const int e = p < hi ? classify(s_ids, p, p % K, E, fl) : -1;
+        const unsigned peers = __match_any_sync(kFull, e >= 0 ? e : -1 - lane);
+        if (e >= 0 && (peers & lanemask_lt()) == 0) my[e] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+// Second walk over the same pairs: my[e] now holds the stable index of the
+// warp's first pair of expert e; each pair's index j goes through `look`.
+template <class Lookup>
+__device__ __forceinline__ void warp_assign(const int32_t *s_ids, int lo, int hi, int K, int E, int32_t *my,
+                                            int32_t *__restrict__ dest_row, Lookup look) {
+    const int lane = threadIdx.x & 31;
+    uint32_t fl = 0;
+    for (int base = lo; base < hi; base += 32) {
+        const int p = base + lane;
+        const int e = p < hi ? classify(s_ids, p, p % K, E, fl) : -1;
+        const unsigned peers = __match_any_sync(kFull, e >= 0 ? e : -1 - lane);
+        int dest = -1;
+        if (e >= 0) dest = look(e, my[e] + __popc(peers & lanemask_lt()));
+        __syncwarp();
+        if (e >= 0 && (peers & lanemask_lt()) == 0) my[e] += __popc(peers);
+        __syncwarp();
+        if (p < hi) dest_row[p] = dest;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// layouts (s_cnt holds the per-expert counts of routed pairs)
+// ---------------------------------------------------------------------------
+
+// HT: experts in id order; LL: [E][cap] rows, pairs beyond cap dropped.
+// Every thread of the CTA calls it; it leaves the kept length and first row
+// of every expert in s_len / s_base and returns the number of kept rows.
+__device__ int plain_tables(const Dims &d, const int32_t *s_cnt, int32_t *s_len, int32_t *s_base, int32_t *s_warp,
+                            uint32_t *s_fl) {
+    const int E = d.E, tid = threadIdx.x, nth = blockDim.x;
+    const bool ll = d.mode == EP_MODE_LL;
+    uint32_t fl = 0;
+    for (int e = tid; e < E; e += nth) {
+        const int c = s_cnt[e];
+        const int kept = ll ? min(c, d.cap) : c;
+        if (ll && c > d.cap) fl |= EP_FLAG_CAPACITY;
+        s_len[e] = kept;
+        s_base[e] = ll ? e * d.cap : kept;
+    }
+    block_or(fl, s_fl);
+    __syncthreads();
+    int total = 0;
+    if (!ll) total = block_exscan(s_base, E, s_warp);
+    __syncthreads();
+    return total;
+}
+
+// The plain layout's outputs (one CTA writes them).
+__device__ void plain_outputs(const Dims &d, const Workspace &ws, const int32_t *s_len, const int32_t *s_base,
+                              int total) {
+    const int E = d.E, R = d.R, g = d.g, tid = threadIdx.x, nth = blockDim.x;
+    const bool ll = d.mode == EP_MODE_LL;
+    for (int e = tid; e < E; e += nth) {
+        ws.len0[e] = s_len[e];
+        ws.base0[e] = s_base[e];
+        ws.recv_counts[e] = s_len[e];
+    }
+    for (int r = tid; r < R; r += nth) {
+        int s = 0;
+        for (int i = 0; i < g; ++i) s += s_len[r * g + i];
+        ws.rank_load[r] = s;
+        ws.rank_off[r] = ll ? r * g * d.cap : s_base[r * g];
+    }
+    if (tid == 0) {
+        ws.rank_off[R] = ll ? E * d.cap : total;
+        *ws.red_count = 0;
+    }
+}
+
+__device__ __forceinline__ void write_piece(const Dims &d, const Workspace &ws, int e, int pc, int start, int len,
+                                            int rank, int slot) {
+    const int64_t o = (int64_t)e * d.P + pc;
+    ws.piece_start[o] = start;
+    ws.piece_len[o] = len;
+    ws.piece_rank[o] = rank;
+    ws.piece_slot[o] = slot;
+}
+
+// Balanced-replica plan (MoonEP article paras. 3 and 5). The article states
+// only the invariants; this is a deterministic greedy:
+//  keep     each rank visits its own experts by (count asc, id asc) and keeps
+//           rows up to its capacity q or q+1 (q = L/R, first L%R ranks +1);
+//  spill    experts with rows left, by (count desc, id asc), fill the ranks
+//           with a deficit, visited once in (deficit desc, rank asc) order,
+//           each piece taking a new replica slot of the receiving rank
+//           (at most S per rank); rows no rank can take stay with the owner
+//           and EP_FLAG_PLAN_SLOTS is raised;
+//  layout   rank regions in rank order; inside one, own experts in id order
+//           then replica slots in slot order.
+// Every piece of an expert covers a run of its stable indices; the owner's
+// run [0, keep) is piece 0, the others ("extra" pieces) are stored compactly.
+__device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_t *s_cnt, int32_t *sm,
+                                int32_t *s_warp, uint32_t *s_fl) {
+    const int E = d.E, R = d.R, g = d.g, S = d.S, tid = threadIdx.x, nth = blockDim.x;
+    int32_t *s_keep = sm;                     // [E]
+    int32_t *s_tail = s_keep + E;             // [E] rows left on the owner after the fill
+    int32_t *s_list = s_tail + E;             // [E] scratch list / flags
+    int32_t *s_spill = s_list + E;            // [E] spilled experts
+    int32_t *s_own = s_spill + E;             // [E] own lengths, then own offsets
+    int32_t *s_npc = s_own + E;               // [E] pieces per expert
+    int32_t *s_D = s_npc + E;                 // [R] deficits, then loads
+    int32_t *s_nrep = s_D + R;                // [R]
+    int32_t *s_recv = s_nrep + R;             // [R] receivers in visiting order
+    int32_t *s_roff = s_recv + R;             // [R+1]
+    int32_t *s_slot_e = s_roff + R + 1;       // [R*S]
+    int32_t *s_slot_len = s_slot_e + R * S;   // [R*S]
+    int32_t *s_slot_off = s_slot_len + R * S; // [R*S]
+    __shared__ int s_L, s_nrecv;
+
+    if (tid == 0) {
+        s_L = 0;
+        s_nrecv = 0;
+    }
+    for (int i = tid; i < R * S; i += nth) {
+        s_slot_e[i] = -1;
+        s_slot_len[i] = 0;
+    }
+    for (int r = tid; r < R; r += nth) s_nrep[r] = 0;
+    __syncthreads();
+    int part = 0;
+    for (int e = tid; e < E; e += nth) {
+        s_tail[e] = 0;
+        s_npc[e] = 1;
+        part += s_cnt[e];
+    }
+    part = __reduce_add_sync(kFull, part);
+    if ((tid & 31) == 0) atomicAdd(&s_L, part);
+    __syncthreads();
+    const int L = s_L, q = L / R, rem = L % R;
+
+    // keep: rows of the experts visited before e on its rank (sorted order)
+    for (int e = tid; e < E; e += nth) {
+        const int r = e / g, c = s_cnt[e];
+        int before = 0;
+        for (int i = 0; i < g; ++i) {
+            const int e2 = r * g + i, c2 = s_cnt[e2];
+            if (c2 < c || (c2 == c && e2 < e)) before += c2;
+        }
+        const int cap = q + (r < rem ? 1 : 0);
+        s_keep[e] = max(0, min(c, cap - before));
+    }
+    __syncthreads();
+    for (int r = tid; r < R; r += nth) {
+        int used = 0;
+        for (int i = 0; i < g; ++i) used += s_keep[r * g + i];
+        s_D[r] = q + (r < rem ? 1 : 0) - used;
+    }
+    for (int e = tid; e < E; e += nth) s_list[e] = s_cnt[e] > s_keep[e] ? 1 : 0;
+    __syncthreads();
+    const int nsp = block_exscan(s_list, E, s_warp); // position among spilled, id order
+    for (int e = tid; e < E; e += nth)
+        if (s_cnt[e] > s_keep[e]) s_spill[s_list[e]] = e;
+    __syncthreads();
+    // spilled experts by (count desc, id asc): rank within the compact list
+    for (int i = tid; i < nsp; i += nth) {
+        const int e = s_spill[i], c = s_cnt[e];
+        int pos = 0;
+        for (int i2 = 0; i2 < nsp; ++i2) {
+            const int e2 = s_spill[i2], c2 = s_cnt[e2];
+            if (c2 > c || (c2 == c && e2 < e)) ++pos;
+        }
+        s_list[pos] = e;
+    }
+    // receivers: deficit > 0, by (deficit desc, rank asc)
+    for (int r = tid; r < R; r += nth) {
+        if (s_D[r] <= 0) continue;
+        int pos = 0;
+        for (int r2 = 0; r2 < R; ++r2)
+            if (s_D[r2] > 0 && (s_D[r2] > s_D[r] || (s_D[r2] == s_D[r] && r2 < r))) ++pos;
+        s_recv[pos] = r;
+        atomicAdd(&s_nrecv, 1);
+    }
+    __syncthreads();
+
+    // fill: one thread, one step per piece (receivers that ran out of deficit
+    // or slots never qualify again, so one cursor over them suffices)
+    if (tid == 0) {
+        const int nrecv = s_nrecv;
+        int p = 0;
+        uint32_t fl = 0;
+        for (int i = 0; i < nsp; ++i) {
+            const int e = s_list[i], owner = e / g;
+            int left = s_cnt[e] - s_keep[e], next = s_keep[e], npc = 1;
+            while (left > 0) {
+                while (p < nrecv && (s_D[s_recv[p]] == 0 || s_nrep[s_recv[p]] >= S)) ++p;
+                if (p == nrecv) {
+                    s_tail[e] = left;
+                    write_piece(d, ws, e, npc++, next, left, owner, -2);
+                    fl |= EP_FLAG_PLAN_SLOTS;
+                    break;
+                }
+                const int r = s_recv[p];
+                const int give = min(left, s_D[r]);
+                const int s = s_nrep[r]++;
+                s_slot_e[r * S + s] = e;
+                s_slot_len[r * S + s] = give;
+                write_piece(d, ws, e, npc++, next, give, r, s);
+                s_D[r] -= give;
+                left -= give;
+                next += give;
+            }
+            s_npc[e] = npc;
+        }
+        if (fl) atomicOr(s_fl, fl);
+    }
+    __syncthreads();
+
+    // layout inside each rank region
+    for (int e = tid; e < E; e += nth) s_own[e] = s_keep[e] + s_tail[e];
+    __syncthreads();
+    for (int r = tid; r < R; r += nth) {
+        int run = 0;
+        int32_t *rc = ws.recv_counts + (int64_t)r * (g + S);
+        for (int i = 0; i < g; ++i) {
+            const int e = r * g + i, v = s_own[e];
+            rc[i] = v;
+            s_own[e] = run;
+            run += v;
+        }
+        for (int s = 0; s < S; ++s) {
+            const int v = s_slot_len[r * S + s];
+            rc[g + s] = v;
+            s_slot_off[r * S + s] = run;
+            run += v;
+        }
+        s_roff[r] = run;
+        ws.rank_load[r] = run;
+    }
+    __syncthreads();
+    const int total = block_exscan(s_roff, R, s_warp);
+    for (int r = tid; r < R; r += nth) ws.rank_off[r] = s_roff[r];
+    if (tid == 0) ws.rank_off[R] = total;
+    for (int i = tid; i < R * S; i += nth) ws.replica_expert[i] = s_slot_e[i];
+    for (int e = tid; e < E; e += nth) s_list[e] = s_npc[e] - 1;
+    __syncthreads();
+    const int nx = block_exscan(s_list, E, s_warp); // s_list[e] = first extra piece of e
+    if (tid == 0) ws.xoff[E] = nx;
+
+    // piece 0, the compact extra pieces, and the per-expert replica lists
+    for (int e = tid; e < E; e += nth) {
+        const int owner = e / g;
+        const int own_base = s_roff[owner] + s_own[e];
+        ws.base0[e] = own_base;
+        ws.len0[e] = s_keep[e];
+        ws.xoff[e] = s_list[e];
+        const int64_t o = (int64_t)e * d.P;
+        int32_t *lst = ws.red_list + (int64_t)e * R;
+        int n = 0;
+        for (int pc = 1; pc < s_npc[e]; ++pc) {
+            const int r = ws.piece_rank[o + pc], s = ws.piece_slot[o + pc];
+            const int x = s_list[e] + pc - 1;
+            ws.xstart[x] = ws.piece_start[o + pc];
+            ws.xlen[x] = ws.piece_len[o + pc];
+            if (s == -2) {
+                ws.xdst[x] = own_base + s_keep[e];
+                continue;
+            }
+            ws.xdst[x] = s_roff[r] + s_slot_off[r * S + s];
+            const int key = r * S + s;
+            int a = n++;
+            while (a > 0 && lst[a - 1] > key) { // insertion sort, at most R-1 entries
+                lst[a] = lst[a - 1];
+                --a;
+            }
+            lst[a] = key;
+        }
+        ws.red_n[e] = n;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += nth) s_list[e] = ws.red_n[e] > 0 ? 1 : 0;
+    __syncthreads();
+    const int nred = block_exscan(s_list, E, s_warp);
+    for (int e = tid; e < E; e += nth)
+        if (ws.red_n[e] > 0) ws.red_experts[s_list[e]] = e;
+    if (tid == 0) *ws.red_count = nred;
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// 1. per warp tile: validate ids, stable rank of each pair inside the tile,
+//    per-expert counts of the tile
+// ---------------------------------------------------------------------------
+// Each warp owns `wt` consecutive pairs (a warp tile; whole steps of 32).
+// packed[p] = e | rank << 16 for a routed pair (rank = earlier pairs of the
+// same tile with the same expert), 0xffff otherwise. cnt_tile[tile][e].
+__global__ void __launch_bounds__(kRouteThreads) k_route_hist(const int32_t *__restrict__ idx, Dims d,
+                                                               Workspace ws) {
+    extern __shared__ int32_t sm[];
+    __shared__ uint32_t s_fl;
+    const int E = d.E, K = d.K, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int tile = blockIdx.x * kRouteWarps + w;
+    int32_t *my = sm + w * (E + d.wt);   // [E] counters of this warp's tile
+    int32_t *ids = my + E;               // [wt] the tile's expert ids
+    if (threadIdx.x == 0) s_fl = 0;
+    const int64_t lo = (int64_t)tile * d.wt, hi = min(d.L, lo + d.wt);
+    const int n = (int)max((int64_t)0, hi - lo);
+    for (int i = lane; i < E; i += 32) my[i] = 0;
+    // stage the whole tile first: one memory latency per warp, not per step
+    for (int i = lane; i < n; i += 32) ids[i] = __ldg(idx + lo + i);
+    __syncthreads();
+    uint32_t fl = 0;
+    for (int base = 0; base < n; base += 32) { // warp-uniform
+        const int i = base + lane;
+        int e = -1;
+        if (i < n) {
+            e = ids[i];
+            const int k = (int)((lo + i) % K);
+            if (e == -1) {
+            } else if (e < 0 || e >= E) {
+                fl |= EP_FLAG_BAD_EXPERT_ID;
+                e = -1;
+            } else {
+                for (int k2 = 1; k2 <= k; ++k2) {
+                    const int prev = i - k2 >= 0 ? ids[i - k2] : __ldg(idx + lo + i - k2); // token may start in the previous tile
+                    if (prev == e) {
+                        fl |= EP_FLAG_DUP_EXPERT_ID;
+                        e = -1;
+                        break;
+                    }
+                }
+            }
+        }
+        const unsigned peers = __match_any_sync(kFull, e >= 0 ? e : -1 - lane);
+        const unsigned lower = peers & lanemask_lt();
+        int packed = 0xffff;
+        if (e >= 0) packed = e | ((my[e] + __popc(lower)) << 16);
+        __syncwarp();
+        if (e >= 0 && lower == 0) my[e] += __popc(peers);
+        __syncwarp();
+        if (i < n) ws.packed[lo + i] = packed;
+    }
+    if (n > 0)
+        for (int i = lane; i < E; i += 32) ws.blk[(int64_t)tile * E + i] = my[i];
+    block_or(fl, &s_fl);
+    __syncthreads();
+    if (threadIdx.x == 0) ws.tile_flags[blockIdx.x] = s_fl;
+}
+
+// ---------------------------------------------------------------------------
+// 2. per expert: exclusive scan of the tile counts over tiles (lane = expert,
+//    warp = a chunk of tiles, so every access is coalesced); with a plan, the
+//    CTA that finishes last builds it
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kPlanThreads) k_route_scan(Dims d, Workspace ws) {
+    extern __shared__ int32_t sm[];
+    __shared__ int32_t s_warp[33];
+    __shared__ int32_t s_part[32][33];
+    __shared__ uint32_t s_fl;
+    __shared__ int s_last;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, tid = threadIdx.x, nth = blockDim.x;
+    const int e = blockIdx.x * 32 + lane;
+    const int chunk = (d.ntiles + 31) / 32;
+    const int t0 = min(d.ntiles, w * chunk), t1 = min(d.ntiles, t0 + chunk);
+    constexpr int B = 16; // loads in flight per thread
+    int sum = 0;
+    if (e < d.E) {
+        for (int t = t0; t < t1; t += B) {
+            int v[B];
+#pragma unroll
+            for (int u = 0; u < B; ++u) v[u] = t + u < t1 ? ws.blk[(int64_t)(t + u) * d.E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < B; ++u) sum += v[u];
+        }
+    }
+    s_part[w][lane] = sum;
+    __syncthreads();
+    int run = 0;
+    for (int ww = 0; ww < w; ++ww) run += s_part[ww][lane];
+    if (e < d.E) {
+        for (int t = t0; t < t1; t += B) {
+            int v[B];
+#pragma unroll
+            for (int u = 0; u < B; ++u) v[u] = t + u < t1 ? ws.blk[(int64_t)(t + u) * d.E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < B; ++u) {
+                if (t + u < t1) ws.blk[(int64_t)(t + u) * d.E + e] = run;
+                run += v[u];
+            }
+        }
+        if (w == 31) {
+            ws.cnt[e] = run;
+            if (d.balanced) __threadfence();
+        }
+    }
+    if (!d.balanced) return;
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const unsigned long long t = atomicAdd(ws.ticket, 1ull);
+        s_last = ((t + 1) % gridDim.x) == 0; // every launch draws exactly gridDim.x tickets
+        s_fl = 0;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    int32_t *s_cnt = sm; // [E]
+    uint32_t fl = 0;
+    for (int i = tid; i < d.E; i += nth) s_cnt[i] = __ldcg(ws.cnt + i);
+    for (int b = tid; b < d.nhist; b += nth) fl |= __ldcg(ws.tile_flags + b);
+    block_or(fl, &s_fl);
+    __syncthreads();
+    layout_balanced(d, ws, s_cnt, sm + d.E, s_warp, &s_fl);
+    if (tid == 0) *ws.flags = s_fl;
+}
+
+// ---------------------------------------------------------------------------
+// 3. destination rows: j = tile base + rank in tile, then the layout tables
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspace ws) {
+    extern __shared__ int32_t sm[];
+    __shared__ int32_t s_warp[33];
+    __shared__ uint32_t s_fl;
+    const int E = d.E, tid = threadIdx.x, nth = blockDim.x;
+    int32_t *s_len = sm;         // [E] length of piece 0
+    int32_t *s_base = s_len + E; // [E] first row of piece 0
+    int32_t *s_cnt = s_base + E; // [E] (plain layouts)
+    int32_t *s_xoff = s_cnt + E; // [E+1] extra pieces (plan only)
+    int32_t *s_xs = s_xoff + E + 1;
+    int32_t *s_xl = s_xs + d.nx_max;
+    int32_t *s_xd = s_xl + d.nx_max;
+    if (tid == 0) s_fl = 0;
+    if (d.balanced) {
+        for (int i = tid; i < E; i += nth) {
+            s_base[i] = ws.base0[i];
+            s_len[i] = ws.len0[i];
+        }
+        for (int i = tid; i <= E; i += nth) s_xoff[i] = ws.xoff[i];
+        const int nx = ws.xoff[E];
+        for (int i = tid; i < nx; i += nth) {
+            s_xs[i] = ws.xstart[i];
+            s_xl[i] = ws.xlen[i];
+            s_xd[i] = ws.xdst[i];
+        }
+        __syncthreads();
+    } else {
+        for (int i = tid; i < E; i += nth) s_cnt[i] = ws.cnt[i];
+        __syncthreads();
+        const int total = plain_tables(d, s_cnt, s_len, s_base, s_warp, &s_fl);
+        if (blockIdx.x == 0) {
+            plain_outputs(d, ws, s_len, s_base, total);
+            uint32_t fl = 0;
+            for (int b = tid; b < d.nhist; b += nth) fl |= ws.tile_flags[b];
+            block_or(fl, &s_fl);
+            __syncthreads();
+            if (tid == 0) *ws.flags = s_fl;
+        }
+    }
+    // kAssignPer pairs per thread; all loads are issued before any is used
+    const int64_t p0 = (int64_t)blockIdx.x * nth * kAssignPer + tid;
+    int pk[kAssignPer], jb[kAssignPer];
+#pragma unroll
+    for (int u = 0; u < kAssignPer; ++u) {
+        const int64_t p = p0 + (int64_t)u * nth;
+        pk[u] = p < d.L ? ws.packed[p] : 0xffff;
+    }
+#pragma unroll
+    for (int u = 0; u < kAssignPer; ++u) {
+        const int64_t p = p0 + (int64_t)u * nth;
+        const int e = pk[u] & 0xffff;
+        jb[u] = e != 0xffff ? ws.blk[(p / d.wt) * E + e] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kAssignPer; ++u) {
+        const int64_t p = p0 + (int64_t)u * nth;
+        if (p >= d.L) continue;
+        const int e = pk[u] & 0xffff;
+        int dest = -1;
+        if (e != 0xffff) {
+            const int j = jb[u] + (pk[u] >> 16);
+            if (j < s_len[e]) {
+                dest = s_base[e] + j;
+            } else if (d.balanced) {
+                for (int x = s_xoff[e]; x < s_xoff[e + 1]; ++x)
+                    if (j >= s_xs[x] && j < s_xs[x] + s_xl[x]) {
+                        dest = s_xd[x] + (j - s_xs[x]);
+                        break;
+                    }
+            }
+        }
+        ws.dest_row[p] = dest;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// small batches, plain layouts: everything in one CTA
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__restrict__ idx, Dims d,
+                                                                Workspace ws) {
+    extern __shared__ int32_t sm[];
+    __shared__ int32_t s_warp[33];
+    __shared__ uint32_t s_fl;
+    const int E = d.E, K = d.K, w = threadIdx.x >> 5, np = (int)d.L;
+    int32_t *s_wc = sm;                   // [warps][E]
+    int32_t *s_cnt = s_wc + kSmallWarps * E;
+    int32_t *s_len = s_cnt + E;
+    int32_t *s_base = s_len + E;
+    int32_t *s_ids = s_base + E;          // [L]
+    if (threadIdx.x == 0) s_fl = 0;
+    for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) s_wc[i] = 0;
+    load_ids(idx, 0, np, s_ids);
+    __syncthreads();
+    // each warp owns a contiguous run of pairs; the repeat check reads the
+    // earlier choices of a token from s_ids, whichever warp owns them
+    const int per_warp = ((np + kSmallWarps - 1) / kSmallWarps + 31) & ~31;
+    const int lo = w * per_warp, hi = min(np, lo + per_warp);
+    int32_t *my = s_wc + w * E;
+    uint32_t fl = 0;
+    warp_count(s_ids, lo, hi, K, E, my, fl);
+    block_or(fl, &s_fl);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int ww = 0; ww < kSmallWarps; ++ww) {
+            const int v = s_wc[ww * E + e];
+            s_wc[ww * E + e] = run;
+            run += v;
+        }
+        s_cnt[e] = run;
+        ws.cnt[e] = run;
+    }
+    __syncthreads();
+    const int total = plain_tables(d, s_cnt, s_len, s_base, s_warp, &s_fl);
+    plain_outputs(d, ws, s_len, s_base, total);
+    warp_assign(s_ids, lo, hi, K, E, my, ws.dest_row,
+                [&](int e, int j) { return j < s_len[e] ? s_base[e] + j : -1; });
+    __syncthreads();
+    if (threadIdx.x == 0) *ws.flags = s_fl;
+}
+
+} // namespace
+
+size_t route_smem_layout(const Dims &d) {
+    if (!d.balanced) return 0;
+    const size_t E = d.E, R = d.R, S = d.S;
+    return sizeof(int32_t) * (E + 6 * E + 4 * R + 1 + 3 * R * S);
+}
+
+size_t route_smem_assign(const Dims &d) {
+    const size_t E = d.E;
+    size_t n = 3 * E;
+    if (d.balanced) n += E + 1 + 3 * (size_t)d.nx_max;
+    return sizeof(int32_t) * n;
+}
+
+size_t route_smem_hist(const Dims &d) { return sizeof(int32_t) * (size_t)kRouteWarps * (d.E + d.wt); }
+
+size_t route_smem_small(const Dims &d) { return sizeof(int32_t) * ((size_t)(kSmallWarps + 3) * d.E + d.L); }
+
+bool route_use_small(const Dims &d) {
+    return !d.balanced && d.L <= kSmallMaxPairs && d.E <= kSmallMaxExperts;
+}
+
+cudaError_t launch_plan(const Dims &d, const Workspace &ws, const int32_t *topk_idx, cudaStream_t st) {
+    static bool attrs_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attrs_set[dev]) { // per-device function attributes, set once
+        const int max_dyn = kMaxRouteSmem;
+        cudaFuncSetAttribute(k_route_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+        cudaFuncSetAttribute(k_route_assign, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+        cudaFuncSetAttribute(k_route_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+        cudaFuncSetAttribute(k_route_small, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+        attrs_set[dev] = true;
+    }
+    cudaError_t err;
+    if (route_use_small(d)) {
+        k_route_small<<<1, kSmallThreads, route_smem_small(d), st>>>(topk_idx, d, ws);
+        return cudaGetLastError();
+    }
+    if (d.L > 0) {
+        k_route_hist<<<d.nhist, kRouteThreads, route_smem_hist(d), st>>>(topk_idx, d, ws);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    }
+    k_route_scan<<<(d.E + 31) / 32, kPlanThreads, route_smem_layout(d), st>>>(d, ws);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    k_route_assign<<<d.nassign, kRouteThreads, route_smem_assign(d), st>>>(d, ws);
+    return cudaGetLastError();
+}
+
+int plan_launches(const Dims &d) { return route_use_small(d) ? 1 : (d.L > 0 ? 3 : 2); }
+
+} // namespace epb

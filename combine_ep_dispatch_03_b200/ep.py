@@ -1,0 +1,263 @@
+"""Thin ctypes binding of the C ABI in include/ep.h (argument marshalling only).
+
+Every step of dispatch / combine runs in libep_b200.so's CUDA kernels; this
+module checks tensor shapes and dtypes, passes raw device pointers and the
+current CUDA stream, and turns status codes into exceptions. PyTorch is used
+for device memory and streams only. There is no fallback: if the library is
+missing, ``lib()`` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libep_b200.so")
+
+MODE_LL, MODE_HT = 0, 1
+FLAG_BAD_EXPERT_ID, FLAG_DUP_EXPERT_ID, FLAG_CAPACITY, FLAG_PLAN_SLOTS = 0x1, 0x2, 0x4, 0x8
+T_DEST_ROW, T_EXPERT_COUNTS, T_RECV_COUNTS, T_RANK_LOAD, T_RANK_OFFSET, T_REPLICA_EXPERT = range(6)
+
+
+class EpConfig(ctypes.Structure):
+    _fields_ = [
+        ("num_tokens", ctypes.c_int32),
+        ("hidden", ctypes.c_int32),
+        ("num_experts", ctypes.c_int32),
+        ("topk", ctypes.c_int32),
+        ("num_ranks", ctypes.c_int32),
+        ("mode", ctypes.c_int32),
+        ("ll_capacity", ctypes.c_int32),
+        ("fp8", ctypes.c_int32),
+        ("balanced", ctypes.c_int32),
+        ("replica_slots", ctypes.c_int32),
+        ("grad_elems_per_expert", ctypes.c_int64),
+    ]
+
+
+class EpError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        self.status = status
+        super().__init__(f"{call} failed: {_lib_status_string(status)} ({status})")
+
+
+# name -> (restype, argtypes); every entry point of include/ep.h
+_P, _I32, _I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+_CFG = ctypes.POINTER(EpConfig)
+SIGNATURES = {
+    "ep_validate_config": (ctypes.c_int, [_CFG]),
+    "ep_recv_rows": (ctypes.c_int, [_CFG, ctypes.POINTER(_I64)]),
+    "ep_recv_counts_len": (ctypes.c_int, [_CFG, ctypes.POINTER(_I64)]),
+    "ep_workspace_bytes": (ctypes.c_int, [_CFG, ctypes.POINTER(ctypes.c_size_t)]),
+    "ep_plan_kernel_count": (ctypes.c_int, [_CFG, ctypes.POINTER(_I32)]),
+    "ep_version": (ctypes.c_char_p, []),
+    "ep_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ep_create": (ctypes.c_int, [_CFG, ctypes.POINTER(_P)]),
+    "ep_destroy": (ctypes.c_int, [_P]),
+    "ep_plan": (ctypes.c_int, [_P, _P, _P]),
+    "ep_dispatch": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "ep_combine": (ctypes.c_int, [_P, _P, _P, _P, _P]),
+    "ep_combine_backward": (ctypes.c_int, [_P, _P, _P, _P, _P]),
+    "ep_dispatch_backward": (ctypes.c_int, [_P, _P, _P, _P]),
+    "ep_reduce_replica_grads": (ctypes.c_int, [_P, _P, _P, _P]),
+    "ep_get_plan": (ctypes.c_int, [_P, _P, _P, _P]),
+    "ep_get_status": (ctypes.c_int, [_P, ctypes.POINTER(_I32), _P]),
+    "ep_get_tensor": (ctypes.c_int, [_P, ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(_I64)]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libep_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m combine_ep_dispatch_03_b200.build` "
+                "(there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _lib_status_string(status: int) -> str:
+    try:
+        return lib().ep_status_string(status).decode()
+    except Exception:  # pragma: no cover
+        return "status"
+
+
+def _check(call: str, status: int) -> None:
+    if status != 0:
+        raise EpError(call, status)
+
+
+def make_config(T: int, H: int, E: int, K: int, R: int, mode: str = "ht", ll_capacity: int = 0,
+                fp8: bool = False, balanced: bool = False, replica_slots: int = 0,
+                grad_elems_per_expert: int = 0) -> EpConfig:
+    return EpConfig(T, H, E, K, R, MODE_LL if mode == "ll" else MODE_HT, ll_capacity, int(fp8), int(balanced),
+                    replica_slots, grad_elems_per_expert)
+
+
+def validate(cfg: EpConfig) -> int:
+    return lib().ep_validate_config(ctypes.byref(cfg))
+
+
+def plan_launches(h: "Ep") -> int:
+    """Kernels one ep_plan of this handle's configuration launches."""
+    n = ctypes.c_int32()
+    _check("ep_plan_kernel_count", lib().ep_plan_kernel_count(ctypes.byref(h.cfg), ctypes.byref(n)))
+    return n.value
+
+
+def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, numel: int | None = None,
+         name: str = "tensor") -> ctypes.c_void_p | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} must have {numel} elements, got {t.numel()}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: torch.cuda.Stream | None) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class _DeviceArray:
+    """__cuda_array_interface__ view of a device pointer owned by the handle."""
+
+    def __init__(self, ptr: int, n: int, typestr: str = "<i4"):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": typestr, "data": (ptr, False), "version": 3}
+
+
+class Ep:
+    """One EP configuration and its routing state (group + handle in one)."""
+
+    def __init__(self, T: int, H: int, E: int, K: int, R: int, mode: str = "ht", ll_capacity: int = 0,
+                 fp8: bool = False, balanced: bool = False, replica_slots: int = 0,
+                 grad_elems_per_expert: int = 0):
+        L = lib()
+        self.cfg = make_config(T, H, E, K, R, mode, ll_capacity, fp8, balanced, replica_slots,
+                               grad_elems_per_expert)
+        self.T, self.H, self.E, self.K, self.R = T, H, E, K, R
+        self.mode, self.fp8, self.balanced = mode, fp8, balanced
+        self.S = (replica_slots or E // R) if balanced else 0
+        self.G = grad_elems_per_expert
+        rows, clen = ctypes.c_int64(), ctypes.c_int64()
+        _check("ep_recv_rows", L.ep_recv_rows(ctypes.byref(self.cfg), ctypes.byref(rows)))
+        _check("ep_recv_counts_len", L.ep_recv_counts_len(ctypes.byref(self.cfg), ctypes.byref(clen)))
+        self.recv_rows, self.counts_len = rows.value, clen.value
+        h = ctypes.c_void_p()
+        _check("ep_create", L.ep_create(ctypes.byref(self.cfg), ctypes.byref(h)))
+        self._h = h
+
+    # -- lifetime
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            _check("ep_destroy", lib().ep_destroy(self._h))
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    # -- output allocation helpers (plumbing)
+    def empty_recv(self, device="cuda") -> dict:
+        rows, H = self.recv_rows, self.H
+        out = {
+            "recv_x": torch.empty((rows, H), dtype=torch.float8_e4m3fn if self.fp8 else torch.bfloat16,
+                                  device=device),
+            "recv_scales": torch.empty((rows, H // 128), dtype=torch.float32, device=device) if self.fp8 else None,
+            "recv_w": torch.empty(rows, dtype=torch.float32, device=device),
+            "recv_expert": torch.empty(rows, dtype=torch.int32, device=device),
+            "recv_counts": torch.empty(self.counts_len, dtype=torch.int32, device=device),
+        }
+        return out
+
+    # -- forward
+    def plan(self, topk_idx: torch.Tensor, stream=None) -> None:
+        _check("ep_plan", lib().ep_plan(self._h, _ptr(topk_idx, torch.int32, self.T * self.K, "topk_idx"),
+                                        _stream(stream)))
+
+    def dispatch(self, x, topk_idx, topk_w, recv_x, recv_scales=None, recv_w=None, recv_expert=None,
+                 recv_counts=None, stream=None) -> None:
+        """Rows, scales (FP8), weights, expert ids and per-slot counts into the
+        caller's receive buffers (see empty_recv)."""
+        rows, H = self.recv_rows, self.H
+        _check("ep_dispatch", lib().ep_dispatch(
+            self._h, _ptr(x, torch.bfloat16, self.T * H, "x"),
+            _ptr(topk_idx, torch.int32, self.T * self.K, "topk_idx"),
+            _ptr(topk_w, torch.float32, self.T * self.K, "topk_w"),
+            _ptr(recv_x, torch.float8_e4m3fn if self.fp8 else torch.bfloat16, rows * H, "recv_x"),
+            _ptr(recv_scales, torch.float32, rows * (H // 128), "recv_scales"),
+            _ptr(recv_w, torch.float32, rows, "recv_w"),
+            _ptr(recv_expert, torch.int32, rows, "recv_expert"),
+            _ptr(recv_counts, torch.int32, self.counts_len, "recv_counts"),
+            _stream(stream)))
+
+    def combine(self, expert_out, topk_w, out, stream=None) -> None:
+        _check("ep_combine", lib().ep_combine(
+            self._h, _ptr(expert_out, torch.bfloat16, self.recv_rows * self.H, "expert_out"),
+            _ptr(topk_w, torch.float32, self.T * self.K, "topk_w"),
+            _ptr(out, torch.bfloat16, self.T * self.H, "out"), _stream(stream)))
+
+    # -- backward
+    def combine_backward(self, grad_out, topk_w, grad_expert_out, stream=None) -> None:
+        _check("ep_combine_backward", lib().ep_combine_backward(
+            self._h, _ptr(grad_out, torch.bfloat16, self.T * self.H, "grad_out"),
+            _ptr(topk_w, torch.float32, self.T * self.K, "topk_w"),
+            _ptr(grad_expert_out, torch.bfloat16, self.recv_rows * self.H, "grad_expert_out"), _stream(stream)))
+
+    def dispatch_backward(self, grad_recv, grad_x, stream=None) -> None:
+        _check("ep_dispatch_backward", lib().ep_dispatch_backward(
+            self._h, _ptr(grad_recv, torch.bfloat16, self.recv_rows * self.H, "grad_recv"),
+            _ptr(grad_x, torch.bfloat16, self.T * self.H, "grad_x"), _stream(stream)))
+
+    def reduce_replica_grads(self, replica_grad, owner_grad, stream=None) -> None:
+        _check("ep_reduce_replica_grads", lib().ep_reduce_replica_grads(
+            self._h, _ptr(replica_grad, torch.float32, self.R * max(self.S, 1) * self.G, "replica_grad"),
+            _ptr(owner_grad, torch.float32, self.E * self.G, "owner_grad"), _stream(stream)))
+
+    # -- inspection
+    def get_plan(self, stream=None) -> tuple[list[int], list[int]]:
+        S = max(self.S, 1)
+        rep = (ctypes.c_int32 * (self.R * S))()
+        load = (ctypes.c_int32 * self.R)()
+        _check("ep_get_plan", lib().ep_get_plan(self._h, ctypes.cast(rep, _P), ctypes.cast(load, _P),
+                                                _stream(stream)))
+        return list(rep)[: self.R * self.S], list(load)
+
+    def status(self, stream=None) -> int:
+        f = ctypes.c_int32()
+        _check("ep_get_status", lib().ep_get_status(self._h, ctypes.byref(f), _stream(stream)))
+        return f.value
+
+    def tensor(self, which: int) -> torch.Tensor:
+        """A copy of one piece of the routing state (int32, on the device)."""
+        p, n = ctypes.c_void_p(), ctypes.c_int64()
+        _check("ep_get_tensor", lib().ep_get_tensor(self._h, which, ctypes.byref(p), ctypes.byref(n)))
+        if n.value == 0:
+            return torch.empty(0, dtype=torch.int32, device="cuda")
+        return torch.as_tensor(_DeviceArray(p.value, n.value), device="cuda").clone()

@@ -1,0 +1,226 @@
+/*
+ * ep.h -- C ABI of libep_b200: MoE expert-parallel token dispatch and
+ * combine on one B200 (sm_100a), with the EP world of R ranks held as R
+ * logical partitions of one HBM.
+ *
+ * The calls follow the statement of the problem on these pages:
+ *   - NCCL EP paper page (arXiv 2603.13606): long-lived groups and
+ *     per-forward-pass handles (Table II, Fig. 2); LL mode with a 3D
+ *     expert-major output and HT mode with a 2D concatenated output plus
+ *     per-expert token counts (Table III, Figs. 3-4); the tensor roles
+ *     TOKENS, TOPK_IDX, TOPK_WEIGHTS and FP8 quantization scales (Table IV);
+ *     dispatch(x, topk_i, topk_w, handle) -> recv_x, recv_i, recv_w
+ *     (Table V); combine gathers expert outputs and reduces them to the
+ *     original token order (Table II); routing state shared by the forward
+ *     and backward passes (Fig. 5).
+ *   - MoonEP news article (opensourceforu.com): a GPU planner that
+ *     replicates hot experts online so that every rank receives a
+ *     predictable load (para. 3), placement straight into expert-grouped rank
+ *     positions with static shapes and no per-layer host sync (para. 4), at
+ *     most E/R prefetch slots per rank in training, and a reduce buffer for
+ *     the gradients of duplicated experts (para. 5).
+ *
+ * Conventions for every call:
+ *   - Device pointers are plain CUDA device addresses owned by the caller;
+ *     the library never frees them and keeps none of them after the call
+ *     returns. Token rows (x, recv_x, expert outputs, gradients) must be
+ *     16-byte aligned; every other pointer naturally aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Every call except ep_get_* is asynchronous and stream-ordered:
+ *     it enqueues kernels and returns without a host synchronisation.
+ *   - Arguments the host can check are checked before anything is launched;
+ *     a failed check returns an error status and launches nothing.
+ *   - Conditions only the device can see (a bad or repeated expert id, LL
+ *     capacity overflow, a balanced plan that runs out of slots) never trap
+ *     and never hang: the offending pairs are skipped (or, for the plan,
+ *     kept on the owner rank) and a bit is set in the handle's status word,
+ *     read by ep_get_status.
+ *   - A handle is not thread-safe; calls on one handle must be ordered by
+ *     the caller (one stream, or explicit events).
+ */
+#ifndef EP_B200_H
+#define EP_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ep_status {
+    EP_OK = 0,
+    EP_ERR_INVALID_ARG = 1, /* a bad size, a NULL or misaligned pointer */
+    EP_ERR_CUDA = 2,        /* a CUDA runtime call or a launch failed */
+    EP_ERR_UNSUPPORTED = 3, /* a valid but unsupported combination */
+    EP_ERR_NOT_PLANNED = 4, /* a data call before the first ep_plan */
+    EP_ERR_NO_MEMORY = 5    /* workspace allocation failed */
+} ep_status_t;
+
+/* Bits of the device status word (ep_get_status). */
+#define EP_FLAG_BAD_EXPERT_ID 0x1 /* an id outside [0, E) other than -1 */
+#define EP_FLAG_DUP_EXPERT_ID 0x2 /* a token chose the same expert twice */
+#define EP_FLAG_CAPACITY 0x4      /* LL: an expert received more than ll_capacity rows */
+#define EP_FLAG_PLAN_SLOTS 0x8    /* balanced plan ran out of replica slots */
+
+typedef enum ep_mode { EP_MODE_LL = 0, EP_MODE_HT = 1 } ep_mode_t;
+
+/* Which piece of a handle's routing state ep_get_tensor exposes. */
+typedef enum ep_tensor {
+    EP_T_DEST_ROW = 0,       /* int32 [T*K]: receive-buffer row of pair (t,k), -1 if none */
+    EP_T_EXPERT_COUNTS = 1,  /* int32 [E]: routed pairs per expert */
+    EP_T_RECV_COUNTS = 2,    /* int32 [R*(E/R + S)] HT, [E] LL: rows per local slot */
+    EP_T_RANK_LOAD = 3,      /* int32 [R]: rows received by each logical rank */
+    EP_T_RANK_OFFSET = 4,    /* int32 [R+1]: first row of each rank's region */
+    EP_T_REPLICA_EXPERT = 5  /* int32 [R*S]: expert held by replica slot (r,s), -1 empty */
+} ep_tensor_t;
+
+/* One EP configuration: fixed for the lifetime of a handle (static shapes,
+ * MoonEP article para. 4). T tokens of H hidden values, E experts chosen
+ * top-K per token, R logical ranks owning E/R consecutive experts each;
+ * token t belongs to source rank t / (T/R) (contiguous blocks). */
+typedef struct ep_config {
+    int32_t num_tokens;            /* T >= 0 (T = 0 is an empty batch) */
+    int32_t hidden;                /* H > 0, multiple of 8 (of 128 with fp8) */
+    int32_t num_experts;           /* E in [1, 4096], multiple of R */
+    int32_t topk;                  /* K in [1, min(E, 32)] */
+    int32_t num_ranks;             /* R >= 1 */
+    int32_t mode;                  /* ep_mode_t */
+    int32_t ll_capacity;           /* LL: rows per expert (>= 1); ignored in HT */
+    int32_t fp8;                   /* 1: dispatch casts to FP8 e4m3 + fp32 scales */
+    int32_t balanced;              /* 1: balanced-replica plan (HT only; its tables must
+                                      fit one CTA's shared memory, about E <= 2048) */
+    int32_t replica_slots;         /* S in [1, E/R] with balanced; 0 = E/R */
+    int64_t grad_elems_per_expert; /* G for ep_reduce_replica_grads; 0 if unused */
+} ep_config_t;
+
+typedef struct ep_handle ep_handle_t;
+
+/* ---- host-only queries (no GPU needed) -------------------------------- */
+
+/* Check a configuration without touching the GPU. */
+ep_status_t ep_validate_config(const ep_config_t *cfg);
+
+/* Rows of the receive buffer: T*K in HT (one row per (token, k) pair,
+ * NCCL EP Table III "2D"), E*ll_capacity in LL (the 3D expert-major buffer
+ * [R][E/R][ll_capacity] flattened, Table III "3D"). */
+ep_status_t ep_recv_rows(const ep_config_t *cfg, int64_t *rows);
+
+/* Number of int32 entries of recv_counts: R*(E/R + S) in HT (per rank: its
+ * own experts in id order, then its S replica slots; S = 0 without a
+ * balanced plan, giving the per-expert counts [E]), E in LL. */
+ep_status_t ep_recv_counts_len(const ep_config_t *cfg, int64_t *len);
+
+/* Device bytes ep_create will allocate for the handle's workspace. */
+ep_status_t ep_workspace_bytes(const ep_config_t *cfg, size_t *bytes);
+
+/* Number of kernels one ep_plan launches for this configuration (one for
+ * small batches without a plan, else three); every other data call launches
+ * one kernel. */
+ep_status_t ep_plan_kernel_count(const ep_config_t *cfg, int32_t *count);
+
+/* "major.minor.patch" of the library. */
+const char *ep_version(void);
+
+/* Human-readable name of a status code. */
+const char *ep_status_string(ep_status_t status);
+
+/* ---- group / handle lifetime (NCCL EP Table II, Fig. 2) --------------- */
+
+/* Validate cfg and allocate the handle and all of its device workspace once
+ * (routing state, plan tables, status word), on the current CUDA device.
+ * No later call allocates. On error *out is NULL. */
+ep_status_t ep_create(const ep_config_t *cfg, ep_handle_t **out);
+
+/* Free the handle and its workspace (synchronises the device first).
+ * NULL is accepted. */
+ep_status_t ep_destroy(ep_handle_t *h);
+
+/* ---- forward ----------------------------------------------------------- */
+
+/* Routing for one forward pass (NCCL EP Fig. 5: the state it builds is
+ * reused by dispatch, combine and both backward calls until the next
+ * ep_plan). Clears the status word, then on the device:
+ *   counts   cnt[e] = routed pairs (t,k) with topk_idx[t,k] == e;
+ *   slots    j(t,k) = earlier routed pairs (t',k') < (t,k) in row-major
+ *            order with the same expert (stable, deterministic);
+ *   layout   HT: rows grouped by expert id, so rank r's region holds
+ *            experts r*E/R .. (r+1)*E/R-1; LL: row e*ll_capacity + j, pairs
+ *            with j >= ll_capacity dropped (EP_FLAG_CAPACITY);
+ *   plan     with cfg.balanced, the balanced-replica plan: each rank
+ *            receives floor or ceil of L/R rows (L = routed pairs), hot
+ *            experts spilling into at most S replica slots per rank
+ *            (MoonEP article paras. 3 and 5).
+ * topk_idx: device int32 [T, K] row-major. -1 marks a masked choice (not
+ * routed, no flag); other ids outside [0, E) and repeats within a token are
+ * skipped and flagged. */
+ep_status_t ep_plan(ep_handle_t *h, const int32_t *topk_idx, void *stream);
+
+/* Dispatch (NCCL EP Table V): for every routed pair (t,k) with row
+ * d = dest_row[t,k]:
+ *   recv_x[d, :]   = x[t, :]                       (bf16 rows [rows, H]), or
+ *   recv_x[d, :]   = e4m3(x[t, b-block] / s_b)     (fp8 rows [rows, H] bytes)
+ *   recv_scales[d, b] = s_b = amax_b / 448         (fp32 [rows, H/128])
+ *     with amax_b the max |x| of the b-th 128-element block of x[t], fp32
+ *     division, round-to-nearest-even, saturation to +-448; an all-zero
+ *     block gives s = 0 and codes +0 (NCCL EP Table IV FP8 scales);
+ *   recv_w[d]      = topk_w[t,k]       (fp32 [rows]; may be NULL)
+ *   recv_expert[d] = topk_idx[t,k]     (int32 [rows]; may be NULL)
+ * and recv_counts (int32, ep_recv_counts_len entries; may be NULL) receives
+ * the rows per local slot. Rows no pair targets (LL padding) are not
+ * written. x: device bf16 [T, H]. topk_idx must be the array given to the
+ * last ep_plan (it may be NULL when recv_expert is NULL). recv_scales must
+ * be non-NULL iff cfg.fp8. */
+ep_status_t ep_dispatch(ep_handle_t *h, const void *x, const int32_t *topk_idx, const float *topk_w,
+                        void *recv_x, float *recv_scales, float *recv_w, int32_t *recv_expert,
+                        int32_t *recv_counts, void *stream);
+
+/* Combine (NCCL EP Table II combine row, Table III per-token reduction):
+ *   out[t, :] = bf16( fold_k acc = fmaf(topk_w[t,k], y[dest_row[t,k], :], acc) )
+ * over k = 0..K-1 in order, acc starting at +0 in fp32, pairs without a row
+ * skipped, one round-to-nearest-even at the end.
+ * expert_out: device bf16 [rows, H]; topk_w: fp32 [T, K]; out: bf16 [T, H]. */
+ep_status_t ep_combine(ep_handle_t *h, const void *expert_out, const float *topk_w, void *out, void *stream);
+
+/* ---- backward (NCCL EP Fig. 5: same routing state, roles swapped) ------ */
+
+/* Gradient of combine w.r.t. the expert outputs, a dispatch-shaped pass:
+ *   grad_expert_out[dest_row[t,k], :] = bf16(topk_w[t,k] * grad_out[t, :])
+ * (fp32 product, one bf16 rounding). grad_out: bf16 [T, H];
+ * grad_expert_out: bf16 [rows, H]; rows without a pair are not written. */
+ep_status_t ep_combine_backward(ep_handle_t *h, const void *grad_out, const float *topk_w, void *grad_expert_out,
+                                void *stream);
+
+/* Gradient of dispatch w.r.t. x, a combine-shaped pass (unweighted):
+ *   grad_x[t, :] = bf16( sum_k grad_recv[dest_row[t,k], :] )
+ * fp32 adds in k order from +0. Only bf16 dispatch has a gradient here (an
+ * FP8 payload is forward-only). grad_recv: bf16 [rows, H]; grad_x: bf16 [T, H]. */
+ep_status_t ep_dispatch_backward(ep_handle_t *h, const void *grad_recv, void *grad_x, void *stream);
+
+/* Replica-gradient reduce (MoonEP article para. 5): for every expert e
+ * that has replicas under the current plan,
+ *   owner_grad[e, :] += replica_grad[r, s, :] for each slot (r, s) with
+ *                       replica_expert[r, s] == e, in ascending (r, s) order,
+ * fp32. replica_grad: device fp32 [R, S, G]; owner_grad: fp32 [E, G], updated
+ * in place; G = cfg.grad_elems_per_expert. Needs cfg.balanced. */
+ep_status_t ep_reduce_replica_grads(ep_handle_t *h, const float *replica_grad, float *owner_grad, void *stream);
+
+/* ---- inspection (these synchronise the stream) ------------------------- */
+
+/* Wait for `stream`, then copy the plan to host memory: replica_expert
+ * [R*S] (-1 = empty slot; may be NULL) and rank_load [R] (may be NULL). */
+ep_status_t ep_get_plan(ep_handle_t *h, int32_t *replica_expert_host, int32_t *rank_load_host, void *stream);
+
+/* Wait for `stream`, then read the device status word (EP_FLAG_* bits set
+ * since the last ep_plan). */
+ep_status_t ep_get_status(ep_handle_t *h, int32_t *flags, void *stream);
+
+/* Read-only device pointer and element count of one piece of the handle's
+ * routing state (valid until the next ep_plan or ep_destroy). */
+ep_status_t ep_get_tensor(const ep_handle_t *h, ep_tensor_t which, const void **dptr, int64_t *numel);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_B200_H */

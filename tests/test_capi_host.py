@@ -1,0 +1,94 @@
+"""The C-ABI library loads and exports every entry point include/ep.h
+declares; the host-only queries validate configurations without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def L():
+    from combine_ep_dispatch_03_b200 import build, ep
+
+    build.build()
+    return ep.lib()
+
+
+def _declared() -> list[str]:
+    src = open(os.path.join(ROOT, "include", "ep.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ep_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_api():
+    names = _declared()
+    for n in ["ep_create", "ep_destroy", "ep_plan", "ep_dispatch", "ep_combine", "ep_combine_backward",
+              "ep_dispatch_backward", "ep_reduce_replica_grads", "ep_get_plan", "ep_get_status"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from combine_ep_dispatch_03_b200 import ep
+
+    for name in _declared():
+        assert hasattr(L, name), name
+        assert name in ep.SIGNATURES, f"binding lacks {name}"
+
+
+def test_version_and_status_strings(L):
+    assert L.ep_version().decode().count(".") == 2
+    assert L.ep_status_string(0) == b"EP_OK"
+    assert L.ep_status_string(1) == b"EP_ERR_INVALID_ARG"
+
+
+def _cfg(**kw):
+    from combine_ep_dispatch_03_b200 import ep
+
+    base = dict(T=128, H=1024, E=16, K=2, R=4)
+    base.update(kw)
+    return ep.make_config(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({}, 0),
+    (dict(T=0), 0),
+    (dict(H=1004), 1),                # not a multiple of 8
+    (dict(H=1032, fp8=True), 1),      # fp8 needs 128-element blocks
+    (dict(E=18), 1),                  # E % R != 0
+    (dict(K=17), 1),                  # K > E
+    (dict(K=33, E=64), 1),            # K > 32
+    (dict(E=8192, R=8), 1),           # too many experts
+    (dict(mode="ll", ll_capacity=0), 1),
+    (dict(mode="ll", ll_capacity=64, balanced=True), 3),
+    (dict(balanced=True, replica_slots=5), 1),  # more than E/R slots
+    (dict(balanced=True, replica_slots=4), 0),
+    (dict(replica_slots=2), 1),       # slots without a plan
+    (dict(grad_elems_per_expert=6), 1),
+    (dict(T=-1), 1),
+])
+def test_validate(L, kw, status):
+    cfg = _cfg(**kw)
+    assert L.ep_validate_config(ctypes.byref(cfg)) == status
+
+
+def test_recv_rows_and_counts(L):
+    rows, n = ctypes.c_int64(), ctypes.c_int64()
+    cfg = _cfg()
+    assert L.ep_recv_rows(ctypes.byref(cfg), ctypes.byref(rows)) == 0 and rows.value == 256
+    assert L.ep_recv_counts_len(ctypes.byref(cfg), ctypes.byref(n)) == 0 and n.value == 16
+    cfg = _cfg(mode="ll", ll_capacity=100)
+    assert L.ep_recv_rows(ctypes.byref(cfg), ctypes.byref(rows)) == 0 and rows.value == 1600
+    cfg = _cfg(balanced=True)
+    assert L.ep_recv_counts_len(ctypes.byref(cfg), ctypes.byref(n)) == 0 and n.value == 4 * (4 + 4)
+    b = ctypes.c_size_t()
+    assert L.ep_workspace_bytes(ctypes.byref(cfg), ctypes.byref(b)) == 0 and b.value > 0
+
+
+def test_null_arguments_rejected_without_gpu(L):
+    assert L.ep_create(None, None) == 1
+    assert L.ep_destroy(None) == 0
+    assert L.ep_plan(None, None, None) == 1
+    assert L.ep_get_status(None, None, None) == 1
