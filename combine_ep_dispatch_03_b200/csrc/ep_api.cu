@@ -180,6 +180,7 @@ const char *ep_status_string(ep_status_t s) {
     case EP_ERR_UNSUPPORTED: return "EP_ERR_UNSUPPORTED";
     case EP_ERR_NOT_PLANNED: return "EP_ERR_NOT_PLANNED";
     case EP_ERR_NO_MEMORY: return "EP_ERR_NO_MEMORY";
+    case EP_ERR_TOO_LARGE: return "EP_ERR_TOO_LARGE";
     }
     return "EP_ERR_UNKNOWN";
 }

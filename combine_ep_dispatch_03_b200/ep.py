@@ -65,6 +65,7 @@ SIGNATURES = {
     "ep_get_plan": (ctypes.c_int, [_P, _P, _P, _P]),
     "ep_get_status": (ctypes.c_int, [_P, ctypes.POINTER(_I32), _P]),
     "ep_get_tensor": (ctypes.c_int, [_P, ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(_I64)]),
+    "ep_route_noalloc": (ctypes.c_int, [_P, _I32, _I32, _I32, _P, _P, _P, _P]),
 }
 
 _lib = None
@@ -135,6 +136,20 @@ def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, numel: int | 
 def _stream(stream: torch.cuda.Stream | None) -> ctypes.c_void_p:
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def route_noalloc(topk_idx: torch.Tensor, num_experts: int, dest_row: torch.Tensor, expert_counts: torch.Tensor,
+                  flags: torch.Tensor, stream=None) -> None:
+    """Routing without any device allocation (ep_route_noalloc): for callers
+    that own all device memory up front. All tensors are caller-provided
+    int32 CUDA tensors: topk_idx [T, K], dest_row [T*K], expert_counts [E],
+    flags [1]."""
+    T, K = topk_idx.shape
+    _check("ep_route_noalloc", lib().ep_route_noalloc(
+        _ptr(topk_idx, torch.int32, T * K, "topk_idx"), T, K, num_experts,
+        _ptr(dest_row, torch.int32, T * K, "dest_row"), _ptr(expert_counts, torch.int32, num_experts,
+                                                             "expert_counts"),
+        _ptr(flags, torch.int32, 1, "flags"), _stream(stream)))
 
 
 class _DeviceArray:

@@ -54,7 +54,8 @@ typedef enum ep_status {
     EP_ERR_CUDA = 2,        /* a CUDA runtime call or a launch failed */
     EP_ERR_UNSUPPORTED = 3, /* a valid but unsupported combination */
     EP_ERR_NOT_PLANNED = 4, /* a data call before the first ep_plan */
-    EP_ERR_NO_MEMORY = 5    /* workspace allocation failed */
+    EP_ERR_NO_MEMORY = 5,   /* workspace allocation failed */
+    EP_ERR_TOO_LARGE = 6    /* sizes beyond ep_route_noalloc's fixed scratch */
 } ep_status_t;
 
 /* Bits of the device status word (ep_get_status). */
@@ -218,6 +219,40 @@ ep_status_t ep_get_status(ep_handle_t *h, int32_t *flags, void *stream);
 /* Read-only device pointer and element count of one piece of the handle's
  * routing state (valid until the next ep_plan or ep_destroy). */
 ep_status_t ep_get_tensor(const ep_handle_t *h, ep_tensor_t which, const void **dptr, int64_t *numel);
+
+/* ---- routing without allocation ---------------------------------------- */
+
+/* Bytes of the fixed device scratch behind ep_route_noalloc (4 MiB); every
+ * GPU that loads the library holds this much until the process exits. */
+#define EP_NOALLOC_SCRATCH_BYTES (4 << 20)
+
+/* The routing pass of ep_plan for the plain HT layout, for callers that
+ * cannot allocate device memory: no handle, no cudaMalloc, no cudaFree and
+ * no allocating library call. This has no counterpart on the pages; it
+ * exists for hosts that reserve all device memory up front (for example a
+ * serving engine whose memory pool owns nearly all of HBM, where an extra
+ * allocation would fail, fragment the pool, or stall the device) and for
+ * plugin environments that forbid allocation after initialisation.
+ *
+ * Computes, exactly as ep_plan does for an HT configuration without a plan:
+ *   expert_counts[e] (device int32 [E]) = routed pairs of expert e;
+ *   dest_row[t*K+k] (device int32 [T*K]) = sum of the counts of experts
+ *     below e + the pair's stable index within e, or -1 if not routed;
+ *   *flags (one device int32) = EP_FLAG_* bits (bad or repeated ids).
+ * topk_idx: device int32 [T, K]; -1 marks a masked choice. T*K may be 0.
+ *
+ * Scratch lives in one static device array of EP_NOALLOC_SCRATCH_BYTES per
+ * GPU. Sizes whose scratch would not fit (about T*K above 500k pairs, fewer
+ * with many experts) return EP_ERR_TOO_LARGE and launch nothing; other
+ * argument errors return EP_ERR_INVALID_ARG. The first call on a device
+ * looks the array's device address up (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture. Every
+ * call shares the array and it keeps the last call's contents (each call
+ * writes every word it later reads, so nothing needs clearing), so calls
+ * whose work overlaps on the GPU (other streams, other host threads) race:
+ * order them. Asynchronous on `stream`, like ep_plan. */
+ep_status_t ep_route_noalloc(const int32_t *topk_idx, int32_t num_tokens, int32_t topk, int32_t num_experts,
+                             int32_t *dest_row, int32_t *expert_counts, int32_t *flags, void *stream);
 
 #ifdef __cplusplus
 }
