@@ -146,14 +146,23 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest value over all ranks (every rank must call it)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(step_bytes: float, ms_local: float, world: int):
+    """Whole-job GB/s when every rank moves step_bytes per step: all ranks'
+    bytes over the slowest rank's step time. Returns (GB/s, max ms)."""
+    ms = max_over_ranks(ms_local, world)
+    return world * step_bytes / (ms * 1e-3) / 1e9, ms
 
 
 # ------------------------------------------------------------------ workloads
@@ -315,7 +324,7 @@ def run_native(args):
     total_ms, per = timed(step, args.steps, args.warmup, stream)
     clocks = sampler.stop()
     barrier(world)
-    ms_step = max_over_ranks(total_ms / args.steps, world)
+    value, ms_step = weak_scaling_value(step_bytes, total_ms / args.steps, world)
     flags = step.h.status(stream)
 
     avg = {k: sum(v) / len(v) for k, v in per.items()}
@@ -330,7 +339,7 @@ def run_native(args):
     e2e = None if args.no_e2e else run_e2e(step, dev, stream, max(3, min(args.steps, 20)), world, step_bytes)
     big = step.h.recv_rows * step.H * (1 if wl["fp8"] else 2)
     result = {
-        "metric": METRIC, "value": round(world * step_bytes / (ms_step * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
@@ -401,10 +410,10 @@ def run_e2e(step: Step, dev, stream, steps, world, step_bytes):
             one()
         e.record(stream)
     torch.cuda.synchronize()
-    ms = max_over_ranks(s.elapsed_time(e) / steps, world)
+    value, ms = weak_scaling_value(step_bytes, s.elapsed_time(e) / steps, world)
     h2d = sum(src.numel() * src.element_size() for src, _ in ins)
     d2h = sum(src.numel() * src.element_size() for src, _ in outs)
-    return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+    return {"value": round(value, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": steps}
 
 
@@ -506,7 +515,7 @@ def run_reference(args):
         "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
-        "config": {"workload": workload, "T": T, "H": H, "E": E, "topk": K, "logical_ranks": R},
+        "config": {"workload": "ht_prefill", "T": T, "H": H, "E": E, "topk": K, "logical_ranks": R},
         "tokens_per_s": round(n / dt, 1),
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
