@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(256) k_dispatch_bf16(const uint4 *__restrict__
                                                        int32_t *__restrict__ recv_expert,
                                                        const int32_t *__restrict__ counts_src,
                                                        int32_t *__restrict__ counts_dst, int counts_len) {
+    pdl_wait();
+    pdl_launch_dependents();
     __shared__ int s_dest[kMaxTopk];
     const int t = blockIdx.x;
     const int64_t pb = (int64_t)t * K;
@@ -119,6 +121,8 @@ __global__ void __launch_bounds__(256) k_dispatch_fp8(const uint4 *__restrict__ 
                                                       float *__restrict__ recv_w, int32_t *__restrict__ recv_expert,
                                                       const int32_t *__restrict__ counts_src,
                                                       int32_t *__restrict__ counts_dst, int counts_len) {
+    pdl_wait();
+    pdl_launch_dependents();
     __shared__ int s_dest[kMaxTopk];
     const int t = blockIdx.x;
     const int64_t pb = (int64_t)t * K;
@@ -199,6 +203,8 @@ template <int CPT, bool UNIT>
 __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, const float *__restrict__ w,
                                                  const int32_t *__restrict__ dest_row, int K, int nvec,
                                                  uint4 *__restrict__ out) {
+    pdl_wait();
+    pdl_launch_dependents();
     __shared__ int s_dest[kMaxTopk];
     __shared__ float s_w[kMaxTopk];
     const int t = blockIdx.x;
@@ -249,6 +255,8 @@ template <int VPT>
 __global__ void __launch_bounds__(256) k_combine_bwd(const uint4 *__restrict__ g, const float *__restrict__ w,
                                                      const int32_t *__restrict__ dest_row, int K, int nvec,
                                                      uint4 *__restrict__ gy) {
+    pdl_wait();
+    pdl_launch_dependents();
     __shared__ int s_dest[kMaxTopk];
     __shared__ float s_w[kMaxTopk];
     const int t = blockIdx.x;
@@ -295,6 +303,8 @@ __global__ void __launch_bounds__(kRedThreads) k_replica_reduce(const float4 *__
                                                                 const int32_t *__restrict__ red_list,
                                                                 const int32_t *__restrict__ red_n, int R,
                                                                 int64_t G4) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int nred = *red_count;
     const int64_t chunk = (int64_t)kRedThreads * kRedUnroll;
     const int64_t per = (G4 + chunk - 1) / chunk;
@@ -349,10 +359,10 @@ void pick_shape(int n, int *per_thread, int *threads) {
 
 #define EPB_SWITCH_VPT(v, KERNEL, ...)                                                                               \
     switch (v) {                                                                                                     \
-    case 1: KERNEL<1><<<grid, threads, 0, st>>>(__VA_ARGS__); break;                                                 \
-    case 2: KERNEL<2><<<grid, threads, 0, st>>>(__VA_ARGS__); break;                                                 \
-    case 4: KERNEL<4><<<grid, threads, 0, st>>>(__VA_ARGS__); break;                                                 \
-    default: KERNEL<8><<<grid, threads, 0, st>>>(__VA_ARGS__); break;                                                \
+    case 1: err = launch_pdl(KERNEL<1>, grid, dim3(threads), 0, st, __VA_ARGS__); break;                             \
+    case 2: err = launch_pdl(KERNEL<2>, grid, dim3(threads), 0, st, __VA_ARGS__); break;                             \
+    case 4: err = launch_pdl(KERNEL<4>, grid, dim3(threads), 0, st, __VA_ARGS__); break;                             \
+    default: err = launch_pdl(KERNEL<8>, grid, dim3(threads), 0, st, __VA_ARGS__); break;                            \
     }
 
 } // namespace
@@ -368,6 +378,7 @@ cudaError_t launch_dispatch(const Dims &d, const Workspace &ws, const void *x, c
     }
     const dim3 grid(d.T);
     int per, threads;
+    cudaError_t err = cudaSuccess;
     if (d.fp8) {
         const int nchunk = d.H / 16;
         pick_shape(nchunk, &per, &threads);
@@ -380,7 +391,7 @@ cudaError_t launch_dispatch(const Dims &d, const Workspace &ws, const void *x, c
         EPB_SWITCH_VPT(per, k_dispatch_bf16, (const uint4 *)x, topk_idx, topk_w, ws.dest_row, d.K, nvec,
                        (uint4 *)recv_x, recv_w, recv_expert, ws.recv_counts, recv_counts, d.counts_len);
     }
-    return cudaGetLastError();
+    return err;
 }
 
 cudaError_t launch_combine_backward(const Dims &d, const Workspace &ws, const void *grad_out, const float *topk_w,
@@ -389,10 +400,11 @@ cudaError_t launch_combine_backward(const Dims &d, const Workspace &ws, const vo
     const dim3 grid(d.T);
     const int nvec = d.H / 8;
     int per, threads;
+    cudaError_t err = cudaSuccess;
     pick_shape(nvec, &per, &threads);
     EPB_SWITCH_VPT(per, k_combine_bwd, (const uint4 *)grad_out, topk_w, ws.dest_row, d.K, nvec,
                    (uint4 *)grad_expert_out);
-    return cudaGetLastError();
+    return err;
 }
 
 cudaError_t launch_combine(const Dims &d, const Workspace &ws, const void *y, const float *topk_w, void *out,
@@ -404,22 +416,22 @@ cudaError_t launch_combine(const Dims &d, const Workspace &ws, const void *y, co
     pick_shape(nvec, &per, &threads);
     const uint4 *yy = (const uint4 *)y;
     uint4 *oo = (uint4 *)out;
+    const dim3 block(threads);
     if (topk_w) {
         switch (per) {
-        case 1: k_combine<1, false><<<grid, threads, 0, st>>>(yy, topk_w, ws.dest_row, d.K, nvec, oo); break;
-        case 2: k_combine<2, false><<<grid, threads, 0, st>>>(yy, topk_w, ws.dest_row, d.K, nvec, oo); break;
-        case 4: k_combine<4, false><<<grid, threads, 0, st>>>(yy, topk_w, ws.dest_row, d.K, nvec, oo); break;
-        default: k_combine<8, false><<<grid, threads, 0, st>>>(yy, topk_w, ws.dest_row, d.K, nvec, oo); break;
-        }
-    } else {
-        switch (per) {
-        case 1: k_combine<1, true><<<grid, threads, 0, st>>>(yy, nullptr, ws.dest_row, d.K, nvec, oo); break;
-        case 2: k_combine<2, true><<<grid, threads, 0, st>>>(yy, nullptr, ws.dest_row, d.K, nvec, oo); break;
-        case 4: k_combine<4, true><<<grid, threads, 0, st>>>(yy, nullptr, ws.dest_row, d.K, nvec, oo); break;
-        default: k_combine<8, true><<<grid, threads, 0, st>>>(yy, nullptr, ws.dest_row, d.K, nvec, oo); break;
+        case 1: return launch_pdl(k_combine<1, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, oo);
+        case 2: return launch_pdl(k_combine<2, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, oo);
+        case 4: return launch_pdl(k_combine<4, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, oo);
+        default: return launch_pdl(k_combine<8, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, oo);
         }
     }
-    return cudaGetLastError();
+    const float *none = nullptr;
+    switch (per) {
+    case 1: return launch_pdl(k_combine<1, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, oo);
+    case 2: return launch_pdl(k_combine<2, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, oo);
+    case 4: return launch_pdl(k_combine<4, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, oo);
+    default: return launch_pdl(k_combine<8, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, oo);
+    }
 }
 
 cudaError_t launch_replica_reduce(const Dims &d, const Workspace &ws, const float *rep, float *owner,
@@ -427,9 +439,9 @@ cudaError_t launch_replica_reduce(const Dims &d, const Workspace &ws, const floa
     const int64_t G4 = d.G / 4;
     if (G4 == 0) return cudaSuccess;
     const int grid = num_sms() * 8;
-    k_replica_reduce<<<grid, kRedThreads, 0, st>>>((const float4 *)rep, (float4 *)owner, ws.red_experts,
-                                                   ws.red_count, ws.red_list, ws.red_n, d.R, G4);
-    return cudaGetLastError();
+    return launch_pdl(k_replica_reduce, dim3(grid), dim3(kRedThreads), 0, st, (const float4 *)rep, (float4 *)owner,
+                      (const int32_t *)ws.red_experts, (const int32_t *)ws.red_count, (const int32_t *)ws.red_list,
+                      (const int32_t *)ws.red_n, d.R, G4);
 }
 
 } // namespace epb

@@ -59,9 +59,9 @@ ep_status_t derive_dims(const ep_config_t *c, Dims *d) {
     }
     d->P = c->balanced ? R + 1 : 1;
     d->nx_max = c->balanced ? R * d->S + E : 0;
-    int64_t wt = (L + kMaxTiles - 1) / kMaxTiles;
-    wt = (wt + 31) / 32 * 32;
-    d->wt = (int)(wt < kMinTilePairs ? kMinTilePairs : (wt > kMaxTilePairs ? kMaxTilePairs : wt));
+    d->wt_log2 = 7; // tiles of 2^7 .. 2^11 pairs, at most about kMaxTiles of them
+    while ((1 << d->wt_log2) < kMaxTilePairs && ((int64_t)kMaxTiles << d->wt_log2) < L) ++d->wt_log2;
+    d->wt = 1 << d->wt_log2;
     d->ntiles = (int)((L + d->wt - 1) / d->wt);
     d->nhist = (d->ntiles + kRouteWarps - 1) / kRouteWarps;
     const int64_t per_cta = (int64_t)kRouteThreads * kAssignPer; // pairs per assignment CTA
@@ -80,6 +80,7 @@ static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
     X(dest_row, d.L > 0 ? d.L : 1)                                                                                    \
     X(packed, d.L > 0 ? d.L : 1)                                                                                      \
     X(blk, (int64_t)d.E * (d.ntiles > 0 ? d.ntiles : 1))                                                              \
+    X(blk_cta, (int64_t)d.E * (d.nhist > 0 ? d.nhist : 1))                                                            \
     X(tile_flags, d.nhist > 0 ? d.nhist : 1)                                                                          \
     X(cnt, d.E)                                                                                                       \
     X(recv_counts, d.counts_len)                                                                                      \

@@ -12,12 +12,12 @@ namespace epb {
 // Routing: each warp of the histogram kernel owns a "warp tile" of
 // consecutive (token, k) pairs; tiles grow with the batch so that there are
 // at most about kMaxTiles of them.
-constexpr int kMinTilePairs = 128;
 constexpr int kMaxTilePairs = 2048;
 constexpr int kMaxTiles = 1024;
 constexpr int kRouteThreads = 256;
 constexpr int kAssignPer = 4;             // pairs per thread of the assignment kernel
 constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kRouteWarpsLog2 = 3;
 constexpr int kPlanThreads = 1024;
 constexpr int kMaxExperts = 4096;
 constexpr int kMaxTopk = 32;
@@ -30,7 +30,8 @@ constexpr int kSmallMaxExperts = 512;     // ... and experts (plain layouts only
 struct Workspace {
     int32_t *dest_row;       // [T*K]: receive-buffer row of each pair, -1 if none
     int32_t *packed;         // [T*K]: expert | rank-in-tile << 16, 0xffff if not routed
-    int32_t *blk;            // [ntiles][E]: per-tile counts, then per-tile bases
+    int32_t *blk;            // [ntiles][E]: each tile's base within its CTA's tiles
+    int32_t *blk_cta;        // [nhist][E]: per-CTA counts, then bases over CTAs
     uint32_t *tile_flags;    // [nhist]: status bits seen by each histogram CTA
     int32_t *cnt;            // [E]
     int32_t *recv_counts;    // [R*(g+S)] (HT) or [E] (LL)
@@ -61,7 +62,7 @@ struct Dims {
     int64_t L;               // T*K pairs
     int64_t rows;            // receive-buffer rows
     int64_t G;               // replica-gradient elements per expert
-    int wt;                  // pairs per warp tile (a multiple of 32)
+    int wt, wt_log2;         // pairs per warp tile (a power of two, >= 128)
     int ntiles, nhist;       // warp tiles, histogram CTAs
     int nassign;             // CTAs of the slot-assignment kernel
     int P;                   // planner scratch pieces per expert (R+1 with a plan)
@@ -96,6 +97,29 @@ cudaError_t launch_replica_reduce(const Dims &d, const Workspace &ws, const floa
                                   cudaStream_t st);
 
 int num_sms();
+
+// Programmatic dependent launch: every kernel of the library waits for the
+// grid before it in the stream to complete (and its writes to be visible)
+// before touching memory, and lets the next grid launch as soon as all of its
+// own CTAs are running, so launch latency overlaps the previous kernel's tail.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 } // namespace epb
 

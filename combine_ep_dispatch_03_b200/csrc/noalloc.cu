@@ -29,6 +29,7 @@ size_t scratch_need(const Dims &d) {
     const size_t i4 = sizeof(int32_t);
     return al256(i4 * (size_t)(d.L > 0 ? d.L : 1))                                   // packed
            + al256(i4 * (size_t)d.E * (d.ntiles > 0 ? d.ntiles : 1))                 // blk
+           + al256(i4 * (size_t)d.E * (d.nhist > 0 ? d.nhist : 1))                   // blk_cta
            + al256(i4 * (size_t)(d.nhist > 0 ? d.nhist : 1))                         // tile_flags
            + 3 * al256(i4 * (size_t)d.E)                                             // recv_counts, base0, len0
            + 3 * al256(i4 * 2);                                                      // rank_load, rank_off, red_count
@@ -81,6 +82,7 @@ extern "C" ep_status_t ep_route_noalloc(const int32_t *topk_idx, int32_t num_tok
     };
     ws.packed = take(sizeof(int32_t) * (size_t)(d.L > 0 ? d.L : 1));
     ws.blk = take(sizeof(int32_t) * (size_t)d.E * (d.ntiles > 0 ? d.ntiles : 1));
+    ws.blk_cta = take(sizeof(int32_t) * (size_t)d.E * (d.nhist > 0 ? d.nhist : 1));
     ws.tile_flags = (uint32_t *)take(sizeof(int32_t) * (size_t)(d.nhist > 0 ? d.nhist : 1));
     ws.recv_counts = take(sizeof(int32_t) * (size_t)d.E);
     ws.base0 = take(sizeof(int32_t) * (size_t)d.E);

@@ -407,12 +407,15 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
 // same tile with the same expert), 0xffff otherwise. cnt_tile[tile][e].
 __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const int32_t *__restrict__ idx, Dims d,
                                                                Workspace ws) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int32_t sm[];
     __shared__ uint32_t s_fl;
     const int E = d.E, K = d.K, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int tile = blockIdx.x * kRouteWarps + w;
-    int32_t *my = sm + w * (E + d.wt);   // [E] counters of this warp's tile
-    int32_t *ids = my + E;               // [wt] the tile's expert ids
+    const int row = E + d.wt;           // shared memory per warp
+    int32_t *my = sm + w * row;         // [E] counters of this warp's tile
+    int32_t *ids = my + E;              // [wt] the tile's expert ids
     if (threadIdx.x == 0) s_fl = 0;
     const int64_t lo = (int64_t)tile * d.wt, hi = min(d.L, lo + d.wt);
     const int n = (int)max((int64_t)0, hi - lo);
@@ -421,24 +424,35 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const int32_t *__r
     for (int i = lane; i < n; i += 32) ids[i] = __ldg(idx + lo + i);
     __syncthreads();
     uint32_t fl = 0;
+    // When K divides 32, every 32-pair step holds whole tokens (tiles start at
+    // multiples of 32), so a repeated id is a lane whose (expert, token in
+    // step) key matches a lower lane's. Otherwise the earlier choices of the
+    // token are compared one by one; k, the lane's choice index, is kept up to
+    // date in 32-bit arithmetic.
+    const bool whole_tokens = (32 % K) == 0;
+    const int step_k = 32 % K;
+    int k = (int)(lo % K) + lane % K;
+    if (k >= K) k -= K;
     for (int base = 0; base < n; base += 32) { // warp-uniform
         const int i = base + lane;
-        int e = -1;
-        if (i < n) {
-            e = ids[i];
-            const int k = (int)((lo + i) % K);
-            if (e == -1) {
-            } else if (e < 0 || e >= E) {
-                fl |= EP_FLAG_BAD_EXPERT_ID;
+        int e = i < n ? ids[i] : -1;
+        if (e != -1 && (e < 0 || e >= E)) {
+            fl |= EP_FLAG_BAD_EXPERT_ID;
+            e = -1;
+        }
+        if (whole_tokens) {
+            const unsigned tok = __match_any_sync(kFull, e >= 0 ? (e << 5) | (lane / K) : -1 - lane);
+            if (e >= 0 && (tok & lanemask_lt()) != 0) {
+                fl |= EP_FLAG_DUP_EXPERT_ID;
                 e = -1;
-            } else {
-                for (int k2 = 1; k2 <= k; ++k2) {
-                    const int prev = i - k2 >= 0 ? ids[i - k2] : __ldg(idx + lo + i - k2); // token may start in the previous tile
-                    if (prev == e) {
-                        fl |= EP_FLAG_DUP_EXPERT_ID;
-                        e = -1;
-                        break;
-                    }
+            }
+        } else if (e >= 0) {
+            for (int k2 = 1; k2 <= k; ++k2) {
+                const int prev = i - k2 >= 0 ? ids[i - k2] : __ldg(idx + lo + i - k2); // token may start in the previous tile
+                if (prev == e) {
+                    fl |= EP_FLAG_DUP_EXPERT_ID;
+                    e = -1;
+                    break;
                 }
             }
         }
@@ -450,11 +464,22 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const int32_t *__r
         if (e >= 0 && lower == 0) my[e] += __popc(peers);
         __syncwarp();
         if (i < n) ws.packed[lo + i] = packed;
+        k += step_k;
+        if (k >= K) k -= K;
     }
-    if (n > 0)
-        for (int i = lane; i < E; i += 32) ws.blk[(int64_t)tile * E + i] = my[i];
     block_or(fl, &s_fl);
     __syncthreads();
+    // each tile's base among this CTA's tiles, and the CTA's totals
+    const int tile0 = blockIdx.x * kRouteWarps;
+    const int ntile = min(kRouteWarps, d.ntiles - tile0);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int ww = 0; ww < ntile; ++ww) {
+            ws.blk[(int64_t)(tile0 + ww) * E + e] = run;
+            run += sm[ww * row + e];
+        }
+        ws.blk_cta[(int64_t)blockIdx.x * E + e] = run;
+    }
     if (threadIdx.x == 0) ws.tile_flags[blockIdx.x] = s_fl;
 }
 
@@ -464,6 +489,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const int32_t *__r
 //    CTA that finishes last builds it
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kPlanThreads) k_route_scan(Dims d, Workspace ws) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int32_t sm[];
     __shared__ int32_t s_warp[33];
     __shared__ int32_t s_part[32][33];
@@ -471,15 +498,15 @@ __global__ void __launch_bounds__(kPlanThreads) k_route_scan(Dims d, Workspace w
     __shared__ int s_last;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, tid = threadIdx.x, nth = blockDim.x;
     const int e = blockIdx.x * 32 + lane;
-    const int chunk = (d.ntiles + 31) / 32;
-    const int t0 = min(d.ntiles, w * chunk), t1 = min(d.ntiles, t0 + chunk);
+    const int chunk = (d.nhist + 31) / 32; // rows: one per histogram CTA
+    const int t0 = min(d.nhist, w * chunk), t1 = min(d.nhist, t0 + chunk);
     constexpr int B = 16; // loads in flight per thread
     int sum = 0;
     if (e < d.E) {
         for (int t = t0; t < t1; t += B) {
             int v[B];
 #pragma unroll
-            for (int u = 0; u < B; ++u) v[u] = t + u < t1 ? ws.blk[(int64_t)(t + u) * d.E + e] : 0;
+            for (int u = 0; u < B; ++u) v[u] = t + u < t1 ? ws.blk_cta[(int64_t)(t + u) * d.E + e] : 0;
 #pragma unroll
             for (int u = 0; u < B; ++u) sum += v[u];
         }
@@ -492,10 +519,10 @@ __global__ void __launch_bounds__(kPlanThreads) k_route_scan(Dims d, Workspace w
         for (int t = t0; t < t1; t += B) {
             int v[B];
 #pragma unroll
-            for (int u = 0; u < B; ++u) v[u] = t + u < t1 ? ws.blk[(int64_t)(t + u) * d.E + e] : 0;
+            for (int u = 0; u < B; ++u) v[u] = t + u < t1 ? ws.blk_cta[(int64_t)(t + u) * d.E + e] : 0;
 #pragma unroll
             for (int u = 0; u < B; ++u) {
-                if (t + u < t1) ws.blk[(int64_t)(t + u) * d.E + e] = run;
+                if (t + u < t1) ws.blk_cta[(int64_t)(t + u) * d.E + e] = run;
                 run += v[u];
             }
         }
@@ -529,6 +556,8 @@ __global__ void __launch_bounds__(kPlanThreads) k_route_scan(Dims d, Workspace w
 // 3. destination rows: j = tile base + rank in tile, then the layout tables
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspace ws) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int32_t sm[];
     __shared__ int32_t s_warp[33];
     __shared__ uint32_t s_fl;
@@ -579,7 +608,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspac
     for (int u = 0; u < kAssignPer; ++u) {
         const int64_t p = p0 + (int64_t)u * nth;
         const int e = pk[u] & 0xffff;
-        jb[u] = e != 0xffff ? ws.blk[(p / d.wt) * E + e] : 0;
+        const int64_t tile = p >> d.wt_log2;
+        jb[u] = e != 0xffff ? ws.blk_cta[(tile >> kRouteWarpsLog2) * E + e] + ws.blk[tile * E + e] : 0;
     }
 #pragma unroll
     for (int u = 0; u < kAssignPer; ++u) {
@@ -608,6 +638,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspac
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__restrict__ idx, Dims d,
                                                                 Workspace ws) {
+    pdl_wait();
+    pdl_launch_dependents();
     extern __shared__ int32_t sm[];
     __shared__ int32_t s_warp[33];
     __shared__ uint32_t s_fl;
@@ -685,18 +717,15 @@ cudaError_t launch_plan(const Dims &d, const Workspace &ws, const int32_t *topk_
         attrs_set[dev] = true;
     }
     cudaError_t err;
-    if (route_use_small(d)) {
-        k_route_small<<<1, kSmallThreads, route_smem_small(d), st>>>(topk_idx, d, ws);
-        return cudaGetLastError();
-    }
+    if (route_use_small(d))
+        return launch_pdl(k_route_small, dim3(1), dim3(kSmallThreads), route_smem_small(d), st, topk_idx, d, ws);
     if (d.L > 0) {
-        k_route_hist<<<d.nhist, kRouteThreads, route_smem_hist(d), st>>>(topk_idx, d, ws);
-        if ((err = cudaGetLastError()) != cudaSuccess) return err;
+        err = launch_pdl(k_route_hist, dim3(d.nhist), dim3(kRouteThreads), route_smem_hist(d), st, topk_idx, d, ws);
+        if (err != cudaSuccess) return err;
     }
-    k_route_scan<<<(d.E + 31) / 32, kPlanThreads, route_smem_layout(d), st>>>(d, ws);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    k_route_assign<<<d.nassign, kRouteThreads, route_smem_assign(d), st>>>(d, ws);
-    return cudaGetLastError();
+    err = launch_pdl(k_route_scan, dim3((d.E + 31) / 32), dim3(kPlanThreads), route_smem_layout(d), st, d, ws);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(k_route_assign, dim3(d.nassign), dim3(kRouteThreads), route_smem_assign(d), st, d, ws);
 }
 
 int plan_launches(const Dims &d) { return route_use_small(d) ? 1 : (d.L > 0 ? 3 : 2); }
