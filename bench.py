@@ -266,29 +266,38 @@ class Step:
         return plan_launches(self.h) + len(self.calls) - 1
 
 
-def timed(step: Step, steps, warmup, stream):
-    """Warm-up, then `steps` steps with CUDA events between the calls on the
-    launching stream. Returns (total_ms, {call: [ms per step]})."""
+def timed(step: Step, steps, warmup, stream, breakdown_steps=None):
+    """Warm-up, then `steps` steps back to back between two CUDA events on the
+    launching stream (the step time), then `breakdown_steps` more with an
+    event between every two calls (the per-call split; events between calls
+    stop consecutive kernels from overlapping their launches, so this loop
+    runs slightly slower). Returns (total_ms, {call: [ms per step]})."""
     import torch
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):
             step.run(stream)
     torch.cuda.synchronize()
-    n = len(step.calls)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         start.record(stream)
-        for s in range(steps):
+        for _ in range(steps):
+            step.run(stream)
+        end.record(stream)
+    torch.cuda.synchronize()
+    total = start.elapsed_time(end)
+    nb = steps if breakdown_steps is None else breakdown_steps
+    n = len(step.calls)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(nb)]
+    with torch.cuda.stream(stream):
+        for s in range(nb):
             ev[s][0].record(stream)
             for i, (_, f) in enumerate(step.calls):
                 f(stream)
                 ev[s][i + 1].record(stream)
-        end.record(stream)
     torch.cuda.synchronize()
     per = {name: [e[i].elapsed_time(e[i + 1]) for e in ev] for i, (name, _) in enumerate(step.calls)}
-    return start.elapsed_time(end), per
+    return total, per
 
 
 def run_native(args):
@@ -321,7 +330,7 @@ def run_native(args):
     barrier(world)
     torch.cuda.synchronize()
     sampler.start()
-    total_ms, per = timed(step, args.steps, args.warmup, stream)
+    total_ms, per = timed(step, args.steps, args.warmup, stream, min(args.steps, 50))
     clocks = sampler.stop()
     barrier(world)
     value, ms_step = weak_scaling_value(step_bytes, total_ms / args.steps, world)
@@ -356,6 +365,7 @@ def run_native(args):
         "frac_of_hbm": round(step_bytes / (ms_step * 1e-3) / 1e9 / peak, 4),
         "frac_of_8tbs_nominal": round(step_bytes / (ms_step * 1e-3) / 1e9 / 8000.0, 4),
         "per_call_us": {k: round(v * 1e3, 2) for k, v in avg.items()},
+        "per_call_note": "separate loop with an event between calls (blocks launch overlap)",
         "per_call_gbs": {k: round(nbytes[k] / (avg[k] * 1e-3) / 1e9, 1) for k in avg},
         "bytes_per_step": step_bytes,
         "roofline": roofline,

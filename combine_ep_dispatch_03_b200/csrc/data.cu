@@ -68,8 +68,7 @@ __global__ void __launch_bounds__(256) k_dispatch_bf16(const uint4 *__restrict__
                                                        int32_t *__restrict__ recv_expert,
                                                        const int32_t *__restrict__ counts_src,
                                                        int32_t *__restrict__ counts_dst, int counts_len) {
-    pdl_wait();
-    pdl_launch_dependents();
+    pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     __shared__ int s_dest[kMaxTopk];
     const int t = blockIdx.x;
     const int64_t pb = (int64_t)t * K;
@@ -121,8 +120,7 @@ __global__ void __launch_bounds__(256) k_dispatch_fp8(const uint4 *__restrict__ 
                                                       float *__restrict__ recv_w, int32_t *__restrict__ recv_expert,
                                                       const int32_t *__restrict__ counts_src,
                                                       int32_t *__restrict__ counts_dst, int counts_len) {
-    pdl_wait();
-    pdl_launch_dependents();
+    pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     __shared__ int s_dest[kMaxTopk];
     const int t = blockIdx.x;
     const int64_t pb = (int64_t)t * K;
@@ -203,8 +201,7 @@ template <int CPT, bool UNIT>
 __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, const float *__restrict__ w,
                                                  const int32_t *__restrict__ dest_row, int K, int nvec,
                                                  uint4 *__restrict__ out) {
-    pdl_wait();
-    pdl_launch_dependents();
+    pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     __shared__ int s_dest[kMaxTopk];
     __shared__ float s_w[kMaxTopk];
     const int t = blockIdx.x;
@@ -255,8 +252,7 @@ template <int VPT>
 __global__ void __launch_bounds__(256) k_combine_bwd(const uint4 *__restrict__ g, const float *__restrict__ w,
                                                      const int32_t *__restrict__ dest_row, int K, int nvec,
                                                      uint4 *__restrict__ gy) {
-    pdl_wait();
-    pdl_launch_dependents();
+    pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     __shared__ int s_dest[kMaxTopk];
     __shared__ float s_w[kMaxTopk];
     const int t = blockIdx.x;
@@ -303,8 +299,7 @@ __global__ void __launch_bounds__(kRedThreads) k_replica_reduce(const float4 *__
                                                                 const int32_t *__restrict__ red_list,
                                                                 const int32_t *__restrict__ red_n, int R,
                                                                 int64_t G4) {
-    pdl_wait();
-    pdl_launch_dependents();
+    pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     const int nred = *red_count;
     const int64_t chunk = (int64_t)kRedThreads * kRedUnroll;
     const int64_t per = (G4 + chunk - 1) / chunk;

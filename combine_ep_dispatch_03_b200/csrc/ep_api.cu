@@ -66,6 +66,16 @@ ep_status_t derive_dims(const ep_config_t *c, Dims *d) {
     d->nhist = (d->ntiles + kRouteWarps - 1) / kRouteWarps;
     const int64_t per_cta = (int64_t)kRouteThreads * kAssignPer; // pairs per assignment CTA
     d->nassign = (int)(L > 0 ? (L + per_cta - 1) / per_cta : 1);
+    // cluster routing (plain layouts, batches small enough that each warp of a
+    // cluster of 8 takes at most kClusterMaxPairsPerWarp pairs: measured
+    // faster than the three-kernel path there, slower beyond)
+    if (!c->balanced) {
+        const int cs = 8;
+        const int64_t ppw = ((L + (int64_t)cs * kClusterWarps - 1) / ((int64_t)cs * kClusterWarps) + 31) / 32 * 32;
+        d->cl_size = cs;
+        d->cl_ppw = (int)(ppw > 0 ? ppw : 32);
+        if (ppw > kClusterMaxPairsPerWarp || route_smem_cluster(*d) > (size_t)kMaxRouteSmem) d->cl_size = 0;
+    }
     // the routing kernels keep their tables in one CTA's shared memory
     if (route_smem_layout(*d) > (size_t)kMaxRouteSmem || route_smem_assign(*d) > (size_t)kMaxRouteSmem ||
         route_smem_hist(*d) > (size_t)kMaxRouteSmem)

@@ -24,6 +24,9 @@ constexpr int kMaxTopk = 32;
 constexpr int kMaxRouteSmem = 200 * 1024; // dynamic shared memory cap of the routing kernels
 constexpr int kSmallMaxPairs = 1024;      // single-CTA routing up to this many pairs ...
 constexpr int kSmallMaxExperts = 512;     // ... and experts (plain layouts only)
+constexpr int kClusterThreads = 1024;     // one-launch cluster routing: threads per CTA
+constexpr int kClusterWarps = kClusterThreads / 32;
+constexpr int kClusterMaxPairsPerWarp = 128;
 
 // Device workspace of a handle: the routing state one ep_plan builds and the
 // later calls of the same forward/backward pass read.
@@ -65,6 +68,7 @@ struct Dims {
     int wt, wt_log2;         // pairs per warp tile (a power of two, >= 128)
     int ntiles, nhist;       // warp tiles, histogram CTAs
     int nassign;             // CTAs of the slot-assignment kernel
+    int cl_size, cl_ppw;     // cluster routing: CTAs (8 or 16, 0 = not used), pairs per warp
     int P;                   // planner scratch pieces per expert (R+1 with a plan)
     int nx_max;              // bound on extra pieces (R*S + E with a plan, else 0)
     int counts_len;          // recv_counts entries
@@ -81,7 +85,9 @@ size_t route_smem_layout(const Dims &d);
 size_t route_smem_assign(const Dims &d);
 size_t route_smem_hist(const Dims &d);
 size_t route_smem_small(const Dims &d);
+size_t route_smem_cluster(const Dims &d);
 bool route_use_small(const Dims &d);
+bool route_use_cluster(const Dims &d);
 int plan_launches(const Dims &d);
 
 // ---- launchers (each returns the launch's cudaError_t) ----
@@ -100,8 +106,10 @@ int num_sms();
 
 // Programmatic dependent launch: every kernel of the library waits for the
 // grid before it in the stream to complete (and its writes to be visible)
-// before touching memory, and lets the next grid launch as soon as all of its
-// own CTAs are running, so launch latency overlaps the previous kernel's tail.
+// before touching memory, so its launch overlaps the previous kernel's tail.
+// The short routing kernels also let the next grid launch as soon as all of
+// their CTAs run; the long row movers do not (their grids span many waves,
+// and an early launch of the next grid measured slower there).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 

@@ -20,9 +20,19 @@
 //   k_route_assign  per pair: stable index j = tile base + rank in tile ->
 //                   destination row through the layout tables (each CTA
 //                   computes the plain layouts' expert offsets itself)
-// Small batches without a plan, one kernel:
+// Batches up to 32768 pairs without a plan, one kernel:
+//   k_route_cluster a thread-block cluster of 8 CTAs; each CTA counts
+//                   and ranks its share of the pairs in shared memory, the
+//                   CTAs exchange per-expert totals through distributed
+//                   shared memory across two cluster barriers, and each then
+//                   assigns its own pairs
+// Tiny batches without a plan, one kernel:
 //   k_route_small   one CTA does all of the above in shared memory
+#include <cooperative_groups.h>
+
 #include "ep_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace epb {
 namespace {
@@ -634,6 +644,131 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspac
 }
 
 // ---------------------------------------------------------------------------
+// plain layouts, one cluster: counts, scan, layout and assignment in one launch
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t *__restrict__ idx, Dims d,
+                                                                    Workspace ws) {
+    pdl_wait();
+    pdl_launch_dependents();
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = (int)cluster.num_blocks(), r = (int)cluster.block_rank();
+    extern __shared__ int32_t sm[];
+    __shared__ int32_t s_warp[33];
+    __shared__ uint32_t s_fl, s_fl_all;
+    const int E = d.E, K = d.K, lane = threadIdx.x & 31, w = threadIdx.x >> 5, tid = threadIdx.x;
+    const int ppw = d.cl_ppw, ppc = ppw * kClusterWarps;
+    const int64_t c0 = (int64_t)r * ppc;
+    const int nc = (int)max((int64_t)0, min((int64_t)ppc, d.L - c0));
+    int32_t *s_wc = sm;                     // [warps][E]: per-warp counts, then per-warp bases
+    int32_t *s_tot = s_wc + kClusterWarps * E; // [E]: this CTA's totals (read by the other CTAs)
+    int32_t *s_cta = s_tot + E;             // [E]: pairs of each expert in lower-ranked CTAs
+    int32_t *s_cnt = s_cta + E;             // [E]: routed pairs per expert (whole batch)
+    int32_t *s_len = s_cnt + E;             // [E]: kept rows per expert
+    int32_t *s_off = s_len + E;             // [E]: first row of each expert
+    int32_t *s_ids = s_off + E;             // [ppc]: this CTA's expert ids
+    int32_t *s_pk = s_ids + ppc;            // [ppc]: packed (expert, rank in warp range)
+    if (tid == 0) {
+        s_fl = 0;
+        s_fl_all = 0;
+    }
+    for (int i = tid; i < kClusterWarps * E; i += blockDim.x) s_wc[i] = 0;
+    for (int i = tid; i < nc; i += blockDim.x) s_ids[i] = __ldg(idx + c0 + i);
+    __syncthreads();
+
+    // 1. per warp range: repeat check, rank among the range's pairs of the same expert
+    const int lo = w * ppw, hi = min(nc, lo + ppw);
+    int32_t *my = s_wc + w * E;
+    const bool whole_tokens = (32 % K) == 0; // ranges start at multiples of 32
+    const int step_k = 32 % K;
+    int k = (int)((c0 + lo) % K) + lane % K;
+    if (k >= K) k -= K;
+    uint32_t fl = 0;
+    for (int base = lo; base < hi; base += 32) { // warp-uniform
+        const int i = base + lane;
+        int e = i < hi ? s_ids[i] : -1;
+        if (e != -1 && (e < 0 || e >= E)) {
+            fl |= EP_FLAG_BAD_EXPERT_ID;
+            e = -1;
+        }
+        if (whole_tokens) {
+            const unsigned tok = __match_any_sync(kFull, e >= 0 ? (e << 5) | (lane / K) : -1 - lane);
+            if (e >= 0 && (tok & lanemask_lt()) != 0) {
+                fl |= EP_FLAG_DUP_EXPERT_ID;
+                e = -1;
+            }
+        } else if (e >= 0) {
+            for (int k2 = 1; k2 <= k; ++k2) {
+                const int prev = i - k2 >= 0 ? s_ids[i - k2] : __ldg(idx + c0 + i - k2);
+                if (prev == e) {
+                    fl |= EP_FLAG_DUP_EXPERT_ID;
+                    e = -1;
+                    break;
+                }
+            }
+        }
+        const unsigned peers = __match_any_sync(kFull, e >= 0 ? e : -1 - lane);
+        const unsigned lower = peers & lanemask_lt();
+        if (i < hi) s_pk[i] = e >= 0 ? (e | ((my[e] + __popc(lower)) << 16)) : 0xffff;
+        __syncwarp();
+        if (e >= 0 && lower == 0) my[e] += __popc(peers);
+        __syncwarp();
+        k += step_k;
+        if (k >= K) k -= K;
+    }
+    block_or(fl, &s_fl);
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) { // per-warp bases and the CTA's totals
+        int run = 0;
+        for (int ww = 0; ww < kClusterWarps; ++ww) {
+            const int v = s_wc[ww * E + e];
+            s_wc[ww * E + e] = run;
+            run += v;
+        }
+        s_tot[e] = run;
+    }
+    cluster.sync(); // every CTA's totals and flags are complete
+
+    // 2. totals of the whole batch and of the lower-ranked CTAs, read from
+    //    each CTA's shared memory
+    for (int e = tid; e < E; e += blockDim.x) {
+        int before = 0, all = 0;
+        for (int q = 0; q < C; ++q) {
+            const int v = cluster.map_shared_rank(s_tot, q)[e];
+            if (q < r) before += v;
+            all += v;
+        }
+        s_cta[e] = before;
+        s_cnt[e] = all;
+    }
+    if (tid < C) {
+        const uint32_t v = *cluster.map_shared_rank(&s_fl, tid);
+        if (v) atomicOr(&s_fl_all, v);
+    }
+    cluster.sync(); // no remote reads after this point; s_fl_all complete
+    if (tid == 0) s_fl = s_fl_all;
+    __syncthreads();
+
+    // 3. layout (every CTA computes it; CTA 0 publishes it) and assignment
+    const int total = plain_tables(d, s_cnt, s_len, s_off, s_warp, &s_fl);
+    if (r == 0) {
+        plain_outputs(d, ws, s_len, s_off, total);
+        for (int e = tid; e < E; e += blockDim.x) ws.cnt[e] = s_cnt[e];
+        __syncthreads();
+        if (tid == 0) *ws.flags = s_fl;
+    }
+    for (int i = lo + lane; i < hi; i += 32) {
+        const int pk = s_pk[i];
+        const int e = pk & 0xffff;
+        int dest = -1;
+        if (e != 0xffff) {
+            const int j = s_cta[e] + my[e] + (pk >> 16);
+            if (j < s_len[e]) dest = s_off[e] + j;
+        }
+        ws.dest_row[c0 + i] = dest;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // small batches, plain layouts: everything in one CTA
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__restrict__ idx, Dims d,
@@ -700,6 +835,45 @@ size_t route_smem_hist(const Dims &d) { return sizeof(int32_t) * (size_t)kRouteW
 
 size_t route_smem_small(const Dims &d) { return sizeof(int32_t) * ((size_t)(kSmallWarps + 3) * d.E + d.L); }
 
+size_t route_smem_cluster(const Dims &d) {
+    return sizeof(int32_t) * ((size_t)(kClusterWarps + 5) * d.E + 2 * (size_t)d.cl_ppw * kClusterWarps);
+}
+
+// Can a cluster of d.cl_size CTAs of this kernel be resident at once on this
+// device? (Asked once per device and size.)
+static bool cluster_fits(const Dims &d) {
+    static signed char ok[64][2][64]; // [device][size 8/16][smem in 4 KB steps], 0 unknown, 1 yes, -1 no
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    const size_t smem = route_smem_cluster(d);
+    const int si = d.cl_size == 16 ? 1 : 0, mi = (int)((smem + 4095) / 4096);
+    if (mi >= 64) return false;
+    if (ok[dev][si][mi] == 0) {
+        cudaFuncSetAttribute(k_route_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxRouteSmem);
+        cudaFuncSetAttribute(k_route_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(d.cl_size);
+        cfg.blockDim = dim3(kClusterThreads);
+        cfg.dynamicSmemBytes = (size_t)mi * 4096;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = d.cl_size;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, k_route_cluster, &cfg);
+        if (e != cudaSuccess) cudaGetLastError();
+        ok[dev][si][mi] = (e == cudaSuccess && n >= 1) ? 1 : -1;
+    }
+    return ok[dev][si][mi] == 1;
+}
+
+bool route_use_cluster(const Dims &d) {
+    return !d.balanced && d.cl_size > 0 && d.L > kSmallMaxPairs && cluster_fits(d);
+}
+
 bool route_use_small(const Dims &d) {
     return !d.balanced && d.L <= kSmallMaxPairs && d.E <= kSmallMaxExperts;
 }
@@ -717,6 +891,23 @@ cudaError_t launch_plan(const Dims &d, const Workspace &ws, const int32_t *topk_
         attrs_set[dev] = true;
     }
     cudaError_t err;
+    if (route_use_cluster(d)) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(d.cl_size);
+        cfg.blockDim = dim3(kClusterThreads);
+        cfg.dynamicSmemBytes = route_smem_cluster(d);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = d.cl_size;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        return cudaLaunchKernelEx(&cfg, k_route_cluster, topk_idx, d, ws);
+    }
     if (route_use_small(d))
         return launch_pdl(k_route_small, dim3(1), dim3(kSmallThreads), route_smem_small(d), st, topk_idx, d, ws);
     if (d.L > 0) {
@@ -728,6 +919,8 @@ cudaError_t launch_plan(const Dims &d, const Workspace &ws, const int32_t *topk_
     return launch_pdl(k_route_assign, dim3(d.nassign), dim3(kRouteThreads), route_smem_assign(d), st, d, ws);
 }
 
-int plan_launches(const Dims &d) { return route_use_small(d) ? 1 : (d.L > 0 ? 3 : 2); }
+int plan_launches(const Dims &d) {
+    return (route_use_cluster(d) || route_use_small(d)) ? 1 : (d.L > 0 ? 3 : 2);
+}
 
 } // namespace epb
