@@ -179,12 +179,20 @@ WORKLOADS = {
                         backward=True, G=7168 * 256),
     "tiny": dict(T=128, H=1024, E=16, K=2, R=4, mode="ht", cap=0, fp8=False, balanced=False, s=0.0,
                  backward=False, G=0),
+    # the two steps around the path (next rows): router top-K on the HT
+    # prefill logits, and replica weight prefetch under the large step's plan
+    # (stand-in weights: one 7168 x 2048 bf16 projection per expert)
+    "router": dict(T=32768, H=7168, E=256, K=8, R=8, mode="ht", cap=0, fp8=False, balanced=False, s=0.0,
+                   backward=False, G=0, kind="router"),
+    "prefetch": dict(T=131072, H=7168, E=384, K=8, R=16, mode="ht", cap=0, fp8=False, balanced=True, s=1.0,
+                     backward=False, G=0, kind="prefetch", wbytes=7168 * 2048 * 2),
 }
 HT = WORKLOADS["ht_prefill"]
 SWEEP = WORKLOADS["imbalance"]
 
 KERNEL_OF = {"plan": "k_route_*", "combine": "k_combine", "combine_backward": "k_combine_bwd",
-             "dispatch_backward": "k_combine", "replica_reduce": "k_replica_reduce"}
+             "dispatch_backward": "k_combine", "replica_reduce": "k_replica_reduce", "router": "k_router_topk",
+             "prefetch": "k_prefetch"}
 
 
 class Step:
@@ -199,6 +207,13 @@ class Step:
         self.wl = wl
         T, H, E, K, R = wl["T"], wl["H"], wl["E"], wl["K"], wl["R"]
         self.T, self.H, self.E, self.K, self.R = T, H, E, K, R
+        self.kind = wl.get("kind", "path")
+        if self.kind == "router":
+            self._init_router(wl, dev, seed, host_inputs)
+            return
+        if self.kind == "prefetch":
+            self._init_prefetch(wl, dev, seed)
+            return
         x = synth.tokens_bf16(T, H, seed=seed)
         idx, w = synth.routing(T, E, K, zipf_s=wl["s"], seed=seed)
         self.x_host = x.pin_memory() if host_inputs else x
@@ -238,6 +253,38 @@ class Step:
             self.outputs.append(self.gx)
         self.bytes = None
 
+    def _init_router(self, wl, dev, seed, host_inputs):
+        import torch
+
+        from combine_ep_dispatch_03_b200 import ep, synth
+
+        T, E, K = self.T, self.E, self.K
+        lg = synth.router_logits(T, E, zipf_s=wl["s"], seed=seed)
+        self.logits_host = lg.pin_memory() if host_inputs else lg
+        self.logits = self.logits_host.to(dev)
+        self.idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+        self.w = torch.empty((T, K), dtype=torch.float32, device=dev)
+        self.h = None
+        self.calls = [("router", lambda st: ep.router_topk(self.logits, K, self.idx, self.w, st))]
+        self.ins = [(self.logits_host, self.logits)]
+        self.outputs = [self.idx, self.w]
+
+    def _init_prefetch(self, wl, dev, seed):
+        import torch
+
+        from combine_ep_dispatch_03_b200 import ep, synth
+
+        T, E, K, R = self.T, self.E, self.K, self.R
+        idx, _ = synth.routing(T, E, K, zipf_s=wl["s"], seed=seed)
+        self.h = ep.Ep(T, 128, E, K, R, balanced=True)
+        self.h.plan(idx.to(dev))
+        nb = wl["wbytes"]
+        g = torch.Generator(device=dev).manual_seed(3000 + seed)
+        self.weights = torch.randint(0, 256, (E, nb), dtype=torch.uint8, device=dev, generator=g)
+        self.slots = torch.empty((R, self.h.S, nb), dtype=torch.uint8, device=dev)
+        self.calls = [("prefetch", lambda st: self.h.prefetch_replica_weights(self.weights, self.slots, st))]
+        self.ins, self.outputs = [], []
+
     def run(self, st):
         for _, f in self.calls:
             f(st)
@@ -247,6 +294,16 @@ class Step:
         self.run(st)
         st.synchronize()  # recv_counts is written on `st`
         T, H, K, wl = self.T, self.H, self.K, self.wl
+        if self.kind == "router":
+            self.placed = T * K
+            self.bytes = {"router": 4 * T * self.E + 8 * T * K}
+            return self.bytes
+        if self.kind == "prefetch":
+            rep, _ = self.h.get_plan(st)
+            used = sum(1 for e in rep if e >= 0)
+            self.placed = used
+            self.bytes = {"prefetch": 2 * wl["wbytes"] * used}
+            return self.bytes
         L = T * K
         placed = int(self.bufs["recv_counts"].sum().item())
         b = algorithmic_bytes(T, H, K, placed, wl["fp8"])
@@ -263,6 +320,8 @@ class Step:
     def launches(self):
         from combine_ep_dispatch_03_b200.ep import plan_launches
 
+        if self.kind != "path":
+            return len(self.calls)
         return plan_launches(self.h) + len(self.calls) - 1
 
 
@@ -334,19 +393,20 @@ def run_native(args):
     clocks = sampler.stop()
     barrier(world)
     value, ms_step = weak_scaling_value(step_bytes, total_ms / args.steps, world)
-    flags = step.h.status(stream)
+    flags = step.h.status(stream) if step.h is not None else 0
 
     avg = {k: sum(v) / len(v) for k, v in per.items()}
     peak, peak_kind = hbm_peak()
-    dom = max((k for k in avg if k != "plan"), key=lambda k: avg[k])
+    dom = max((k for k in avg if k != "plan" or len(avg) == 1), key=lambda k: avg[k])
     kname = KERNEL_OF.get(dom) or ("k_dispatch_fp8" if wl["fp8"] else "k_dispatch_bf16")
     achieved = nbytes[dom] / (avg[dom] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "call": dom, "kernel": kname, "achieved": round(achieved, 1), "peak": peak,
                 "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy)",
                 "traffic": committed_traffic(kname, name), "algorithmic_bytes_per_launch": nbytes[dom]}
 
-    e2e = None if args.no_e2e else run_e2e(step, dev, stream, max(3, min(args.steps, 20)), world, step_bytes)
-    big = step.h.recv_rows * step.H * (1 if wl["fp8"] else 2)
+    e2e = None if (args.no_e2e or step.kind == "prefetch") else run_e2e(step, dev, stream, max(3, min(args.steps, 20)),
+                                                                        world, step_bytes)
+    big = (step.h.recv_rows * step.H * (1 if wl["fp8"] else 2)) if step.kind == "path" else 4 * wl["T"] * wl["E"]
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -374,10 +434,11 @@ def run_native(args):
         "clocks": clocks,
         "device_flags": flags,
     }
-    if wl["balanced"] or wl["mode"] == "ht":
+    if step.kind == "path" and (wl["balanced"] or wl["mode"] == "ht"):
         load = step.h.tensor(ep.T_RANK_LOAD).cpu().tolist()
         result["rank_load_max_over_mean"] = round(max(load) / (sum(load) / len(load)), 4) if sum(load) else None
-    step.h.close()
+    if step.h is not None:
+        step.h.close()
     del step
     torch.cuda.empty_cache()
     if not args.no_sweep and args.workload == "ht_prefill":
@@ -398,9 +459,12 @@ def run_e2e(step: Step, dev, stream, steps, world, step_bytes):
     a backward pass) read back to pinned host memory, inside the timed region."""
     import torch
 
-    ins = [(step.x_host, step.xd), (step.idx_host, step.idxd), (step.w_host, step.wd)]
-    if step.wl["backward"]:
-        ins.append((step.gout_host, step.gout))
+    if step.kind == "path":
+        ins = [(step.x_host, step.xd), (step.idx_host, step.idxd), (step.w_host, step.wd)]
+        if step.wl["backward"]:
+            ins.append((step.gout_host, step.gout))
+    else:
+        ins = step.ins
     outs = [(o, torch.empty(o.shape, dtype=o.dtype).pin_memory()) for o in step.outputs]
 
     def one():

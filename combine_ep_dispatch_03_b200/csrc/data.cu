@@ -302,11 +302,11 @@ __global__ void __launch_bounds__(kRedThreads) k_replica_reduce(const float4 *__
     pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     const int nred = *red_count;
     const int64_t chunk = (int64_t)kRedThreads * kRedUnroll;
-    const int64_t per = (G4 + chunk - 1) / chunk;
-    const int64_t items = (int64_t)nred * per;
-    for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int per = (int)((G4 + chunk - 1) / chunk); // chunks per expert (host-checked to fit)
+    const int items = nred * per;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
         const int e = red_experts[it / per];
-        const int64_t base = (it % per) * chunk + threadIdx.x;
+        const int64_t base = (int64_t)(it % per) * chunk + threadIdx.x;
         const int n = red_n[e];
         const int32_t *lst = red_list + (int64_t)e * R;
         float4 *o = owner + (int64_t)e * G4;
@@ -334,6 +334,41 @@ __global__ void __launch_bounds__(kRedThreads) k_replica_reduce(const float4 *__
         for (int u = 0; u < kRedUnroll; ++u) {
             const int64_t i = base + (int64_t)u * kRedThreads;
             if (i < G4) o[i] = acc[u];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// replica weight prefetch: slots[r*S+s] = weights[replica_expert[r*S+s]] for
+// every filled slot; a persistent grid over (slot, chunk) items
+// ---------------------------------------------------------------------------
+constexpr int kCopyThreads = 256, kCopyUnroll = 4;
+
+__global__ void __launch_bounds__(kCopyThreads) k_prefetch(const uint4 *__restrict__ weights,
+                                                           uint4 *__restrict__ slots,
+                                                           const int32_t *__restrict__ replica_expert,
+                                                           const int32_t *__restrict__ slot_list,
+                                                           const int32_t *__restrict__ slot_count, int64_t V) {
+    pdl_wait(); // no early trigger: measured slower for these multi-wave grids
+    const int64_t chunk = (int64_t)kCopyThreads * kCopyUnroll;
+    const int per = (int)((V + chunk - 1) / chunk); // chunks per expert (host-checked to fit)
+    const int items = *slot_count * per;            // filled slots only
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+        const int sl = slot_list[it / per];
+        const int e = replica_expert[sl];
+        const int64_t base = (int64_t)(it % per) * chunk + threadIdx.x;
+        const uint4 *src = weights + (int64_t)e * V;
+        uint4 *dst = slots + (int64_t)sl * V;
+        uint4 v[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kCopyThreads;
+            if (i < V) v[u] = __ldcs(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kCopyThreads;
+            if (i < V) __stcs(dst + i, v[u]);
         }
     }
 }
@@ -427,6 +462,16 @@ cudaError_t launch_combine(const Dims &d, const Workspace &ws, const void *y, co
     case 4: return launch_pdl(k_combine<4, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, oo);
     default: return launch_pdl(k_combine<8, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, oo);
     }
+}
+
+cudaError_t launch_prefetch(const Dims &d, const Workspace &ws, const void *weights, int64_t bytes_per_expert,
+                            void *slots, cudaStream_t st) {
+    const int64_t V = bytes_per_expert / 16;
+    if (V == 0 || d.R * d.S == 0) return cudaSuccess;
+    const int grid = num_sms() * 8;
+    return launch_pdl(k_prefetch, dim3(grid), dim3(kCopyThreads), 0, st, (const uint4 *)weights, (uint4 *)slots,
+                      (const int32_t *)ws.replica_expert, (const int32_t *)ws.slot_list,
+                      (const int32_t *)ws.slot_count, V);
 }
 
 cudaError_t launch_replica_reduce(const Dims &d, const Workspace &ws, const float *rep, float *owner,

@@ -31,6 +31,8 @@ ep_status_t derive_dims(const ep_config_t *c, Dims *d) {
     if (c->balanced != 0 && c->balanced != 1) return EP_ERR_INVALID_ARG;
     if (c->fp8 && H % 128 != 0) return EP_ERR_INVALID_ARG;
     if (c->grad_elems_per_expert < 0 || c->grad_elems_per_expert % 4 != 0) return EP_ERR_INVALID_ARG;
+    // the reduce walks (expert, 4096-element chunk) items with 32-bit counters
+    if ((c->grad_elems_per_expert / 4096 + 1) * (int64_t)c->num_experts > INT32_MAX / 2) return EP_ERR_INVALID_ARG;
     const int g = E / R;
     const int64_t L = (int64_t)T * K;
     if (L > INT32_MAX / 2) return EP_ERR_INVALID_ARG;
@@ -97,6 +99,8 @@ static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
     X(rank_load, d.R)                                                                                                 \
     X(rank_off, d.R + 1)                                                                                              \
     X(replica_expert, d.R *(d.S > 0 ? d.S : 1))                                                                       \
+    X(slot_list, d.R *(d.S > 0 ? d.S : 1))                                                                            \
+    X(slot_count, 1)                                                                                                  \
     X(base0, d.E)                                                                                                     \
     X(len0, d.E)                                                                                                      \
     X(xoff, d.E + 1)                                                                                                  \
@@ -306,6 +310,22 @@ ep_status_t ep_reduce_replica_grads(ep_handle_t *h, const float *replica_grad, f
     if (h->d.G > 0 && (!replica_grad || !owner_grad || !aligned(replica_grad, 16) || !aligned(owner_grad, 16)))
         return EP_ERR_INVALID_ARG;
     if (launch_replica_reduce(h->d, h->ws, replica_grad, owner_grad, as_stream(stream)) != cudaSuccess)
+        return EP_ERR_CUDA;
+    return EP_OK;
+}
+
+ep_status_t ep_prefetch_replica_weights(ep_handle_t *h, const void *expert_weights, int64_t bytes_per_expert,
+                                        void *prefetch_slots, void *stream) {
+    if (!h) return EP_ERR_INVALID_ARG;
+    if (!h->d.balanced) return EP_ERR_UNSUPPORTED;
+    if (!h->planned) return EP_ERR_NOT_PLANNED;
+    if (bytes_per_expert <= 0 || bytes_per_expert % 16 != 0 || !expert_weights || !prefetch_slots ||
+        !aligned(expert_weights, 16) || !aligned(prefetch_slots, 16))
+        return EP_ERR_INVALID_ARG;
+    // (slot, 16 KB chunk) items are counted in 32 bits
+    if ((bytes_per_expert / 16384 + 1) * (int64_t)h->d.R * h->d.S > INT32_MAX / 2) return EP_ERR_INVALID_ARG;
+    if (launch_prefetch(h->d, h->ws, expert_weights, bytes_per_expert, prefetch_slots, as_stream(stream)) !=
+        cudaSuccess)
         return EP_ERR_CUDA;
     return EP_OK;
 }

@@ -21,6 +21,7 @@ constexpr int kRouteWarpsLog2 = 3;
 constexpr int kPlanThreads = 1024;
 constexpr int kMaxExperts = 4096;
 constexpr int kMaxTopk = 32;
+constexpr int kRouterMaxExperts = 1024;   // ep_router_topk keeps a token's logits in one warp's registers
 constexpr int kMaxRouteSmem = 200 * 1024; // dynamic shared memory cap of the routing kernels
 constexpr int kSmallMaxPairs = 1024;      // single-CTA routing up to this many pairs ...
 constexpr int kSmallMaxExperts = 512;     // ... and experts (plain layouts only)
@@ -41,6 +42,8 @@ struct Workspace {
     int32_t *rank_load;      // [R]
     int32_t *rank_off;       // [R+1]
     int32_t *replica_expert; // [max(R*S,1)]
+    int32_t *slot_list;      // [max(R*S,1)]: the filled replica slots (r*S+s), ascending
+    int32_t *slot_count;     // [1]
     int32_t *base0;          // [E]: row of stable index 0 of each expert (piece 0)
     int32_t *len0;           // [E]: stable indices [0, len0) live in piece 0
     int32_t *xoff;           // [E+1]: extra pieces of expert e: [xoff[e], xoff[e+1])
@@ -99,6 +102,8 @@ cudaError_t launch_combine_backward(const Dims &d, const Workspace &ws, const vo
                                     void *grad_expert_out, cudaStream_t st);
 cudaError_t launch_combine(const Dims &d, const Workspace &ws, const void *y, const float *topk_w, void *out,
                            cudaStream_t st);
+cudaError_t launch_prefetch(const Dims &d, const Workspace &ws, const void *weights, int64_t bytes_per_expert,
+                            void *slots, cudaStream_t st);
 cudaError_t launch_replica_reduce(const Dims &d, const Workspace &ws, const float *rep, float *owner,
                                   cudaStream_t st);
 

@@ -406,6 +406,15 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
         if (ws.red_n[e] > 0) ws.red_experts[s_list[e]] = e;
     if (tid == 0) *ws.red_count = nred;
     __syncthreads();
+    // the filled replica slots, ascending (the prefetch copies only these);
+    // s_slot_len is free again and serves as the flag array
+    for (int i = tid; i < R * S; i += nth) s_slot_len[i] = s_slot_e[i] >= 0 ? 1 : 0;
+    __syncthreads();
+    const int nslot = block_exscan(s_slot_len, R * S, s_warp);
+    for (int i = tid; i < R * S; i += nth)
+        if (s_slot_e[i] >= 0) ws.slot_list[s_slot_len[i]] = i;
+    if (tid == 0) *ws.slot_count = nslot;
+    __syncthreads();
 }
 
 // ---------------------------------------------------------------------------

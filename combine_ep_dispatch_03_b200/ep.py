@@ -62,10 +62,12 @@ SIGNATURES = {
     "ep_combine_backward": (ctypes.c_int, [_P, _P, _P, _P, _P]),
     "ep_dispatch_backward": (ctypes.c_int, [_P, _P, _P, _P]),
     "ep_reduce_replica_grads": (ctypes.c_int, [_P, _P, _P, _P]),
+    "ep_prefetch_replica_weights": (ctypes.c_int, [_P, _P, _I64, _P, _P]),
     "ep_get_plan": (ctypes.c_int, [_P, _P, _P, _P]),
     "ep_get_status": (ctypes.c_int, [_P, ctypes.POINTER(_I32), _P]),
     "ep_get_tensor": (ctypes.c_int, [_P, ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(_I64)]),
     "ep_route_noalloc": (ctypes.c_int, [_P, _I32, _I32, _I32, _P, _P, _P, _P]),
+    "ep_router_topk": (ctypes.c_int, [_P, _I32, _I32, _I32, _P, _P, _P]),
 }
 
 _lib = None
@@ -136,6 +138,15 @@ def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, numel: int | 
 def _stream(stream: torch.cuda.Stream | None) -> ctypes.c_void_p:
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def router_topk(logits: torch.Tensor, K: int, topk_idx: torch.Tensor, topk_w: torch.Tensor, stream=None) -> None:
+    """Top-K experts and renormalised softmax weights per token (ep_router_topk):
+    logits fp32 [T, E] -> topk_idx int32 [T, K], topk_w fp32 [T, K]."""
+    T, E = logits.shape
+    _check("ep_router_topk", lib().ep_router_topk(
+        _ptr(logits, torch.float32, T * E, "logits"), T, E, K, _ptr(topk_idx, torch.int32, T * K, "topk_idx"),
+        _ptr(topk_w, torch.float32, T * K, "topk_w"), _stream(stream)))
 
 
 def route_noalloc(topk_idx: torch.Tensor, num_experts: int, dest_row: torch.Tensor, expert_counts: torch.Tensor,
@@ -254,6 +265,15 @@ class Ep:
         _check("ep_reduce_replica_grads", lib().ep_reduce_replica_grads(
             self._h, _ptr(replica_grad, torch.float32, self.R * max(self.S, 1) * self.G, "replica_grad"),
             _ptr(owner_grad, torch.float32, self.E * self.G, "owner_grad"), _stream(stream)))
+
+    def prefetch_replica_weights(self, expert_weights, prefetch_slots, stream=None) -> None:
+        """Copy each filled replica slot's expert weights into it: expert_weights
+        [E, ...] and prefetch_slots [R, S, ...] of the same row size in bytes."""
+        nbytes = expert_weights.numel() * expert_weights.element_size() // self.E
+        if prefetch_slots.numel() * prefetch_slots.element_size() != self.R * max(self.S, 1) * nbytes:
+            raise ValueError("prefetch_slots must hold R*S rows of one expert's weights")
+        _check("ep_prefetch_replica_weights", lib().ep_prefetch_replica_weights(
+            self._h, _ptr(expert_weights), nbytes, _ptr(prefetch_slots), _stream(stream)))
 
     # -- inspection
     def get_plan(self, stream=None) -> tuple[list[int], list[int]]:

@@ -139,6 +139,20 @@ ep_status_t ep_destroy(ep_handle_t *h);
 
 /* ---- forward ----------------------------------------------------------- */
 
+/* Router top-K, the gating step that feeds ep_plan ("Ultra-Large MoE Models:
+ * Open-Source Evolution and Heterogeneous Inference Adaptation", §2.1 top-K
+ * routing and §3.1 the fused top-K routing operator). For every token t:
+ *   topk_idx[t, 0..K)  the K experts with the largest logits[t, :], in
+ *                      descending order of logit, a tie going to the lower id;
+ *   topk_w[t, k]       = exp(l_k - l_0) / sum_j exp(l_j - l_0) over the chosen
+ *                      logits l_k (= softmax over all E experts, renormalised
+ *                      over the K chosen), fp32, summed in k order.
+ * logits: device fp32 [T, E] row-major; outputs device int32 / fp32 [T, K].
+ * Needs E <= 1024 and K <= min(E, 32), else EP_ERR_INVALID_ARG. Logits must be
+ * finite. No handle; stream-ordered, no host sync. */
+ep_status_t ep_router_topk(const float *logits, int32_t num_tokens, int32_t num_experts, int32_t topk,
+                           int32_t *topk_idx, float *topk_w, void *stream);
+
 /* Routing for one forward pass (NCCL EP Fig. 5: the state it builds is
  * reused by dispatch, combine and both backward calls until the next
  * ep_plan). Clears the status word, then on the device:
@@ -205,6 +219,18 @@ ep_status_t ep_dispatch_backward(ep_handle_t *h, const void *grad_recv, void *gr
  * fp32. replica_grad: device fp32 [R, S, G]; owner_grad: fp32 [E, G], updated
  * in place; G = cfg.grad_elems_per_expert. Needs cfg.balanced. */
 ep_status_t ep_reduce_replica_grads(ep_handle_t *h, const float *replica_grad, float *owner_grad, void *stream);
+
+/* Replica weight prefetch (MoonEP article paras. 3 and 5: the planner picks
+ * redundant experts online and their weights are prefetched into dedicated
+ * prefetch slots of the receiving ranks). For every replica slot (r, s) the
+ * current plan fills with expert e:
+ *   prefetch_slots[r, s, :] = expert_weights[e, :]   (bytes_per_expert bytes)
+ * Empty slots are not written. expert_weights: device [E, bytes_per_expert];
+ * prefetch_slots: device [R, S, bytes_per_expert]; both 16-byte aligned and
+ * bytes_per_expert a positive multiple of 16. Reads the plan on the device:
+ * no host sync. Needs cfg.balanced. */
+ep_status_t ep_prefetch_replica_weights(ep_handle_t *h, const void *expert_weights, int64_t bytes_per_expert,
+                                        void *prefetch_slots, void *stream);
 
 /* ---- inspection (these synchronise the stream) ------------------------- */
 

@@ -57,6 +57,7 @@ def lib() -> ctypes.CDLL:
             "orc_e4m3_to_f32": (ctypes.c_float, [ctypes.c_uint8]),
             "orc_bf16_from_f32_n": (None, [P, i64, P]),
             "orc_e4m3_from_f32_n": (None, [P, i64, P]),
+            "orc_router_topk": (None, [i32, i32, i32, P, P, P]),
             "orc_route": (i32, [i32, i32, i32, P, P, P]),
             "orc_layout_ht": (None, [i32, i32, i32, P, P, P, P]),
             "orc_layout_ll": (i32, [i32, i32, i32, P, P, P]),
@@ -66,6 +67,7 @@ def lib() -> ctypes.CDLL:
             "orc_combine": (None, [i32, i32, i32, P, P, P, P]),
             "orc_combine_backward": (None, [i32, i32, i32, P, P, P, P]),
             "orc_replica_reduce": (None, [i32, i32, i32, i64, P, P, P]),
+            "orc_prefetch": (None, [i32, i32, i64, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(_lib, name)
@@ -130,6 +132,18 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     """bf16 bits -> float32 values (exact; the bits are the float's top half)."""
     b = np.asarray(b, dtype=np.uint16)
     return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------- router
+
+def router_topk(logits, K: int):
+    """(topk_idx [T, K] int32, topk_w [T, K] float32) from logits [T, E]."""
+    lg = _np(logits, np.float32)
+    T, E = lg.shape
+    idx = np.zeros((T, K), np.int32)
+    w = np.zeros((T, K), np.float32)
+    lib().orc_router_topk(T, E, K, _p(lg), _p(idx), _p(w))
+    return idx, w
 
 
 # ---------------------------------------------------------------- routing
@@ -242,4 +256,16 @@ def replica_reduce(replica_expert, rep, owner) -> np.ndarray:
     out = _np(owner, np.float32).copy()
     E, G = out.shape
     L.orc_replica_reduce(E, R, S, G, _p(re), _p(rep), _p(out))
+    return out
+
+
+def prefetch(replica_expert, weights, slots) -> np.ndarray:
+    """slots [R, S, B] bytes after copying each filled slot's expert weights
+    (weights [E, B] bytes); empty slots keep their contents."""
+    re = _np(replica_expert, np.int32)
+    R, S = re.shape
+    wt = np.ascontiguousarray(np.asarray(weights, dtype=np.uint8))
+    out = np.ascontiguousarray(np.asarray(slots, dtype=np.uint8)).copy()
+    B = wt.shape[1]
+    lib().orc_prefetch(R, S, B, _p(re), _p(wt), _p(out))
     return out

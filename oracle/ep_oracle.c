@@ -106,6 +106,41 @@ void orc_e4m3_from_f32_n(const float *v, int64_t n, uint8_t *out) {
 }
 
 /* ------------------------------------------------------------------ */
+/* Router: top-K of the gating logits   [Baidu article §2.1, §3.1]     */
+/* ------------------------------------------------------------------ */
+
+/* For each token, the K experts with the largest logits (ties: lower id
+ * first), in descending order, and their router weights: a softmax over all
+ * E logits renormalised over the K chosen ones, which is the softmax of the
+ * K chosen logits, w_k = exp(l_k - l_max) / sum_j exp(l_j - l_max), here in
+ * double precision, rounded to float once. */
+void orc_router_topk(int T, int E, int K, const float *logits, int32_t *idx, float *w) {
+    int *taken = (int *)malloc(sizeof(int) * (size_t)E);
+    double *ex = (double *)malloc(sizeof(double) * (size_t)K);
+    for (int t = 0; t < T; t++) {
+        const float *l = logits + (int64_t)t * E;
+        for (int e = 0; e < E; e++) taken[e] = 0;
+        for (int k = 0; k < K; k++) {
+            int best = -1;
+            for (int e = 0; e < E; e++) {
+                if (taken[e]) continue;
+                if (best < 0 || l[e] > l[best]) best = e; /* strict: the lower id wins a tie */
+            }
+            taken[best] = 1;
+            idx[(int64_t)t * K + k] = best;
+        }
+        double lmax = l[idx[(int64_t)t * K]], sum = 0.0;
+        for (int k = 0; k < K; k++) {
+            ex[k] = exp((double)l[idx[(int64_t)t * K + k]] - lmax);
+            sum += ex[k];
+        }
+        for (int k = 0; k < K; k++) w[(int64_t)t * K + k] = (float)(ex[k] / sum);
+    }
+    free(taken);
+    free(ex);
+}
+
+/* ------------------------------------------------------------------ */
 /* Routing: counts and stable slots   [NCCL-EP Table III; MoonEP para 4] */
 /* ------------------------------------------------------------------ */
 
@@ -460,6 +495,23 @@ void orc_combine_backward(int T, int K, int H, const uint16_t *g, const float *w
                 gy[(int64_t)row * H + i] = orc_bf16_from_f32(prod);
             }
         }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Replica weight prefetch   [MoonEP paras 3 and 5, prefetch slots]     */
+/* ------------------------------------------------------------------ */
+
+/* Every replica slot (r, s) that the plan fills with expert e receives a copy
+ * of e's weights: slots[r*S+s] = weights[e] (bytes_per_expert bytes each).
+ * Empty slots (replica_expert = -1) are left as they are. */
+void orc_prefetch(int R, int S, int64_t bytes_per_expert, const int32_t *replica_expert, const void *weights,
+                  void *slots) {
+    for (int sl = 0; sl < R * S; sl++) {
+        int e = replica_expert[sl];
+        if (e < 0) continue;
+        memcpy((char *)slots + (int64_t)sl * bytes_per_expert, (const char *)weights + (int64_t)e * bytes_per_expert,
+               (size_t)bytes_per_expert);
     }
 }
 

@@ -453,3 +453,58 @@ def test_replica_reduce_order_is_slot_ascending(orc):
     rep2 = np.array([[[1.0]], [[1.0]]], np.float32)
     out2 = orc.replica_reduce(rep_exp2, rep2, owner)
     assert out2[0, 0] == np.float32(2.0 ** 24)  # each +1 is lost in turn: (2^24+1)+1
+
+
+# ------------------------------------------------------------------ router top-k
+
+def test_router_topk_matches_library_routines(orc):
+    """Selection against numpy's stable argsort of the negated logits (ties to
+    the lower id); weights against torch's softmax over all experts,
+    renormalised over the chosen ones, in float64."""
+    for T, E, K, s in [(257, 64, 8, 0.0), (100, 16, 2, 1.0), (64, 384, 8, 1.5), (33, 8, 8, 0.0)]:
+        logits = synth.router_logits(T, E, zipf_s=s, seed=T + E)
+        idx, w = orc.router_topk(logits, K)
+        lg = logits.numpy()
+        ref_idx = np.argsort(-lg, axis=1, kind="stable")[:, :K]
+        np.testing.assert_array_equal(idx, ref_idx)
+        full = torch.softmax(logits.double(), dim=1).numpy()
+        sel = np.take_along_axis(full, ref_idx, axis=1)
+        ref_w = (sel / sel.sum(axis=1, keepdims=True)).astype(np.float32)
+        np.testing.assert_allclose(w, ref_w, rtol=2e-7, atol=1e-30)
+        assert np.all(np.diff(np.take_along_axis(lg, idx, axis=1), axis=1) <= 0)  # descending
+
+
+def test_router_topk_ties_take_lower_id(orc):
+    logits = np.array([[1.0, 3.0, 3.0, 2.0, 3.0, -1.0]], np.float32)
+    idx, w = orc.router_topk(logits, 4)
+    np.testing.assert_array_equal(idx[0], [1, 2, 4, 3])
+    e = np.exp(np.array([0.0, 0.0, 0.0, -1.0]))
+    np.testing.assert_allclose(w[0], (e / e.sum()).astype(np.float32), rtol=1e-7)
+
+
+def test_router_topk_equals_the_input_generator(orc):
+    """synth.routing draws its routing with torch (stable sort + float64
+    softmax); the oracle's C selection must give the same ids."""
+    idx_s, w_s = synth.routing(500, 256, 8, zipf_s=1.0, seed=4)
+    idx_o, w_o = orc.router_topk(synth.router_logits(500, 256, zipf_s=1.0, seed=4), 8)
+    np.testing.assert_array_equal(idx_o, idx_s.numpy())
+    np.testing.assert_allclose(w_o, w_s.numpy(), rtol=2e-7)
+
+
+# ------------------------------------------------------------------ replica weight prefetch
+
+def test_prefetch_on_golden_plan(orc):
+    """Plan case A of tests/golden/plan_worked.txt fills slot (rank 1, slot 0)
+    with expert 0: that slot, and only that one, receives expert 0's weights."""
+    c = _golden_plans()[0]
+    R, S = c["R"][0], c["S"][0]
+    rep = np.array(c["replica_expert"], np.int32).reshape(R, S)
+    rng = np.random.default_rng(0)
+    B = 48
+    weights = rng.integers(0, 256, size=(c["E"][0], B), dtype=np.uint8)
+    slots = rng.integers(0, 256, size=(R * S, B), dtype=np.uint8)
+    out = orc.prefetch(rep, weights, slots)
+    for sl in range(R * S):
+        e = rep.reshape(-1)[sl]
+        np.testing.assert_array_equal(out[sl], weights[e] if e >= 0 else slots[sl])
+    assert (rep >= 0).sum() == 1
