@@ -44,35 +44,47 @@ def build(force: bool = False) -> str:
 _lib = None
 
 
+def configure(cdll: ctypes.CDLL) -> ctypes.CDLL:
+    """Declare the argument and result types of the oracle's C functions."""
+    P = ctypes.c_void_p
+    i32, i64 = ctypes.c_int, ctypes.c_int64
+    sig = {
+        "orc_bf16_to_f32": (ctypes.c_float, [ctypes.c_uint16]),
+        "orc_bf16_from_f32": (ctypes.c_uint16, [ctypes.c_float]),
+        "orc_e4m3_from_f32": (ctypes.c_uint8, [ctypes.c_float]),
+        "orc_e4m3_to_f32": (ctypes.c_float, [ctypes.c_uint8]),
+        "orc_bf16_from_f32_n": (None, [P, i64, P]),
+        "orc_e4m3_from_f32_n": (None, [P, i64, P]),
+        "orc_router_topk": (None, [i32, i32, i32, P, P, P]),
+        "orc_route": (i32, [i32, i32, i32, P, P, P]),
+        "orc_layout_ht": (None, [i32, i32, i32, P, P, P, P]),
+        "orc_layout_ll": (i32, [i32, i32, i32, P, P, P]),
+        "orc_plan_balanced": (i32, [i32, i32, i32, P, P, P, P, P, P, P, P, P]),
+        "orc_layout_balanced": (None, [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P]),
+        "orc_dispatch": (None, [i32, i32, i32, i32, P, P, P, P, P, P, P, P]),
+        "orc_combine": (None, [i32, i32, i32, P, P, P, P]),
+        "orc_combine_backward": (None, [i32, i32, i32, P, P, P, P]),
+        "orc_replica_reduce": (None, [i32, i32, i32, i64, P, P, P]),
+        "orc_prefetch": (None, [i32, i32, i64, P, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(cdll, name)
+        f.restype = res
+        f.argtypes = args
+    return cdll
+
+
+def compile_to(src: str, out: str) -> str:
+    """Compile an oracle source file with the oracle's flags."""
+    subprocess.check_call(["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+                           "-Wall", "-o", out, src, "-lm"])
+    return out
+
+
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
-        P = ctypes.c_void_p
-        i32, i64 = ctypes.c_int, ctypes.c_int64
-        sig = {
-            "orc_bf16_to_f32": (ctypes.c_float, [ctypes.c_uint16]),
-            "orc_bf16_from_f32": (ctypes.c_uint16, [ctypes.c_float]),
-            "orc_e4m3_from_f32": (ctypes.c_uint8, [ctypes.c_float]),
-            "orc_e4m3_to_f32": (ctypes.c_float, [ctypes.c_uint8]),
-            "orc_bf16_from_f32_n": (None, [P, i64, P]),
-            "orc_e4m3_from_f32_n": (None, [P, i64, P]),
-            "orc_router_topk": (None, [i32, i32, i32, P, P, P]),
-            "orc_route": (i32, [i32, i32, i32, P, P, P]),
-            "orc_layout_ht": (None, [i32, i32, i32, P, P, P, P]),
-            "orc_layout_ll": (i32, [i32, i32, i32, P, P, P]),
-            "orc_plan_balanced": (i32, [i32, i32, i32, P, P, P, P, P, P, P, P, P]),
-            "orc_layout_balanced": (None, [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P]),
-            "orc_dispatch": (None, [i32, i32, i32, i32, P, P, P, P, P, P, P, P]),
-            "orc_combine": (None, [i32, i32, i32, P, P, P, P]),
-            "orc_combine_backward": (None, [i32, i32, i32, P, P, P, P]),
-            "orc_replica_reduce": (None, [i32, i32, i32, i64, P, P, P]),
-            "orc_prefetch": (None, [i32, i32, i64, P, P, P]),
-        }
-        for name, (res, args) in sig.items():
-            f = getattr(_lib, name)
-            f.restype = res
-            f.argtypes = args
+        _lib = configure(ctypes.CDLL(build()))
     return _lib
 
 

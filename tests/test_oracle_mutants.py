@@ -1,0 +1,108 @@
+"""The pins are strong enough to catch plausible mistakes in the oracle.
+
+Each case plants one mistake in a copy of oracle/ep_oracle.c: a dropped
+term, a wrong operator, a flipped tie-break, an off-by-one, a wrong rounding,
+a wrong order. It compiles the copy on the CPU, points the oracle wrapper at
+it, and checks that at least one of the listed pins then fails. The real
+oracle is restored afterwards.
+"""
+import ctypes
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ep_oracle.c")
+
+# name, text to replace (must occur once), replacement, pins that must catch it
+MUTANTS = [
+    ("combine drops the first choice",
+     "            for (int k = 0; k < K; k++) {\n                int32_t row = dest_row[(int64_t)t * K + k];\n"
+     "                if (row < 0) continue;\n                float v",
+     "            for (int k = 1; k < K; k++) {\n                int32_t row = dest_row[(int64_t)t * K + k];\n"
+     "                if (row < 0) continue;\n                float v",
+     [lambda: pins.test_identity_expert_returns_x(oracle, "ht"), lambda: pins.test_combine_golden(oracle)]),
+    ("FP8 scale multiplies instead of dividing",
+     "float s = amax / 448.0f;", "float s = amax * 448.0f;",
+     [lambda: pins.test_fp8_block_golden(oracle)]),
+    ("plan keeps the higher id first on a count tie",
+     "(cnt[order[b]] > cnt[v] || (cnt[order[b]] == cnt[v] && order[b] > v))",
+     "(cnt[order[b]] > cnt[v] || (cnt[order[b]] == cnt[v] && order[b] < v))",
+     [lambda: pins.test_plan_golden(oracle)]),
+    ("stable index off by one",
+     "j[(int64_t)t * K + k] = cnt[e];", "j[(int64_t)t * K + k] = cnt[e] + 1;",
+     [lambda: pins.test_route_golden(oracle), lambda: pins.test_route_brute_force(oracle, 0)]),
+    ("e4m3 rounds half away from zero",
+     "double m = nearbyint((a / ldexp(1.0, ex) - 1.0) * 8.0);",
+     "double m = round((a / ldexp(1.0, ex) - 1.0) * 8.0);",
+     [lambda: pins.test_e4m3_golden_table(oracle),
+      lambda: pins.test_e4m3_matches_torch_in_range_all_bf16_times_scales(oracle)]),
+    ("bf16 conversion truncates",
+     "if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))", "if (0)",
+     [lambda: pins.test_bf16_rounding_matches_torch(oracle)]),
+    ("replica gradients added in descending slot order",
+     "for (int a = 0; a < n; a++) acc = acc + rep[(int64_t)list[a] * G + i];",
+     "for (int a = n - 1; a >= 0; a--) acc = acc + rep[(int64_t)list[a] * G + i];",
+     [lambda: pins.test_replica_reduce_order_is_slot_ascending(oracle)]),
+    ("router breaks ties towards the higher id",
+     "if (best < 0 || l[e] > l[best]) best = e;", "if (best < 0 || l[e] >= l[best]) best = e;",
+     [lambda: pins.test_router_topk_ties_take_lower_id(oracle),
+      lambda: pins.test_router_topk_matches_library_routines(oracle)]),
+    ("combine backward forgets the router weight",
+     "float prod = wk * orc_bf16_to_f32(g[(int64_t)t * H + i]);",
+     "float prod = orc_bf16_to_f32(g[(int64_t)t * H + i]);",
+     [lambda: pins.test_adjoint_identities_exact(oracle, False)]),
+    ("LL keeps the pair at the capacity",
+     "} else if (j[p] >= cap) {", "} else if (j[p] > cap) {",
+     [lambda: pins.test_route_golden(oracle), lambda: pins.test_route_ll_capacity(oracle)]),
+    ("plan ignores the replica-slot limit",
+     "if (D[r] > 0 && nrep[r] < S) {", "if (D[r] > 0) {",
+     [lambda: pins.test_plan_golden(oracle)]),
+    ("FP8 cast of an all-zero block divides by zero",
+     "            if (amax == 0.0f)\n                q[b * 128 + i] = 0;\n            else\n"
+     "                q[b * 128 + i] = orc_e4m3_from_f32(orc_bf16_to_f32(x[b * 128 + i]) / s);",
+     "            q[b * 128 + i] = orc_e4m3_from_f32(orc_bf16_to_f32(x[b * 128 + i]) / s);",
+     [lambda: pins.test_fp8_dequant_error_bound(oracle), lambda: pins.test_fp8_block_golden(oracle)]),
+    ("balanced plan places replicas at the owner's offset",
+     "int64_t off = rank_off[r];", "int64_t off = rank_off[r - 1 >= 0 ? r - 1 : 0];",
+     [lambda: pins.test_plan_golden(oracle)]),
+]
+
+
+@pytest.fixture
+def mutant_lib(tmp_path):
+    saved = oracle._lib
+    src = open(SRC).read()
+
+    def load(find, repl):
+        assert src.count(find) == 1, f"mutation anchor not unique: {find!r}"
+        path = tmp_path / "mutant.c"
+        path.write_text(src.replace(find, repl))
+        so = oracle.compile_to(str(path), str(tmp_path / "libmutant.so"))
+        oracle._lib = oracle.configure(ctypes.CDLL(so))
+
+    yield load
+    oracle._lib = saved
+
+
+@pytest.mark.parametrize("name,find,repl,checks", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(mutant_lib, name, find, repl, checks):
+    mutant_lib(find, repl)
+    caught = 0
+    for check in checks:
+        try:
+            with np.errstate(all="ignore"):
+                check()
+        except AssertionError:
+            caught += 1
+    assert caught > 0, f"no pin caught the planted mistake: {name}"
+
+
+def test_real_oracle_passes_the_same_checks():
+    oracle._lib = None  # the real library
+    for _, _, _, checks in MUTANTS:
+        for check in checks:
+            check()

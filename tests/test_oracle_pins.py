@@ -442,17 +442,15 @@ def test_replica_reduce_sums_exactly(orc):
 
 
 def test_replica_reduce_order_is_slot_ascending(orc):
-    # fp32 rounding makes the order visible: 2^24 + 1 - 1 differs by order
-    E, R, S, G = 2, 2, 1, 1
-    rep_exp = np.array([[-1], [0]], np.int32)
-    rep = np.array([[[0.0]], [[1.0]]], np.float32)
-    owner = np.array([[2.0 ** 24], [0.0]], np.float32)
-    out = orc.replica_reduce(rep_exp, rep, owner)
-    assert out[0, 0] == np.float32(2.0 ** 24)  # 2^24 + 1 rounds to even
-    rep_exp2 = np.array([[0], [0]], np.int32)
-    rep2 = np.array([[[1.0]], [[1.0]]], np.float32)
-    out2 = orc.replica_reduce(rep_exp2, rep2, owner)
-    assert out2[0, 0] == np.float32(2.0 ** 24)  # each +1 is lost in turn: (2^24+1)+1
+    """fp32 makes the order visible: starting from 2^24, adding +1 then -2^24
+    gives 0 (the +1 is lost), adding -2^24 then +1 gives 1."""
+    E, R, S, G = 1, 2, 1, 1
+    rep_exp = np.array([[0], [0]], np.int32)            # slot 0 (rank 0) then slot 1 (rank 1)
+    rep = np.array([[[1.0]], [[-(2.0 ** 24)]]], np.float32)
+    owner = np.array([[2.0 ** 24]], np.float32)
+    assert orc.replica_reduce(rep_exp, rep, owner)[0, 0] == 0.0
+    rep_swapped = np.array([[[-(2.0 ** 24)]], [[1.0]]], np.float32)
+    assert orc.replica_reduce(rep_exp, rep_swapped, owner)[0, 0] == 1.0
 
 
 # ------------------------------------------------------------------ router top-k
