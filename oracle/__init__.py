@@ -61,6 +61,8 @@ def configure(cdll: ctypes.CDLL) -> ctypes.CDLL:
         "orc_layout_ll": (i32, [i32, i32, i32, P, P, P]),
         "orc_plan_balanced": (i32, [i32, i32, i32, P, P, P, P, P, P, P, P, P]),
         "orc_layout_balanced": (None, [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P]),
+        "orc_plan_direct": (i32, [i32, i32, i32, P, P, P, P, P, P, P, P, P, P, P, P, P]),
+        "orc_layout_direct": (None, [i32, i32, i32, i32, i32] + [P] * 14),
         "orc_dispatch": (None, [i32, i32, i32, i32, P, P, P, P, P, P, P, P]),
         "orc_combine": (None, [i32, i32, i32, P, P, P, P]),
         "orc_combine_backward": (None, [i32, i32, i32, P, P, P, P]),
@@ -172,8 +174,10 @@ class Routing:
 
 
 def route(idx, E: int, R: int, mode: str = "ht", cap: int = 0, balanced: bool = False,
-          slots: int | None = None) -> Routing:
-    """Counts, stable slots and destination rows (HT, LL or balanced HT)."""
+          slots: int | None = None, direct: bool = False) -> Routing:
+    """Counts, stable slots and destination rows (HT, LL or balanced HT; with
+    `direct`, the inference plan whose overflow pieces read the owner's
+    weights directly)."""
     L = lib()
     idx = _np(idx, np.int32)
     T, K = idx.shape
@@ -197,13 +201,26 @@ def route(idx, E: int, R: int, mode: str = "ht", cap: int = 0, balanced: bool = 
     slen = np.zeros(R * S, np.int32)
     load = np.zeros(R, np.int32)
     roff = np.zeros(R + 1, np.int32)
-    flags |= L.orc_plan_balanced(E, R, S, _p(cnt), _p(keep), _p(tail_start), _p(tail_len), _p(rep),
-                                 _p(sstart), _p(slen), _p(load), _p(roff))
-    L.orc_layout_balanced(T, K, E, R, S, _p(idx), _p(j), _p(keep), _p(tail_start), _p(tail_len), _p(rep),
-                          _p(sstart), _p(slen), _p(roff), _p(dest))
+    plan = {}
+    if direct:
+        dn = np.zeros(R, np.int32)
+        de = np.zeros(R * E, np.int32)
+        ds = np.zeros(R * E, np.int32)
+        dl = np.zeros(R * E, np.int32)
+        flags |= L.orc_plan_direct(E, R, S, _p(cnt), _p(keep), _p(tail_start), _p(tail_len), _p(rep), _p(sstart),
+                                   _p(slen), _p(dn), _p(de), _p(ds), _p(dl), _p(load), _p(roff))
+        L.orc_layout_direct(T, K, E, R, S, _p(idx), _p(j), _p(keep), _p(tail_start), _p(tail_len), _p(rep),
+                            _p(sstart), _p(slen), _p(dn), _p(de), _p(ds), _p(dl), _p(roff), _p(dest))
+        plan.update(direct_n=dn, direct_expert=de.reshape(R, E), direct_start=ds.reshape(R, E),
+                    direct_len=dl.reshape(R, E))
+    else:
+        flags |= L.orc_plan_balanced(E, R, S, _p(cnt), _p(keep), _p(tail_start), _p(tail_len), _p(rep),
+                                     _p(sstart), _p(slen), _p(load), _p(roff))
+        L.orc_layout_balanced(T, K, E, R, S, _p(idx), _p(j), _p(keep), _p(tail_start), _p(tail_len), _p(rep),
+                              _p(sstart), _p(slen), _p(roff), _p(dest))
     own = (keep + tail_len).reshape(R, g)
     counts = np.concatenate([own, slen.reshape(R, S)], axis=1).astype(np.int32)
-    plan = dict(keep=keep, tail_start=tail_start, tail_len=tail_len, replica_expert=rep.reshape(R, S),
+    plan.update(keep=keep, tail_start=tail_start, tail_len=tail_len, replica_expert=rep.reshape(R, S),
                 slot_start=sstart.reshape(R, S), slot_len=slen.reshape(R, S), rank_load=load, rank_off=roff)
     return Routing(cnt, j, dest, flags, T * K, counts, plan)
 

@@ -252,9 +252,18 @@ int orc_layout_ll(int T, int K, int cap, const int32_t *idx, const int32_t *j, i
  * replica_expert[R*S] (-1 = empty), slot_start[R*S] (first stable index the
  * slot holds), slot_len[R*S], rank_load[R], rank_off[R+1].
  */
-int orc_plan_balanced(int E, int R, int S, const int32_t *cnt, int32_t *keep, int32_t *tail_start,
-                      int32_t *tail_len, int32_t *replica_expert, int32_t *slot_start, int32_t *slot_len,
-                      int32_t *rank_load, int32_t *rank_off) {
+/* Inference variant [MoonEP para 5: "a small fixed number of slots while
+ * handling overflow via direct symmetric-memory reads"], reading taken: with
+ * `direct` set, step 5 no longer skips a receiver that has a deficit but no
+ * free slot; the piece goes to it as a *direct* piece, whose rows are computed
+ * with the owner's weights read in place, so every spilled row is placed and
+ * loads are always exact. Direct pieces of rank r (at most one per expert)
+ * are listed in creation order in direct_expert / direct_start / direct_len
+ * [r*E + i], i < direct_n[r]; in r's region they follow its replica slots. */
+static int plan_core(int E, int R, int S, int direct, const int32_t *cnt, int32_t *keep, int32_t *tail_start,
+                     int32_t *tail_len, int32_t *replica_expert, int32_t *slot_start, int32_t *slot_len,
+                     int32_t *direct_n, int32_t *direct_expert, int32_t *direct_start, int32_t *direct_len,
+                     int32_t *rank_load, int32_t *rank_off) {
     int g = E / R, flags = 0;
     int64_t L = 0;
     for (int e = 0; e < E; e++) L += cnt[e];
@@ -267,6 +276,14 @@ int orc_plan_balanced(int E, int R, int S, const int32_t *cnt, int32_t *keep, in
         replica_expert[i] = -1;
         slot_start[i] = 0;
         slot_len[i] = 0;
+    }
+    if (direct) {
+        for (int r = 0; r < R; r++) direct_n[r] = 0;
+        for (int i = 0; i < R * E; i++) {
+            direct_expert[i] = -1;
+            direct_start[i] = 0;
+            direct_len[i] = 0;
+        }
     }
     /* 1-2: keep and deficit per rank */
     for (int r = 0; r < R; r++) {
@@ -325,7 +342,7 @@ int orc_plan_balanced(int E, int R, int S, const int32_t *cnt, int32_t *keep, in
             int chosen = -1;
             for (int a = 0; a < nrecv; a++) {
                 int r = recv[a];
-                if (D[r] > 0 && nrep[r] < S) {
+                if (D[r] > 0 && (nrep[r] < S || direct)) {
                     chosen = r;
                     break;
                 }
@@ -337,10 +354,17 @@ int orc_plan_balanced(int E, int R, int S, const int32_t *cnt, int32_t *keep, in
                 break;
             }
             int64_t give = left < D[chosen] ? left : D[chosen];
-            int s = nrep[chosen]++;
-            replica_expert[chosen * S + s] = e;
-            slot_start[chosen * S + s] = (int32_t)next;
-            slot_len[chosen * S + s] = (int32_t)give;
+            if (nrep[chosen] < S) {
+                int s = nrep[chosen]++;
+                replica_expert[chosen * S + s] = e;
+                slot_start[chosen * S + s] = (int32_t)next;
+                slot_len[chosen * S + s] = (int32_t)give;
+            } else { /* a direct piece (only reachable with `direct`) */
+                int i = direct_n[chosen]++;
+                direct_expert[chosen * E + i] = e;
+                direct_start[chosen * E + i] = (int32_t)next;
+                direct_len[chosen * E + i] = (int32_t)give;
+            }
             D[chosen] -= give;
             left -= give;
             next += give;
@@ -352,6 +376,8 @@ int orc_plan_balanced(int E, int R, int S, const int32_t *cnt, int32_t *keep, in
         int64_t load = 0;
         for (int i = 0; i < g; i++) load += keep[r * g + i] + tail_len[r * g + i];
         for (int s = 0; s < S; s++) load += slot_len[r * S + s];
+        if (direct)
+            for (int i = 0; i < direct_n[r]; i++) load += direct_len[r * E + i];
         rank_load[r] = (int32_t)load;
         rank_off[r + 1] = (int32_t)(rank_off[r] + load);
     }
@@ -362,11 +388,27 @@ int orc_plan_balanced(int E, int R, int S, const int32_t *cnt, int32_t *keep, in
     return flags;
 }
 
+int orc_plan_balanced(int E, int R, int S, const int32_t *cnt, int32_t *keep, int32_t *tail_start,
+                      int32_t *tail_len, int32_t *replica_expert, int32_t *slot_start, int32_t *slot_len,
+                      int32_t *rank_load, int32_t *rank_off) {
+    return plan_core(E, R, S, 0, cnt, keep, tail_start, tail_len, replica_expert, slot_start, slot_len, NULL,
+                     NULL, NULL, NULL, rank_load, rank_off);
+}
+
+int orc_plan_direct(int E, int R, int S, const int32_t *cnt, int32_t *keep, int32_t *tail_start, int32_t *tail_len,
+                    int32_t *replica_expert, int32_t *slot_start, int32_t *slot_len, int32_t *direct_n,
+                    int32_t *direct_expert, int32_t *direct_start, int32_t *direct_len, int32_t *rank_load,
+                    int32_t *rank_off) {
+    return plan_core(E, R, S, 1, cnt, keep, tail_start, tail_len, replica_expert, slot_start, slot_len, direct_n,
+                     direct_expert, direct_start, direct_len, rank_load, rank_off);
+}
+
 /* Destination row of every routed pair under a balanced plan (step 6-7). */
-void orc_layout_balanced(int T, int K, int E, int R, int S, const int32_t *idx, const int32_t *j,
-                         const int32_t *keep, const int32_t *tail_start, const int32_t *tail_len,
-                         const int32_t *replica_expert, const int32_t *slot_start, const int32_t *slot_len,
-                         const int32_t *rank_off, int32_t *dest_row) {
+static void layout_core(int T, int K, int E, int R, int S, const int32_t *idx, const int32_t *j,
+                        const int32_t *keep, const int32_t *tail_start, const int32_t *tail_len,
+                        const int32_t *replica_expert, const int32_t *slot_start, const int32_t *slot_len,
+                        const int32_t *direct_n, const int32_t *direct_expert, const int32_t *direct_start,
+                        const int32_t *direct_len, const int32_t *rank_off, int32_t *dest_row) {
     int g = E / R;
     for (int64_t p = 0; p < (int64_t)T * K; p++) {
         dest_row[p] = -1;
@@ -393,7 +435,37 @@ void orc_layout_balanced(int T, int K, int E, int R, int S, const int32_t *idx, 
                 dest_row[p] = (int32_t)(off + (j[p] - slot_start[sl]));
             }
         }
+        if (!direct_n) continue;
+        for (int r = 0; r < R; r++) { /* direct pieces follow the rank's slots */
+            for (int i = 0; i < direct_n[r]; i++) {
+                if (direct_expert[r * E + i] != e) continue;
+                if (j[p] < direct_start[r * E + i] || j[p] >= direct_start[r * E + i] + direct_len[r * E + i])
+                    continue;
+                int64_t off = rank_off[r];
+                for (int e2 = r * g; e2 < r * g + g; e2++) off += keep[e2] + tail_len[e2];
+                for (int s2 = 0; s2 < S; s2++) off += slot_len[r * S + s2];
+                for (int i2 = 0; i2 < i; i2++) off += direct_len[r * E + i2];
+                dest_row[p] = (int32_t)(off + (j[p] - direct_start[r * E + i]));
+            }
+        }
     }
+}
+
+void orc_layout_balanced(int T, int K, int E, int R, int S, const int32_t *idx, const int32_t *j,
+                         const int32_t *keep, const int32_t *tail_start, const int32_t *tail_len,
+                         const int32_t *replica_expert, const int32_t *slot_start, const int32_t *slot_len,
+                         const int32_t *rank_off, int32_t *dest_row) {
+    layout_core(T, K, E, R, S, idx, j, keep, tail_start, tail_len, replica_expert, slot_start, slot_len, NULL, NULL,
+                NULL, NULL, rank_off, dest_row);
+}
+
+void orc_layout_direct(int T, int K, int E, int R, int S, const int32_t *idx, const int32_t *j, const int32_t *keep,
+                       const int32_t *tail_start, const int32_t *tail_len, const int32_t *replica_expert,
+                       const int32_t *slot_start, const int32_t *slot_len, const int32_t *direct_n,
+                       const int32_t *direct_expert, const int32_t *direct_start, const int32_t *direct_len,
+                       const int32_t *rank_off, int32_t *dest_row) {
+    layout_core(T, K, E, R, S, idx, j, keep, tail_start, tail_len, replica_expert, slot_start, slot_len, direct_n,
+                direct_expert, direct_start, direct_len, rank_off, dest_row);
 }
 
 /* ------------------------------------------------------------------ */

@@ -1,6 +1,7 @@
 """The pins are strong enough to catch plausible mistakes in the oracle.
 
-Each case plants one mistake in a copy of oracle/ep_oracle.c: a dropped
+Each case plants one mistake (one that keeps every access in bounds) in a
+copy of oracle/ep_oracle.c: a dropped
 term, a wrong operator, a flipped tie-break, an off-by-one, a wrong rounding,
 a wrong order. It compiles the copy on the CPU, points the oracle wrapper at
 it, and checks that at least one of the listed pins then fails. The real
@@ -58,17 +59,22 @@ MUTANTS = [
     ("LL keeps the pair at the capacity",
      "} else if (j[p] >= cap) {", "} else if (j[p] > cap) {",
      [lambda: pins.test_route_golden(oracle), lambda: pins.test_route_ll_capacity(oracle)]),
-    ("plan ignores the replica-slot limit",
-     "if (D[r] > 0 && nrep[r] < S) {", "if (D[r] > 0) {",
-     [lambda: pins.test_plan_golden(oracle)]),
+    ("inference plan never takes direct pieces",
+     "if (D[r] > 0 && (nrep[r] < S || direct)) {", "if (D[r] > 0 && (nrep[r] < S || 0)) {",
+     [lambda: pins.test_plan_golden(oracle), lambda: pins.test_direct_plan_invariants(oracle, 16, 4, 1)]),
     ("FP8 cast of an all-zero block divides by zero",
      "            if (amax == 0.0f)\n                q[b * 128 + i] = 0;\n            else\n"
      "                q[b * 128 + i] = orc_e4m3_from_f32(orc_bf16_to_f32(x[b * 128 + i]) / s);",
      "            q[b * 128 + i] = orc_e4m3_from_f32(orc_bf16_to_f32(x[b * 128 + i]) / s);",
      [lambda: pins.test_fp8_dequant_error_bound(oracle), lambda: pins.test_fp8_block_golden(oracle)]),
-    ("balanced plan places replicas at the owner's offset",
-     "int64_t off = rank_off[r];", "int64_t off = rank_off[r - 1 >= 0 ? r - 1 : 0];",
+    ("replica slot offset counts its own slot",
+     "for (int s2 = 0; s2 < s; s2++) off += slot_len[r * S + s2];",
+     "for (int s2 = 0; s2 <= s; s2++) off += slot_len[r * S + s2];",
      [lambda: pins.test_plan_golden(oracle)]),
+    ("direct piece placed before the rank's slots",
+     "                for (int s2 = 0; s2 < S; s2++) off += slot_len[r * S + s2];\n                for (int i2 = 0;",
+     "                for (int s2 = 0; s2 < 0; s2++) off += slot_len[r * S + s2];\n                for (int i2 = 0;",
+     [lambda: pins.test_plan_golden(oracle), lambda: pins.test_direct_plan_invariants(oracle, 16, 4, 1)]),
 ]
 
 

@@ -202,9 +202,18 @@ def _idx_from_counts(cnt):
 def test_plan_golden(orc):
     for c in _golden_plans():
         E, R, S = c["E"][0], c["R"][0], c["S"][0]
+        direct = bool(c.get("direct", [0])[0])
         idx = _idx_from_counts(c["cnt"])
-        r = orc.route(idx, E=E, R=R, balanced=True, slots=S)
+        r = orc.route(idx, E=E, R=R, balanced=True, slots=S, direct=direct)
         p = r.plan
+        if direct:
+            np.testing.assert_array_equal(p["direct_n"], c["direct_n"])
+            for rr in range(R):
+                n = c["direct_n"][rr]
+                if n:
+                    np.testing.assert_array_equal(p["direct_expert"][rr, :n], c[f"direct_expert{rr}"])
+                    np.testing.assert_array_equal(p["direct_start"][rr, :n], c[f"direct_start{rr}"])
+                    np.testing.assert_array_equal(p["direct_len"][rr, :n], c[f"direct_len{rr}"])
         np.testing.assert_array_equal(p["keep"], c["keep"])
         np.testing.assert_array_equal(p["replica_expert"].reshape(-1), c["replica_expert"])
         np.testing.assert_array_equal(p["slot_start"].reshape(-1), c["slot_start"])
@@ -274,6 +283,35 @@ def test_plan_invariants_random_counts(orc, E, R):
         n_over += _plan_invariants(orc, cnt.astype(np.int32), R, g)
     if g >= R:
         assert n_over == 0  # the greedy never ran out of slots on these shapes
+
+
+@pytest.mark.parametrize("E,R,S", [(16, 4, 1), (64, 8, 2), (32, 8, 1), (384, 16, 2), (12, 4, 1)])
+def test_direct_plan_invariants(orc, E, R, S):
+    """Inference plan: loads are always exact (no slot overflow can happen),
+    at most S prefetch slots per rank, and every expert's stable indices are
+    covered exactly once by its own rows, its slots and its direct pieces."""
+    rng = np.random.default_rng(E + R + S)
+    for trial in range(40):
+        w = 1.0 / np.arange(1, E + 1) ** rng.uniform(0.0, 2.5)
+        cnt = rng.multinomial(int(rng.integers(1, 5000)), w / w.sum()).astype(np.int32)
+        idx = _idx_from_counts(cnt)
+        r = orc.route(idx, E=E, R=R, balanced=True, slots=S, direct=True)
+        p = r.plan
+        L = int(cnt.sum())
+        q, rem = divmod(L, R)
+        assert r.flags == 0
+        np.testing.assert_array_equal(p["rank_load"], [q + (i < rem) for i in range(R)])
+        assert ((p["replica_expert"] >= 0).sum(axis=1) <= S).all()
+        for e in range(E):
+            pieces = [(0, int(p["keep"][e]))]
+            pieces += [(int(p["slot_start"][a, b]), int(p["slot_len"][a, b])) for a, b in np.argwhere(p["replica_expert"] == e)]
+            for rr in range(R):
+                for i in range(p["direct_n"][rr]):
+                    if p["direct_expert"][rr, i] == e:
+                        assert rr != e // (E // R)
+                        pieces.append((int(p["direct_start"][rr, i]), int(p["direct_len"][rr, i])))
+            assert sorted(x for s0, n in pieces for x in range(s0, s0 + n)) == list(range(int(cnt[e])))
+        assert sorted(r.dest_row.tolist()) == list(range(L))
 
 
 def test_plan_balances_zipf_routing(orc):
