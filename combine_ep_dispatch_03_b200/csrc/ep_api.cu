@@ -29,6 +29,7 @@ ep_status_t derive_dims(const ep_config_t *c, Dims *d) {
     if (c->mode != EP_MODE_LL && c->mode != EP_MODE_HT) return EP_ERR_INVALID_ARG;
     if (c->fp8 != 0 && c->fp8 != 1) return EP_ERR_INVALID_ARG;
     if (c->balanced != 0 && c->balanced != 1) return EP_ERR_INVALID_ARG;
+    if (c->direct_overflow != 0 && (c->direct_overflow != 1 || !c->balanced)) return EP_ERR_INVALID_ARG;
     if (c->fp8 && H % 128 != 0) return EP_ERR_INVALID_ARG;
     if (c->grad_elems_per_expert < 0 || c->grad_elems_per_expert % 4 != 0) return EP_ERR_INVALID_ARG;
     // the reduce walks (expert, 4096-element chunk) items with 32-bit counters
@@ -38,7 +39,7 @@ ep_status_t derive_dims(const ep_config_t *c, Dims *d) {
     if (L > INT32_MAX / 2) return EP_ERR_INVALID_ARG;
     memset(d, 0, sizeof *d);
     d->T = T; d->H = H; d->E = E; d->K = K; d->R = R; d->g = g;
-    d->mode = c->mode; d->fp8 = c->fp8; d->balanced = c->balanced;
+    d->mode = c->mode; d->fp8 = c->fp8; d->balanced = c->balanced; d->direct = c->direct_overflow;
     d->L = L;
     d->G = c->grad_elems_per_expert;
     if (c->mode == EP_MODE_LL) {
@@ -60,7 +61,9 @@ ep_status_t derive_dims(const ep_config_t *c, Dims *d) {
         d->counts_len = R * (g + d->S);
     }
     d->P = c->balanced ? R + 1 : 1;
-    d->nx_max = c->balanced ? R * d->S + E : 0;
+    // pieces beyond each expert's own rows: replica slots, tails, and direct
+    // pieces (each of which ends an expert or exhausts a receiver)
+    d->nx_max = c->balanced ? R * d->S + 2 * E + R : 0;
     d->wt_log2 = 7; // tiles of 2^7 .. 2^11 pairs, at most about kMaxTiles of them
     while ((1 << d->wt_log2) < kMaxTilePairs && ((int64_t)kMaxTiles << d->wt_log2) < L) ++d->wt_log2;
     d->wt = 1 << d->wt_log2;
@@ -101,6 +104,11 @@ static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
     X(replica_expert, d.R *(d.S > 0 ? d.S : 1))                                                                       \
     X(slot_list, d.R *(d.S > 0 ? d.S : 1))                                                                            \
     X(slot_count, 1)                                                                                                  \
+    X(direct_n, d.R)                                                                                                  \
+    X(direct_expert, d.direct ? (int64_t)d.R * d.E : 1)                                                               \
+    X(direct_start, d.direct ? (int64_t)d.R * d.E : 1)                                                                \
+    X(direct_len, d.direct ? (int64_t)d.R * d.E : 1)                                                                  \
+    X(direct_off, d.direct ? (int64_t)d.R * d.E : 1)                                                                  \
     X(base0, d.E)                                                                                                     \
     X(len0, d.E)                                                                                                      \
     X(xoff, d.E + 1)                                                                                                  \
@@ -367,6 +375,9 @@ ep_status_t ep_get_tensor(const ep_handle_t *h, ep_tensor_t which, const void **
     case EP_T_RANK_LOAD: *dptr = h->ws.rank_load; *numel = d.R; break;
     case EP_T_RANK_OFFSET: *dptr = h->ws.rank_off; *numel = d.R + 1; break;
     case EP_T_REPLICA_EXPERT: *dptr = h->ws.replica_expert; *numel = (int64_t)d.R * d.S; break;
+    case EP_T_DIRECT_COUNT: *dptr = h->ws.direct_n; *numel = d.direct ? d.R : 0; break;
+    case EP_T_DIRECT_EXPERT: *dptr = h->ws.direct_expert; *numel = d.direct ? (int64_t)d.R * d.E : 0; break;
+    case EP_T_DIRECT_LEN: *dptr = h->ws.direct_len; *numel = d.direct ? (int64_t)d.R * d.E : 0; break;
     default: return EP_ERR_INVALID_ARG;
     }
     return EP_OK;

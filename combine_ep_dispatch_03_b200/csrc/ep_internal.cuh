@@ -44,6 +44,11 @@ struct Workspace {
     int32_t *replica_expert; // [max(R*S,1)]
     int32_t *slot_list;      // [max(R*S,1)]: the filled replica slots (r*S+s), ascending
     int32_t *slot_count;     // [1]
+    int32_t *direct_n;       // [R]: direct-read pieces per rank (direct_overflow)
+    int32_t *direct_expert;  // [R*E]: piece i of rank r at r*E+i
+    int32_t *direct_start;   // [R*E]: first stable index it covers
+    int32_t *direct_len;     // [R*E]
+    int32_t *direct_off;     // [R*E]: its first row within the rank's region
     int32_t *base0;          // [E]: row of stable index 0 of each expert (piece 0)
     int32_t *len0;           // [E]: stable indices [0, len0) live in piece 0
     int32_t *xoff;           // [E+1]: extra pieces of expert e: [xoff[e], xoff[e+1])
@@ -64,7 +69,7 @@ struct Workspace {
 
 struct Dims {
     int T, H, E, K, R, g, S; // S = replica slots per rank (0 without a plan)
-    int mode, cap, fp8, balanced;
+    int mode, cap, fp8, balanced, direct;
     int64_t L;               // T*K pairs
     int64_t rows;            // receive-buffer rows
     int64_t G;               // replica-gradient elements per expert

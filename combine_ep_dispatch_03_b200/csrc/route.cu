@@ -237,6 +237,7 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     int32_t *s_slot_e = s_roff + R + 1;       // [R*S]
     int32_t *s_slot_len = s_slot_e + R * S;   // [R*S]
     int32_t *s_slot_off = s_slot_len + R * S; // [R*S]
+    int32_t *s_dn = s_slot_off + R * S;       // [R] direct pieces per rank
     __shared__ int s_L, s_nrecv;
 
     if (tid == 0) {
@@ -247,7 +248,12 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
         s_slot_e[i] = -1;
         s_slot_len[i] = 0;
     }
-    for (int r = tid; r < R; r += nth) s_nrep[r] = 0;
+    for (int r = tid; r < R; r += nth) {
+        s_nrep[r] = 0;
+        s_dn[r] = 0;
+    }
+    if (d.direct)
+        for (int i = tid; i < R * E; i += nth) ws.direct_expert[i] = -1;
     __syncthreads();
     int part = 0;
     for (int e = tid; e < E; e += nth) {
@@ -305,7 +311,9 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     __syncthreads();
 
     // fill: one thread, one step per piece (receivers that ran out of deficit
-    // or slots never qualify again, so one cursor over them suffices)
+    // or slots never qualify again, so one cursor over them suffices; with
+    // direct overflow a receiver out of slots still qualifies and takes the
+    // rows as a direct piece)
     if (tid == 0) {
         const int nrecv = s_nrecv;
         int p = 0;
@@ -314,7 +322,7 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
             const int e = s_list[i], owner = e / g;
             int left = s_cnt[e] - s_keep[e], next = s_keep[e], npc = 1;
             while (left > 0) {
-                while (p < nrecv && (s_D[s_recv[p]] == 0 || s_nrep[s_recv[p]] >= S)) ++p;
+                while (p < nrecv && (s_D[s_recv[p]] == 0 || (!d.direct && s_nrep[s_recv[p]] >= S))) ++p;
                 if (p == nrecv) {
                     s_tail[e] = left;
                     write_piece(d, ws, e, npc++, next, left, owner, -2);
@@ -323,10 +331,18 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
                 }
                 const int r = s_recv[p];
                 const int give = min(left, s_D[r]);
-                const int s = s_nrep[r]++;
-                s_slot_e[r * S + s] = e;
-                s_slot_len[r * S + s] = give;
-                write_piece(d, ws, e, npc++, next, give, r, s);
+                if (s_nrep[r] < S) {
+                    const int s = s_nrep[r]++;
+                    s_slot_e[r * S + s] = e;
+                    s_slot_len[r * S + s] = give;
+                    write_piece(d, ws, e, npc++, next, give, r, s);
+                } else { // a direct piece (direct overflow only)
+                    const int i = s_dn[r]++;
+                    ws.direct_expert[(int64_t)r * E + i] = e;
+                    ws.direct_start[(int64_t)r * E + i] = next;
+                    ws.direct_len[(int64_t)r * E + i] = give;
+                    write_piece(d, ws, e, npc++, next, give, r, -3 - i);
+                }
                 s_D[r] -= give;
                 left -= give;
                 next += give;
@@ -354,6 +370,13 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
             rc[g + s] = v;
             s_slot_off[r * S + s] = run;
             run += v;
+        }
+        if (d.direct) {
+            for (int i = 0; i < s_dn[r]; ++i) { // direct pieces follow the slots
+                ws.direct_off[(int64_t)r * E + i] = run;
+                run += ws.direct_len[(int64_t)r * E + i];
+            }
+            ws.direct_n[r] = s_dn[r];
         }
         s_roff[r] = run;
         ws.rank_load[r] = run;
@@ -385,6 +408,10 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
             ws.xlen[x] = ws.piece_len[o + pc];
             if (s == -2) {
                 ws.xdst[x] = own_base + s_keep[e];
+                continue;
+            }
+            if (s <= -3) { // direct piece -3 - s of rank r: no slot, no gradient to reduce
+                ws.xdst[x] = s_roff[r] + ws.direct_off[(int64_t)r * E + (-3 - s)];
                 continue;
             }
             ws.xdst[x] = s_roff[r] + s_slot_off[r * S + s];
@@ -830,7 +857,7 @@ __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__
 size_t route_smem_layout(const Dims &d) {
     if (!d.balanced) return 0;
     const size_t E = d.E, R = d.R, S = d.S;
-    return sizeof(int32_t) * (E + 6 * E + 4 * R + 1 + 3 * R * S);
+    return sizeof(int32_t) * (E + 6 * E + 5 * R + 1 + 3 * R * S);
 }
 
 size_t route_smem_assign(const Dims &d) {

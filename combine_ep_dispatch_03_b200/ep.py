@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_PKG, "libep_b200.so")
 
 MODE_LL, MODE_HT = 0, 1
 FLAG_BAD_EXPERT_ID, FLAG_DUP_EXPERT_ID, FLAG_CAPACITY, FLAG_PLAN_SLOTS = 0x1, 0x2, 0x4, 0x8
-T_DEST_ROW, T_EXPERT_COUNTS, T_RECV_COUNTS, T_RANK_LOAD, T_RANK_OFFSET, T_REPLICA_EXPERT = range(6)
+(T_DEST_ROW, T_EXPERT_COUNTS, T_RECV_COUNTS, T_RANK_LOAD, T_RANK_OFFSET, T_REPLICA_EXPERT, T_DIRECT_COUNT,
+ T_DIRECT_EXPERT, T_DIRECT_LEN) = range(9)
 
 
 class EpConfig(ctypes.Structure):
@@ -34,6 +35,7 @@ class EpConfig(ctypes.Structure):
         ("balanced", ctypes.c_int32),
         ("replica_slots", ctypes.c_int32),
         ("grad_elems_per_expert", ctypes.c_int64),
+        ("direct_overflow", ctypes.c_int32),
     ]
 
 
@@ -104,9 +106,9 @@ def _check(call: str, status: int) -> None:
 
 def make_config(T: int, H: int, E: int, K: int, R: int, mode: str = "ht", ll_capacity: int = 0,
                 fp8: bool = False, balanced: bool = False, replica_slots: int = 0,
-                grad_elems_per_expert: int = 0) -> EpConfig:
+                grad_elems_per_expert: int = 0, direct_overflow: bool = False) -> EpConfig:
     return EpConfig(T, H, E, K, R, MODE_LL if mode == "ll" else MODE_HT, ll_capacity, int(fp8), int(balanced),
-                    replica_slots, grad_elems_per_expert)
+                    replica_slots, grad_elems_per_expert, int(direct_overflow))
 
 
 def validate(cfg: EpConfig) -> int:
@@ -175,10 +177,11 @@ class Ep:
 
     def __init__(self, T: int, H: int, E: int, K: int, R: int, mode: str = "ht", ll_capacity: int = 0,
                  fp8: bool = False, balanced: bool = False, replica_slots: int = 0,
-                 grad_elems_per_expert: int = 0):
+                 grad_elems_per_expert: int = 0, direct_overflow: bool = False):
         L = lib()
         self.cfg = make_config(T, H, E, K, R, mode, ll_capacity, fp8, balanced, replica_slots,
-                               grad_elems_per_expert)
+                               grad_elems_per_expert, direct_overflow)
+        self.direct = direct_overflow
         self.T, self.H, self.E, self.K, self.R = T, H, E, K, R
         self.mode, self.fp8, self.balanced = mode, fp8, balanced
         self.S = (replica_slots or E // R) if balanced else 0

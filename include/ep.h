@@ -73,7 +73,10 @@ typedef enum ep_tensor {
     EP_T_RECV_COUNTS = 2,    /* int32 [R*(E/R + S)] HT, [E] LL: rows per local slot */
     EP_T_RANK_LOAD = 3,      /* int32 [R]: rows received by each logical rank */
     EP_T_RANK_OFFSET = 4,    /* int32 [R+1]: first row of each rank's region */
-    EP_T_REPLICA_EXPERT = 5  /* int32 [R*S]: expert held by replica slot (r,s), -1 empty */
+    EP_T_REPLICA_EXPERT = 5, /* int32 [R*S]: expert held by replica slot (r,s), -1 empty */
+    EP_T_DIRECT_COUNT = 6,   /* int32 [R]: direct-read pieces of each rank (direct_overflow) */
+    EP_T_DIRECT_EXPERT = 7,  /* int32 [R*E]: expert of direct piece i of rank r at [r*E+i], -1 unused */
+    EP_T_DIRECT_LEN = 8      /* int32 [R*E]: rows of that piece */
 } ep_tensor_t;
 
 /* One EP configuration: fixed for the lifetime of a handle (static shapes,
@@ -93,6 +96,7 @@ typedef struct ep_config {
                                       fit one CTA's shared memory, about E <= 2048) */
     int32_t replica_slots;         /* S in [1, E/R] with balanced; 0 = E/R */
     int64_t grad_elems_per_expert; /* G for ep_reduce_replica_grads; 0 if unused */
+    int32_t direct_overflow;       /* 1 (with balanced): inference plan, see ep_plan */
 } ep_config_t;
 
 typedef struct ep_handle ep_handle_t;
@@ -165,7 +169,13 @@ ep_status_t ep_router_topk(const float *logits, int32_t num_tokens, int32_t num_
  *   plan     with cfg.balanced, the balanced-replica plan: each rank
  *            receives floor or ceil of L/R rows (L = routed pairs), hot
  *            experts spilling into at most S replica slots per rank
- *            (MoonEP article paras. 3 and 5).
+ *            (MoonEP article paras. 3 and 5). With cfg.direct_overflow (the
+ *            inference plan, MoonEP para. 5: a small fixed number of slots,
+ *            overflow served by direct reads of the owner's memory), a rank
+ *            with rows to take but no free slot takes them as a direct piece:
+ *            its rows are computed with the owner's weights read in place,
+ *            and it follows the rank's slots in its region (EP_T_DIRECT_*);
+ *            loads are then always floor or ceil of L/R.
  * topk_idx: device int32 [T, K] row-major. -1 marks a masked choice (not
  * routed, no flag); other ids outside [0, E) and repeats within a token are
  * skipped and flagged. */

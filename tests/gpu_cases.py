@@ -64,7 +64,7 @@ def make_inputs(T, H, E, K, zipf_s=0.0, seed=0):
 
 
 def run_forward(T, H, E, K, R, mode="ht", cap=0, fp8=False, balanced=False, slots=0, zipf_s=0.0, seed=0,
-                idx=None, w=None, x=None, check_combine=True, y_kind="random", G=0):
+                idx=None, w=None, x=None, check_combine=True, y_kind="random", G=0, direct=False):
     """Plan + dispatch + combine on the GPU and in the oracle; assert parity.
     Returns a dict of what was compared (for the tests to add checks)."""
     if x is None:
@@ -73,7 +73,7 @@ def run_forward(T, H, E, K, R, mode="ht", cap=0, fp8=False, balanced=False, slot
         idx, w = synth.routing(T, E, K, zipf_s=zipf_s, seed=seed)
     dev = torch.device("cuda")
     h = ep.Ep(T, H, E, K, R, mode=mode, ll_capacity=cap, fp8=fp8, balanced=balanced, replica_slots=slots,
-              grad_elems_per_expert=G)
+              grad_elems_per_expert=G, direct_overflow=direct)
     xd, idxd, wd = x.to(dev), idx.to(dev), w.to(dev)
     bufs = h.empty_recv()
     h.plan(idxd)
@@ -81,7 +81,7 @@ def run_forward(T, H, E, K, R, mode="ht", cap=0, fp8=False, balanced=False, slot
                bufs["recv_counts"])
     flags = h.status()
 
-    ref = oracle.route(idx, E=E, R=R, mode=mode, cap=cap, balanced=balanced, slots=slots or None)
+    ref = oracle.route(idx, E=E, R=R, mode=mode, cap=cap, balanced=balanced, slots=slots or None, direct=direct)
     assert flags == ref.flags, (flags, ref.flags)
     dest = h.tensor(ep.T_DEST_ROW).cpu().numpy()
     np.testing.assert_array_equal(dest, ref.dest_row)
@@ -92,6 +92,15 @@ def run_forward(T, H, E, K, R, mode="ht", cap=0, fp8=False, balanced=False, slot
         np.testing.assert_array_equal(np.array(rep), ref.plan["replica_expert"].reshape(-1))
         np.testing.assert_array_equal(np.array(load), ref.plan["rank_load"])
         np.testing.assert_array_equal(h.tensor(ep.T_RANK_OFFSET).cpu().numpy(), ref.plan["rank_off"])
+        if direct:
+            dn = h.tensor(ep.T_DIRECT_COUNT).cpu().numpy()
+            np.testing.assert_array_equal(dn, ref.plan["direct_n"])
+            de = h.tensor(ep.T_DIRECT_EXPERT).cpu().numpy().reshape(R, E)
+            dl = h.tensor(ep.T_DIRECT_LEN).cpu().numpy().reshape(R, E)
+            for rr in range(R):
+                np.testing.assert_array_equal(de[rr, :dn[rr]], ref.plan["direct_expert"][rr, :dn[rr]])
+                np.testing.assert_array_equal(dl[rr, :dn[rr]], ref.plan["direct_len"][rr, :dn[rr]])
+                assert (de[rr, dn[rr]:] == -1).all()
 
     rx, rs, rw, re = oracle.dispatch(x, idx, w, ref.dest_row, ref.recv_rows, fp8=fp8)
     rows = np.unique(ref.dest_row[ref.dest_row >= 0])

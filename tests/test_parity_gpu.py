@@ -189,6 +189,21 @@ def test_balanced_plan_slot_overflow_keeps_rows_on_owner():
     g.run_backward(r, seed=6)
 
 
+@pytest.mark.parametrize("E,R,S,s", [(64, 8, 1, 2.0), (32, 8, 1, 2.0), (384, 16, 2, 1.0), (16, 4, 1, 1.5)])
+def test_inference_plan_direct_overflow(E, R, S, s):
+    """Inference plan (a few prefetch slots, overflow read from the owner):
+    loads always exact, direct pieces and rows identical to the oracle, and
+    dispatch / combine / backward / replica reduce on top of it."""
+    g = _gc()
+    T, K = 4096, 8
+    r = g.run_forward(T, 512, E, K, R, balanced=True, slots=S, direct=True, zipf_s=s, seed=E + S, G=256)
+    assert r["flags"] == 0
+    _, load = r["h"].get_plan()
+    assert max(load) - min(load) <= 1
+    assert r["h"].tensor(ep.T_DIRECT_COUNT).sum().item() > 0  # the slots did run out
+    g.run_backward(r, seed=E)
+
+
 def test_zero_blocks_and_large_values_fp8():
     g = _gc()
     T, H, E, K, R = 64, 1024, 16, 2, 4
@@ -213,6 +228,11 @@ def test_plan_is_reused_by_backward_after_other_work():
     h.plan(idx.cuda())
     dest = h.tensor(ep.T_DEST_ROW).cpu().numpy()
     np.testing.assert_array_equal(dest, oracle.route(idx, E=16, R=4).dest_row)
+
+
+def test_direct_overflow_needs_a_plan():
+    with pytest.raises(ep.EpError):
+        ep.Ep(16, 128, 8, 2, 2, direct_overflow=True)
 
 
 def test_host_argument_errors():
