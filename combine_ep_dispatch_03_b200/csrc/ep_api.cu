@@ -60,7 +60,6 @@ ep_status_t derive_dims(const ep_config_t *c, Dims *d) {
         }
         d->counts_len = R * (g + d->S);
     }
-    d->P = c->balanced ? R + 1 : 1;
     // pieces beyond each expert's own rows: replica slots, tails, and direct
     // pieces (each of which ends an expert or exhausts a receiver)
     d->nx_max = c->balanced ? R * d->S + 2 * E + R : 0;
@@ -108,17 +107,12 @@ static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
     X(direct_expert, d.direct ? (int64_t)d.R * d.E : 1)                                                               \
     X(direct_start, d.direct ? (int64_t)d.R * d.E : 1)                                                                \
     X(direct_len, d.direct ? (int64_t)d.R * d.E : 1)                                                                  \
-    X(direct_off, d.direct ? (int64_t)d.R * d.E : 1)                                                                  \
     X(base0, d.E)                                                                                                     \
     X(len0, d.E)                                                                                                      \
     X(xoff, d.E + 1)                                                                                                  \
     X(xstart, d.nx_max > 0 ? d.nx_max : 1)                                                                            \
     X(xlen, d.nx_max > 0 ? d.nx_max : 1)                                                                              \
     X(xdst, d.nx_max > 0 ? d.nx_max : 1)                                                                              \
-    X(piece_start, (int64_t)d.E * d.P)                                                                                \
-    X(piece_len, (int64_t)d.E * d.P)                                                                                  \
-    X(piece_rank, (int64_t)d.E * d.P)                                                                                 \
-    X(piece_slot, (int64_t)d.E * d.P)                                                                                 \
     X(red_list, (int64_t)d.E * d.R)                                                                                   \
     X(red_n, d.E)                                                                                                     \
     X(red_experts, d.E)                                                                                               \

@@ -48,17 +48,12 @@ struct Workspace {
     int32_t *direct_expert;  // [R*E]: piece i of rank r at r*E+i
     int32_t *direct_start;   // [R*E]: first stable index it covers
     int32_t *direct_len;     // [R*E]
-    int32_t *direct_off;     // [R*E]: its first row within the rank's region
     int32_t *base0;          // [E]: row of stable index 0 of each expert (piece 0)
     int32_t *len0;           // [E]: stable indices [0, len0) live in piece 0
     int32_t *xoff;           // [E+1]: extra pieces of expert e: [xoff[e], xoff[e+1])
     int32_t *xstart;         // [nx_max]: first stable index of an extra piece
     int32_t *xlen;           // [nx_max]
     int32_t *xdst;           // [nx_max]: row of the extra piece's first index
-    int32_t *piece_start;    // [E][P]: planner scratch, pieces in creation order
-    int32_t *piece_len;      // [E][P]
-    int32_t *piece_rank;     // [E][P]: rank holding the piece
-    int32_t *piece_slot;     // [E][P]: replica slot, -2 owner tail
     int32_t *red_list;       // [E][R]: slots (r*S+s) holding e, ascending
     int32_t *red_n;          // [E]
     int32_t *red_experts;    // [E]: experts with at least one replica
@@ -77,7 +72,6 @@ struct Dims {
     int ntiles, nhist;       // warp tiles, histogram CTAs
     int nassign;             // CTAs of the slot-assignment kernel
     int cl_size, cl_ppw;     // cluster routing: CTAs (8 or 16, 0 = not used), pairs per warp
-    int P;                   // planner scratch pieces per expert (R+1 with a plan)
     int nx_max;              // bound on extra pieces (R*S + E with a plan, else 0)
     int counts_len;          // recv_counts entries
 };

@@ -199,15 +199,6 @@ __device__ void plain_outputs(const Dims &d, const Workspace &ws, const int32_t 
     }
 }
 
-__device__ __forceinline__ void write_piece(const Dims &d, const Workspace &ws, int e, int pc, int start, int len,
-                                            int rank, int slot) {
-    const int64_t o = (int64_t)e * d.P + pc;
-    ws.piece_start[o] = start;
-    ws.piece_len[o] = len;
-    ws.piece_rank[o] = rank;
-    ws.piece_slot[o] = slot;
-}
-
 // Balanced-replica plan (MoonEP article paras. 3 and 5). The article states
 // only the invariants; this is a deterministic greedy:
 //  keep     each rank visits its own experts by (count asc, id asc) and keeps
@@ -223,22 +214,34 @@ __device__ __forceinline__ void write_piece(const Dims &d, const Workspace &ws, 
 // run [0, keep) is piece 0, the others ("extra" pieces) are stored compactly.
 __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_t *s_cnt, int32_t *sm,
                                 int32_t *s_warp, uint32_t *s_fl) {
-    const int E = d.E, R = d.R, g = d.g, S = d.S, tid = threadIdx.x, nth = blockDim.x;
+    const int E = d.E, R = d.R, g = d.g, S = d.S, NX = d.nx_max, tid = threadIdx.x, nth = blockDim.x;
     int32_t *s_keep = sm;                     // [E]
     int32_t *s_tail = s_keep + E;             // [E] rows left on the owner after the fill
     int32_t *s_list = s_tail + E;             // [E] scratch list / flags
     int32_t *s_spill = s_list + E;            // [E] spilled experts
     int32_t *s_own = s_spill + E;             // [E] own lengths, then own offsets
-    int32_t *s_npc = s_own + E;               // [E] pieces per expert
-    int32_t *s_D = s_npc + E;                 // [R] deficits, then loads
+    int32_t *s_pfirst = s_own + E;            // [E] first extra piece of each expert (creation order)
+    int32_t *s_pn = s_pfirst + E;             // [E] extra pieces of each expert
+    int32_t *s_D = s_pn + E;                  // [R] deficits, then loads
     int32_t *s_nrep = s_D + R;                // [R]
     int32_t *s_recv = s_nrep + R;             // [R] receivers in visiting order
     int32_t *s_roff = s_recv + R;             // [R+1]
-    int32_t *s_slot_e = s_roff + R + 1;       // [R*S]
+    int32_t *s_dn = s_roff + R + 1;           // [R] direct pieces per rank
+    int32_t *s_dsum = s_dn + R;               // [R] rows in direct pieces per rank
+    int32_t *s_dbase = s_dsum + R;            // [R] own + slot rows per rank
+    int32_t *s_slot_e = s_dbase + R;          // [R*S]
     int32_t *s_slot_len = s_slot_e + R * S;   // [R*S]
     int32_t *s_slot_off = s_slot_len + R * S; // [R*S]
-    int32_t *s_dn = s_slot_off + R * S;       // [R] direct pieces per rank
-    __shared__ int s_L, s_nrecv;
+    // the extra pieces (beyond each expert's own rows) in creation order,
+    // which groups them by expert
+    int32_t *s_x_start = s_slot_off + R * S;  // [NX] first stable index
+    int32_t *s_x_len = s_x_start + NX;        // [NX]
+    int32_t *s_x_rank = s_x_len + NX;         // [NX] rank holding the piece
+    int32_t *s_x_slot = s_x_rank + NX;        // [NX] slot >= 0, -2 owner tail, -3 direct
+    int32_t *s_x_aux = s_x_slot + NX;         // [NX] direct: rows before it among the rank's direct rows
+    int32_t *s_A = s_x_aux + NX;              // [E+1] first spilled row of each spilled expert (fill order)
+    int32_t *s_B = s_A + E + 1;               // [R+1] first deficit row of each receiver (visiting order)
+    __shared__ int s_L, s_nrecv, s_seq;
 
     if (tid == 0) {
         s_L = 0;
@@ -251,6 +254,7 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     for (int r = tid; r < R; r += nth) {
         s_nrep[r] = 0;
         s_dn[r] = 0;
+        s_dsum[r] = 0;
     }
     if (d.direct)
         for (int i = tid; i < R * E; i += nth) ws.direct_expert[i] = -1;
@@ -258,7 +262,8 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     int part = 0;
     for (int e = tid; e < E; e += nth) {
         s_tail[e] = 0;
-        s_npc[e] = 1;
+        s_pfirst[e] = 0;
+        s_pn[e] = 0;
         part += s_cnt[e];
     }
     part = __reduce_add_sync(kFull, part);
@@ -310,50 +315,143 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     }
     __syncthreads();
 
-    // fill: one thread, one step per piece (receivers that ran out of deficit
-    // or slots never qualify again, so one cursor over them suffices; with
-    // direct overflow a receiver out of slots still qualifies and takes the
-    // rows as a direct piece)
+    // fill, parallel form. Without a slot running out, the greedy walk below
+    // pairs the spilled rows (experts in fill order, one after the other) with
+    // the deficit rows (receivers in visiting order) position by position: a
+    // piece is the overlap of one expert's spilled rows with one receiver's
+    // deficit rows. Receiver p's pieces come from consecutive experts, so a
+    // piece's slot is its expert's position minus that of the expert holding
+    // p's first deficit row. If some receiver would need more than S slots
+    // (and overflow is not served directly) the walk below runs instead.
+    for (int i = tid; i < nsp; i += nth) s_A[i] = s_cnt[s_list[i]] - s_keep[s_list[i]];
+    for (int i = tid; i < s_nrecv; i += nth) s_B[i] = s_D[s_recv[i]];
+    if (tid == 0) s_seq = 0;
+    __syncthreads();
+    const int nrecv_all = s_nrecv;
+    const int spill_total = block_exscan(s_A, nsp, s_warp);
+    block_exscan(s_B, nrecv_all, s_warp);
     if (tid == 0) {
+        s_A[nsp] = spill_total;
+        s_B[nrecv_all] = spill_total; // the deficits add up to the spilled rows
+    }
+    __syncthreads();
+    // the last index i in [0, n) with a[i] <= v (a ascending, a[0] <= v)
+    auto last_le = [](const int32_t *a, int n, int v) {
+        int lo = 0, hi = n - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (a[mid] <= v) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    };
+    for (int i = tid; i < nsp; i += nth) { // pass 1: pieces per expert, slot check
+        const int a0 = s_A[i], a1 = s_A[i + 1];
+        int n = 0;
+        for (int q = last_le(s_B, nrecv_all, a0); q < nrecv_all && s_B[q] < a1; ++q, ++n) {
+            const int slot = i - last_le(s_A, nsp, s_B[q]);
+            if (slot >= S && !d.direct) s_seq = 1;
+        }
+        s_spill[i] = n; // s_spill is free again: pieces of the i-th expert in fill order
+    }
+    __syncthreads();
+    if (!s_seq) {
+        for (int i = tid; i < nsp; i += nth) { // pass 2: write the pieces
+            const int e = s_list[i];
+            const int a0 = s_A[i], a1 = s_A[i + 1];
+            int x = 0;
+            for (int i2 = 0; i2 < i; ++i2) x += s_spill[i2]; // pieces of earlier experts
+            s_pfirst[e] = x;
+            s_pn[e] = s_spill[i];
+            for (int q = last_le(s_B, nrecv_all, a0); q < nrecv_all && s_B[q] < a1; ++q, ++x) {
+                const int r = s_recv[q];
+                const int lo = max(a0, s_B[q]), hi = min(a1, s_B[q + 1]);
+                const int fe = last_le(s_A, nsp, s_B[q]);
+                const int slot = i - fe;
+                s_x_start[x] = s_keep[e] + (lo - a0);
+                s_x_len[x] = hi - lo;
+                s_x_rank[x] = r;
+                if (slot < S) {
+                    s_x_slot[x] = slot;
+                    s_slot_e[r * S + slot] = e;
+                    s_slot_len[r * S + slot] = hi - lo;
+                } else { // direct piece slot - S of rank r
+                    const int first_direct_row = min(s_B[q + 1], s_A[fe + S]);
+                    s_x_slot[x] = -3;
+                    s_x_aux[x] = lo - first_direct_row;
+                    ws.direct_expert[(int64_t)r * E + slot - S] = e;
+                    ws.direct_start[(int64_t)r * E + slot - S] = s_keep[e] + (lo - a0);
+                    ws.direct_len[(int64_t)r * E + slot - S] = hi - lo;
+                }
+            }
+        }
+        for (int q = tid; q < nrecv_all; q += nth) { // per receiver: slots and direct rows used
+            const int r = s_recv[q];
+            const int fe = last_le(s_A, nsp, s_B[q]), le = last_le(s_A, nsp, s_B[q + 1] - 1);
+            const int npc = le - fe + 1;
+            s_nrep[r] = min(S, npc);
+            s_dn[r] = max(0, npc - S);
+            s_dsum[r] = npc > S ? s_B[q + 1] - s_A[fe + S] : 0;
+            s_D[r] = 0;
+        }
+    }
+    __syncthreads();
+
+    // fill, sequential form: one thread, one step per piece (receivers that
+    // ran out of deficit or slots never qualify again, so one cursor over them
+    // suffices; with direct overflow a receiver out of slots still qualifies
+    // and takes the rows as a direct piece). Pieces go to shared memory in
+    // creation order.
+    if (tid == 0 && s_seq) {
         const int nrecv = s_nrecv;
-        int p = 0;
+        int p = 0, nx = 0;
         uint32_t fl = 0;
         for (int i = 0; i < nsp; ++i) {
             const int e = s_list[i], owner = e / g;
-            int left = s_cnt[e] - s_keep[e], next = s_keep[e], npc = 1;
+            int left = s_cnt[e] - s_keep[e], next = s_keep[e];
+            s_pfirst[e] = nx;
             while (left > 0) {
                 while (p < nrecv && (s_D[s_recv[p]] == 0 || (!d.direct && s_nrep[s_recv[p]] >= S))) ++p;
                 if (p == nrecv) {
                     s_tail[e] = left;
-                    write_piece(d, ws, e, npc++, next, left, owner, -2);
+                    s_x_start[nx] = next;
+                    s_x_len[nx] = left;
+                    s_x_rank[nx] = owner;
+                    s_x_slot[nx] = -2;
+                    ++nx;
                     fl |= EP_FLAG_PLAN_SLOTS;
                     break;
                 }
                 const int r = s_recv[p];
                 const int give = min(left, s_D[r]);
+                s_x_start[nx] = next;
+                s_x_len[nx] = give;
+                s_x_rank[nx] = r;
                 if (s_nrep[r] < S) {
-                    const int s = s_nrep[r]++;
-                    s_slot_e[r * S + s] = e;
-                    s_slot_len[r * S + s] = give;
-                    write_piece(d, ws, e, npc++, next, give, r, s);
+                    const int sl = s_nrep[r]++;
+                    s_slot_e[r * S + sl] = e;
+                    s_slot_len[r * S + sl] = give;
+                    s_x_slot[nx] = sl;
                 } else { // a direct piece (direct overflow only)
-                    const int i = s_dn[r]++;
-                    ws.direct_expert[(int64_t)r * E + i] = e;
-                    ws.direct_start[(int64_t)r * E + i] = next;
-                    ws.direct_len[(int64_t)r * E + i] = give;
-                    write_piece(d, ws, e, npc++, next, give, r, -3 - i);
+                    const int di = s_dn[r]++;
+                    ws.direct_expert[(int64_t)r * E + di] = e;
+                    ws.direct_start[(int64_t)r * E + di] = next;
+                    ws.direct_len[(int64_t)r * E + di] = give;
+                    s_x_slot[nx] = -3;
+                    s_x_aux[nx] = s_dsum[r];
+                    s_dsum[r] += give;
                 }
+                ++nx;
                 s_D[r] -= give;
                 left -= give;
                 next += give;
             }
-            s_npc[e] = npc;
+            s_pn[e] = nx - s_pfirst[e];
         }
         if (fl) atomicOr(s_fl, fl);
     }
     __syncthreads();
 
-    // layout inside each rank region
+    // layout inside each rank region: own experts, replica slots, direct pieces
     for (int e = tid; e < E; e += nth) s_own[e] = s_keep[e] + s_tail[e];
     __syncthreads();
     for (int r = tid; r < R; r += nth) {
@@ -365,19 +463,15 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
             s_own[e] = run;
             run += v;
         }
-        for (int s = 0; s < S; ++s) {
-            const int v = s_slot_len[r * S + s];
-            rc[g + s] = v;
-            s_slot_off[r * S + s] = run;
+        for (int sl = 0; sl < S; ++sl) {
+            const int v = s_slot_len[r * S + sl];
+            rc[g + sl] = v;
+            s_slot_off[r * S + sl] = run;
             run += v;
         }
-        if (d.direct) {
-            for (int i = 0; i < s_dn[r]; ++i) { // direct pieces follow the slots
-                ws.direct_off[(int64_t)r * E + i] = run;
-                run += ws.direct_len[(int64_t)r * E + i];
-            }
-            ws.direct_n[r] = s_dn[r];
-        }
+        s_dbase[r] = run;
+        run += s_dsum[r];
+        if (d.direct) ws.direct_n[r] = s_dn[r];
         s_roff[r] = run;
         ws.rank_load[r] = run;
     }
@@ -386,51 +480,52 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     for (int r = tid; r < R; r += nth) ws.rank_off[r] = s_roff[r];
     if (tid == 0) ws.rank_off[R] = total;
     for (int i = tid; i < R * S; i += nth) ws.replica_expert[i] = s_slot_e[i];
-    for (int e = tid; e < E; e += nth) s_list[e] = s_npc[e] - 1;
+    for (int e = tid; e < E; e += nth) s_list[e] = s_pn[e];
     __syncthreads();
-    const int nx = block_exscan(s_list, E, s_warp); // s_list[e] = first extra piece of e
-    if (tid == 0) ws.xoff[E] = nx;
+    const int nxt = block_exscan(s_list, E, s_warp); // s_list[e] = first compact extra piece of e (id order)
+    if (tid == 0) ws.xoff[E] = nxt;
 
     // piece 0, the compact extra pieces, and the per-expert replica lists
+    // (slots r*S+s in ascending order: each entry's place is the number of
+    // the expert's slot pieces with a smaller key)
     for (int e = tid; e < E; e += nth) {
         const int owner = e / g;
         const int own_base = s_roff[owner] + s_own[e];
         ws.base0[e] = own_base;
         ws.len0[e] = s_keep[e];
         ws.xoff[e] = s_list[e];
-        const int64_t o = (int64_t)e * d.P;
-        int32_t *lst = ws.red_list + (int64_t)e * R;
-        int n = 0;
-        for (int pc = 1; pc < s_npc[e]; ++pc) {
-            const int r = ws.piece_rank[o + pc], s = ws.piece_slot[o + pc];
-            const int x = s_list[e] + pc - 1;
-            ws.xstart[x] = ws.piece_start[o + pc];
-            ws.xlen[x] = ws.piece_len[o + pc];
-            if (s == -2) {
-                ws.xdst[x] = own_base + s_keep[e];
-                continue;
+        const int f = s_pfirst[e], n = s_pn[e];
+        int nrep = 0;
+        for (int i = 0; i < n; ++i) {
+            const int x = f + i, r = s_x_rank[x], sl = s_x_slot[x];
+            const int o = s_list[e] + i;
+            ws.xstart[o] = s_x_start[x];
+            ws.xlen[o] = s_x_len[x];
+            if (sl == -2) {
+                ws.xdst[o] = own_base + s_keep[e];
+            } else if (sl == -3) { // direct piece: no slot, no gradient to reduce
+                ws.xdst[o] = s_roff[r] + s_dbase[r] + s_x_aux[x];
+            } else {
+                ws.xdst[o] = s_roff[r] + s_slot_off[r * S + sl];
+                const int key = r * S + sl;
+                int pos = 0;
+                for (int i2 = 0; i2 < n; ++i2) {
+                    const int sl2 = s_x_slot[f + i2];
+                    if (sl2 >= 0 && s_x_rank[f + i2] * S + sl2 < key) ++pos;
+                }
+                ws.red_list[(int64_t)e * R + pos] = key;
+                ++nrep;
             }
-            if (s <= -3) { // direct piece -3 - s of rank r: no slot, no gradient to reduce
-                ws.xdst[x] = s_roff[r] + ws.direct_off[(int64_t)r * E + (-3 - s)];
-                continue;
-            }
-            ws.xdst[x] = s_roff[r] + s_slot_off[r * S + s];
-            const int key = r * S + s;
-            int a = n++;
-            while (a > 0 && lst[a - 1] > key) { // insertion sort, at most R-1 entries
-                lst[a] = lst[a - 1];
-                --a;
-            }
-            lst[a] = key;
         }
-        ws.red_n[e] = n;
+        ws.red_n[e] = nrep;
+        s_pn[e] = nrep; // reused below as "has replicas"
     }
     __syncthreads();
-    for (int e = tid; e < E; e += nth) s_list[e] = ws.red_n[e] > 0 ? 1 : 0;
+    for (int e = tid; e < E; e += nth) s_list[e] = s_pn[e] > 0 ? 1 : 0;
     __syncthreads();
     const int nred = block_exscan(s_list, E, s_warp);
     for (int e = tid; e < E; e += nth)
-        if (ws.red_n[e] > 0) ws.red_experts[s_list[e]] = e;
+        if (s_pn[e] > 0) ws.red_experts[s_list[e]] = e;
     if (tid == 0) *ws.red_count = nred;
     __syncthreads();
     // the filled replica slots, ascending (the prefetch copies only these);
@@ -856,8 +951,8 @@ __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__
 
 size_t route_smem_layout(const Dims &d) {
     if (!d.balanced) return 0;
-    const size_t E = d.E, R = d.R, S = d.S;
-    return sizeof(int32_t) * (E + 6 * E + 5 * R + 1 + 3 * R * S);
+    const size_t E = d.E, R = d.R, S = d.S, NX = d.nx_max;
+    return sizeof(int32_t) * (E + 7 * E + 7 * R + 1 + 3 * R * S + 5 * NX + E + 1 + R + 1);
 }
 
 size_t route_smem_assign(const Dims &d) {
