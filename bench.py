@@ -378,6 +378,8 @@ def run_native(args):
         wl["s"] = args.zipf
     if args.balanced is not None:
         wl["balanced"] = bool(args.balanced)
+    if args.capacity:
+        wl["cap"] = args.capacity
     name = args.workload if wl == WORKLOADS[args.workload] else args.workload + "_custom"
     seed = rank  # each rank: its own EP world (weak scaling)
     step = Step(wl, dev, seed)
@@ -456,7 +458,14 @@ def run_native(args):
 def run_e2e(step: Step, dev, stream, steps, world, step_bytes):
     """The same step through the public API, its inputs copied from pinned
     host memory and its results (combined tokens, and the input gradient with
-    a backward pass) read back to pinned host memory, inside the timed region."""
+    a backward pass) read back to pinned host memory, inside the timed region.
+
+    Steps are pipelined over three streams: the host-to-device copies of step
+    i+1 run while the device-to-host copies of step i drain, since the two
+    PCIe directions are independent. Each step's copies and kernels are
+    ordered by events: a step's inputs are overwritten only after the previous
+    step's kernels have finished with them, and its outputs are written only
+    after the previous step's results have been read back."""
     import torch
 
     if step.kind == "path":
@@ -466,28 +475,49 @@ def run_e2e(step: Step, dev, stream, steps, world, step_bytes):
     else:
         ins = step.ins
     outs = [(o, torch.empty(o.shape, dtype=o.dtype).pin_memory()) for o in step.outputs]
+    h2d_st, d2h_st = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    state = {"computed": None, "drained": None}
 
     def one():
-        for src, dst in ins:
-            dst.copy_(src, non_blocking=True)
+        # inputs: wait until the previous step's kernels are done reading them
+        if state["computed"] is not None:
+            h2d_st.wait_event(state["computed"])
+        with torch.cuda.stream(h2d_st):
+            for src, dst in ins:
+                dst.copy_(src, non_blocking=True)
+        loaded = torch.cuda.Event()
+        loaded.record(h2d_st)
+        # kernels: wait for this step's inputs and for the previous read-back
+        stream.wait_event(loaded)
+        if state["drained"] is not None:
+            stream.wait_event(state["drained"])
         step.run(stream)
-        for src, dst in outs:
-            dst.copy_(src, non_blocking=True)
+        computed = torch.cuda.Event()
+        computed.record(stream)
+        d2h_st.wait_event(computed)
+        with torch.cuda.stream(d2h_st):
+            for src, dst in outs:
+                dst.copy_(src, non_blocking=True)
+        drained = torch.cuda.Event()
+        drained.record(d2h_st)
+        state["computed"], state["drained"] = computed, drained
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            one()
-        torch.cuda.synchronize()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record(stream)
-        for _ in range(steps):
-            one()
-        e.record(stream)
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    h2d_st.wait_event(s)
+    state["computed"] = state["drained"] = s
+    for _ in range(steps):
+        one()
+    stream.wait_event(state["drained"])
+    e.record(stream)
     torch.cuda.synchronize()
     value, ms = weak_scaling_value(step_bytes, s.elapsed_time(e) / steps, world)
     h2d = sum(src.numel() * src.element_size() for src, _ in ins)
     d2h = sum(src.numel() * src.element_size() for src, _ in outs)
-    return {"value": round(value, 2), "unit": "GB/s",
+    return {"value": round(value, 2), "unit": "GB/s", "pipelined": True,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": steps}
 
 
@@ -606,6 +636,7 @@ def main():
     ap.add_argument("--tokens", type=int, default=0, help="override T (smaller cases for profiling)")
     ap.add_argument("--zipf", type=float, default=None, help="override the router's Zipf bias s")
     ap.add_argument("--balanced", type=int, choices=[0, 1], default=None, help="override the balanced plan")
+    ap.add_argument("--capacity", type=int, default=0, help="override the LL per-expert capacity (smaller buffers)")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
