@@ -57,6 +57,38 @@ __device__ __forceinline__ void stage_routing(const int32_t *__restrict__ dest_r
     }
 }
 
+// read_before_wait: a dispatch reads its token row x[t] before
+// griddepcontrol.wait. The kernels that may run concurrently with that read
+// are the routing kernels of the plan just before it (they write routing state
+// only, never x) and, through them, nothing older: each routing kernel lets its
+// dependents start only after its own wait, that is after every earlier kernel
+// of the stream has completed. A caller that writes x with a kernel of its own
+// that triggers its dependents early must write x before the trigger.
+template <int VPT>
+__device__ __forceinline__ void load_slab(const uint4 *__restrict__ src, int c0, int nvec, uint4 *v) {
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+        const int c = c0 + threadIdx.x + i * blockDim.x;
+        if (c < nvec) v[i] = __ldcs(src + c);
+    }
+}
+
+// the two 16-byte halves of each thread's 16-element chunks (zeros past the row)
+template <int CPT>
+__device__ __forceinline__ void load_pairs(const uint4 *__restrict__ src, int c0, int nchunk, uint4 *a, uint4 *b) {
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = c0 + threadIdx.x + i * blockDim.x;
+        if (c < nchunk) {
+            a[i] = __ldcs(src + 2 * c);
+            b[i] = __ldcs(src + 2 * c + 1);
+        } else {
+            a[i] = make_uint4(0, 0, 0, 0);
+            b[i] = a[i];
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // dispatch, bf16 payload: recv[dest_row[t,k]] = x[t]
 // ---------------------------------------------------------------------------
@@ -64,42 +96,40 @@ template <int VPT>
 __global__ void __launch_bounds__(256) k_dispatch_bf16(const uint4 *__restrict__ x, const int32_t *__restrict__ idx,
                                                        const float *__restrict__ w,
                                                        const int32_t *__restrict__ dest_row, int K, int nvec,
-                                                       uint4 *__restrict__ recv, float *__restrict__ recv_w,
+                                                       int part, uint4 *__restrict__ recv, float *__restrict__ recv_w,
                                                        int32_t *__restrict__ recv_expert,
                                                        const int32_t *__restrict__ counts_src,
                                                        int32_t *__restrict__ counts_dst, int counts_len) {
-    pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     __shared__ int s_dest[kMaxTopk];
     const int t = blockIdx.x;
     const int64_t pb = (int64_t)t * K;
+    const int cb = blockIdx.y * part, n = min(part, nvec - cb); // this CTA's vectors of the row
+    const uint4 *src = x + (int64_t)t * nvec + cb;
+    const int step = VPT * blockDim.x;
+    uint4 v[VPT];
+    load_slab<VPT>(src, 0, n, v); // before the wait: see read_before_wait
+    pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     if (threadIdx.x < K) {
         const int dr = dest_row[pb + threadIdx.x];
         s_dest[threadIdx.x] = dr;
-        if (dr >= 0) {
+        if (dr >= 0 && blockIdx.y == 0) {
             if (recv_w) recv_w[dr] = w[pb + threadIdx.x];
             if (recv_expert) recv_expert[dr] = idx[pb + threadIdx.x];
         }
     }
-    if (t == 0 && counts_dst)
+    if (t == 0 && blockIdx.y == 0 && counts_dst)
         for (int i = threadIdx.x; i < counts_len; i += blockDim.x) counts_dst[i] = counts_src[i];
-    const uint4 *src = x + (int64_t)t * nvec;
-    const int step = VPT * blockDim.x;
-    for (int c0 = 0; c0 < nvec; c0 += step) {
-        uint4 v[VPT];
-#pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            const int c = c0 + threadIdx.x + i * blockDim.x;
-            if (c < nvec) v[i] = __ldcs(src + c);
-        }
+    for (int c0 = 0; c0 < n; c0 += step) {
+        if (c0 > 0) load_slab<VPT>(src, c0, n, v);
         if (c0 == 0) __syncthreads();
         for (int k = 0; k < K; ++k) {
             const int dr = s_dest[k];
             if (dr < 0) continue;
-            uint4 *dst = recv + (int64_t)dr * nvec;
+            uint4 *dst = recv + (int64_t)dr * nvec + cb;
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 const int c = c0 + threadIdx.x + i * blockDim.x;
-                if (c < nvec) __stcs(dst + c, v[i]);
+                if (c < n) __stcs(dst + c, v[i]);
             }
         }
     }
@@ -116,40 +146,33 @@ template <int CPT>
 __global__ void __launch_bounds__(256) k_dispatch_fp8(const uint4 *__restrict__ x, const int32_t *__restrict__ idx,
                                                       const float *__restrict__ w,
                                                       const int32_t *__restrict__ dest_row, int K, int nchunk,
-                                                      uint4 *__restrict__ recv, float *__restrict__ scales,
+                                                      int part, uint4 *__restrict__ recv, float *__restrict__ scales,
                                                       float *__restrict__ recv_w, int32_t *__restrict__ recv_expert,
                                                       const int32_t *__restrict__ counts_src,
                                                       int32_t *__restrict__ counts_dst, int counts_len) {
-    pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     __shared__ int s_dest[kMaxTopk];
     const int t = blockIdx.x;
     const int64_t pb = (int64_t)t * K;
     const int nb = nchunk >> 3; // 128-element blocks per row
+    // this CTA's chunks of the row (part is a multiple of 8: whole blocks)
+    const int cb = blockIdx.y * part, n = min(part, nchunk - cb);
+    const uint4 *src = x + (int64_t)t * 2 * nchunk + 2 * cb;
+    const int step = CPT * blockDim.x;
+    uint4 a[CPT], b[CPT];
+    load_pairs<CPT>(src, 0, n, a, b); // before the wait: see read_before_wait
+    pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     if (threadIdx.x < K) {
         const int dr = dest_row[pb + threadIdx.x];
         s_dest[threadIdx.x] = dr;
-        if (dr >= 0) {
+        if (dr >= 0 && blockIdx.y == 0) {
             if (recv_w) recv_w[dr] = w[pb + threadIdx.x];
             if (recv_expert) recv_expert[dr] = idx[pb + threadIdx.x];
         }
     }
-    if (t == 0 && counts_dst)
+    if (t == 0 && blockIdx.y == 0 && counts_dst)
         for (int i = threadIdx.x; i < counts_len; i += blockDim.x) counts_dst[i] = counts_src[i];
-    const uint4 *src = x + (int64_t)t * 2 * nchunk;
-    const int step = CPT * blockDim.x;
-    for (int c0 = 0; c0 < nchunk; c0 += step) {
-        uint4 a[CPT], b[CPT];
-#pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-            const int c = c0 + threadIdx.x + i * blockDim.x;
-            if (c < nchunk) {
-                a[i] = __ldcs(src + 2 * c);
-                b[i] = __ldcs(src + 2 * c + 1);
-            } else {
-                a[i] = make_uint4(0, 0, 0, 0);
-                b[i] = a[i];
-            }
-        }
+    for (int c0 = 0; c0 < n; c0 += step) {
+        if (c0 > 0) load_pairs<CPT>(src, c0, n, a, b);
         uint4 q[CPT];
         float sc[CPT];
 #pragma unroll
@@ -180,13 +203,13 @@ __global__ void __launch_bounds__(256) k_dispatch_fp8(const uint4 *__restrict__ 
         for (int k = 0; k < K; ++k) {
             const int dr = s_dest[k];
             if (dr < 0) continue;
-            uint4 *dst = recv + (int64_t)dr * nchunk;
+            uint4 *dst = recv + (int64_t)dr * nchunk + cb;
 #pragma unroll
             for (int i = 0; i < CPT; ++i) {
                 const int c = c0 + threadIdx.x + i * blockDim.x;
-                if (c < nchunk) {
+                if (c < n) {
                     __stcs(dst + c, q[i]);
-                    if ((c & 7) == 0) scales[(int64_t)dr * nb + (c >> 3)] = sc[i];
+                    if ((c & 7) == 0) scales[(int64_t)dr * nb + ((cb + c) >> 3)] = sc[i];
                 }
             }
         }
@@ -200,19 +223,21 @@ __global__ void __launch_bounds__(256) k_dispatch_fp8(const uint4 *__restrict__ 
 template <int CPT, bool UNIT>
 __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, const float *__restrict__ w,
                                                  const int32_t *__restrict__ dest_row, int K, int nvec,
-                                                 uint4 *__restrict__ out) {
+                                                 int part, uint4 *__restrict__ out) {
     pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     __shared__ int s_dest[kMaxTopk];
     __shared__ float s_w[kMaxTopk];
     const int t = blockIdx.x;
     stage_routing(dest_row, w, (int64_t)t * K, K, s_dest, s_w);
     __syncthreads();
+    const int cb = blockIdx.y * part, n = min(part, nvec - cb); // this CTA's vectors of the row
+    const uint4 *yb = y + cb;
     const int step = CPT * blockDim.x;
-    for (int c0 = 0; c0 < nvec; c0 += step) {
+    for (int c0 = 0; c0 < n; c0 += step) {
 #pragma unroll
         for (int i = 0; i < CPT; ++i) {
             const int c = c0 + threadIdx.x + i * blockDim.x;
-            if (c >= nvec) continue;
+            if (c >= n) continue;
             float acc[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
@@ -222,7 +247,7 @@ __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, co
                 for (int kk = 0; kk < 8; ++kk) {
                     const int k = k0 + kk;
                     const int dr = k < K ? s_dest[k] : -1;
-                    v[kk] = dr >= 0 ? __ldcs(y + (int64_t)dr * nvec + c) : make_uint4(0, 0, 0, 0);
+                    v[kk] = dr >= 0 ? __ldcs(yb + (int64_t)dr * nvec + c) : make_uint4(0, 0, 0, 0);
                 }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -240,7 +265,7 @@ __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, co
                     }
                 }
             }
-            __stcs(out + (int64_t)t * nvec + c, pack8(acc));
+            __stcs(out + (int64_t)t * nvec + cb + c, pack8(acc));
         }
     }
 }
@@ -251,31 +276,28 @@ __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, co
 template <int VPT>
 __global__ void __launch_bounds__(256) k_combine_bwd(const uint4 *__restrict__ g, const float *__restrict__ w,
                                                      const int32_t *__restrict__ dest_row, int K, int nvec,
-                                                     uint4 *__restrict__ gy) {
+                                                     int part, uint4 *__restrict__ gy) {
     pdl_wait(); // no early trigger: measured slower for these multi-wave grids
     __shared__ int s_dest[kMaxTopk];
     __shared__ float s_w[kMaxTopk];
     const int t = blockIdx.x;
     stage_routing(dest_row, w, (int64_t)t * K, K, s_dest, s_w);
-    const uint4 *src = g + (int64_t)t * nvec;
+    const int cb = blockIdx.y * part, n = min(part, nvec - cb); // this CTA's vectors of the row
+    const uint4 *src = g + (int64_t)t * nvec + cb;
     const int step = VPT * blockDim.x;
-    for (int c0 = 0; c0 < nvec; c0 += step) {
+    for (int c0 = 0; c0 < n; c0 += step) {
         uint4 v[VPT];
-#pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            const int c = c0 + threadIdx.x + i * blockDim.x;
-            if (c < nvec) v[i] = __ldcs(src + c);
-        }
+        load_slab<VPT>(src, c0, n, v);
         if (c0 == 0) __syncthreads();
         for (int k = 0; k < K; ++k) {
             const int dr = s_dest[k];
             if (dr < 0) continue;
             const float wk = s_w[k];
-            uint4 *dst = gy + (int64_t)dr * nvec;
+            uint4 *dst = gy + (int64_t)dr * nvec + cb;
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 const int c = c0 + threadIdx.x + i * blockDim.x;
-                if (c >= nvec) continue;
+                if (c >= n) continue;
                 float f[8];
                 unpack8(v[i], f);
 #pragma unroll
@@ -387,6 +409,21 @@ void pick_shape(int n, int *per_thread, int *threads) {
     *threads = 256; // rows longer than 2048 vectors loop over slabs
 }
 
+// Vectors of a row per CTA. A batch of a few thousand tokens gives a grid of
+// one or two waves of one-row CTAs, whose last, partial wave leaves most SMs
+// idle while it drains; such rows are cut into parts (whole warps of vectors,
+// at least kSplitMinVectors each) until the grid has about kSplitCtasPerSm
+// CTAs per SM. Large batches keep one CTA per row.
+constexpr int kSplitCtasPerSm = 32, kSplitMinVectors = 128;
+
+int row_part(int T, int nvec) {
+    const int64_t want = (int64_t)kSplitCtasPerSm * num_sms();
+    int parts = 1;
+    while ((int64_t)T * parts < want && nvec / (2 * parts) >= kSplitMinVectors) parts *= 2;
+    if (parts == 1) return nvec;
+    return ((nvec + parts - 1) / parts + 31) / 32 * 32;
+}
+
 #define EPB_SWITCH_VPT(v, KERNEL, ...)                                                                               \
     switch (v) {                                                                                                     \
     case 1: err = launch_pdl(KERNEL<1>, grid, dim3(threads), 0, st, __VA_ARGS__); break;                             \
@@ -406,19 +443,22 @@ cudaError_t launch_dispatch(const Dims &d, const Workspace &ws, const void *x, c
                                    cudaMemcpyDeviceToDevice, st);
         return cudaSuccess;
     }
-    const dim3 grid(d.T);
     int per, threads;
     cudaError_t err = cudaSuccess;
     if (d.fp8) {
-        const int nchunk = d.H / 16;
-        pick_shape(nchunk, &per, &threads);
-        EPB_SWITCH_VPT(per, k_dispatch_fp8, (const uint4 *)x, topk_idx, topk_w, ws.dest_row, d.K, nchunk,
+        const int nchunk = d.H / 16; // a multiple of 8, and so is every part
+        const int part = row_part(d.T, nchunk);
+        const dim3 grid(d.T, (nchunk + part - 1) / part);
+        pick_shape(part, &per, &threads);
+        EPB_SWITCH_VPT(per, k_dispatch_fp8, (const uint4 *)x, topk_idx, topk_w, ws.dest_row, d.K, nchunk, part,
                        (uint4 *)recv_x, recv_scales, recv_w, recv_expert, ws.recv_counts, recv_counts,
                        d.counts_len);
     } else {
         const int nvec = d.H / 8;
-        pick_shape(nvec, &per, &threads);
-        EPB_SWITCH_VPT(per, k_dispatch_bf16, (const uint4 *)x, topk_idx, topk_w, ws.dest_row, d.K, nvec,
+        const int part = row_part(d.T, nvec);
+        const dim3 grid(d.T, (nvec + part - 1) / part);
+        pick_shape(part, &per, &threads);
+        EPB_SWITCH_VPT(per, k_dispatch_bf16, (const uint4 *)x, topk_idx, topk_w, ws.dest_row, d.K, nvec, part,
                        (uint4 *)recv_x, recv_w, recv_expert, ws.recv_counts, recv_counts, d.counts_len);
     }
     return err;
@@ -427,12 +467,13 @@ cudaError_t launch_dispatch(const Dims &d, const Workspace &ws, const void *x, c
 cudaError_t launch_combine_backward(const Dims &d, const Workspace &ws, const void *grad_out, const float *topk_w,
                                     void *grad_expert_out, cudaStream_t st) {
     if (d.T == 0) return cudaSuccess;
-    const dim3 grid(d.T);
     const int nvec = d.H / 8;
+    const int part = row_part(d.T, nvec);
+    const dim3 grid(d.T, (nvec + part - 1) / part);
     int per, threads;
     cudaError_t err = cudaSuccess;
-    pick_shape(nvec, &per, &threads);
-    EPB_SWITCH_VPT(per, k_combine_bwd, (const uint4 *)grad_out, topk_w, ws.dest_row, d.K, nvec,
+    pick_shape(part, &per, &threads);
+    EPB_SWITCH_VPT(per, k_combine_bwd, (const uint4 *)grad_out, topk_w, ws.dest_row, d.K, nvec, part,
                    (uint4 *)grad_expert_out);
     return err;
 }
@@ -440,27 +481,28 @@ cudaError_t launch_combine_backward(const Dims &d, const Workspace &ws, const vo
 cudaError_t launch_combine(const Dims &d, const Workspace &ws, const void *y, const float *topk_w, void *out,
                            cudaStream_t st) {
     if (d.T == 0) return cudaSuccess;
-    const dim3 grid(d.T);
     const int nvec = d.H / 8;
+    const int part = row_part(d.T, nvec);
+    const dim3 grid(d.T, (nvec + part - 1) / part);
     int per, threads;
-    pick_shape(nvec, &per, &threads);
+    pick_shape(part, &per, &threads);
     const uint4 *yy = (const uint4 *)y;
     uint4 *oo = (uint4 *)out;
     const dim3 block(threads);
     if (topk_w) {
         switch (per) {
-        case 1: return launch_pdl(k_combine<1, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, oo);
-        case 2: return launch_pdl(k_combine<2, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, oo);
-        case 4: return launch_pdl(k_combine<4, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, oo);
-        default: return launch_pdl(k_combine<8, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, oo);
+        case 1: return launch_pdl(k_combine<1, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, part, oo);
+        case 2: return launch_pdl(k_combine<2, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, part, oo);
+        case 4: return launch_pdl(k_combine<4, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, part, oo);
+        default: return launch_pdl(k_combine<8, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, part, oo);
         }
     }
     const float *none = nullptr;
     switch (per) {
-    case 1: return launch_pdl(k_combine<1, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, oo);
-    case 2: return launch_pdl(k_combine<2, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, oo);
-    case 4: return launch_pdl(k_combine<4, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, oo);
-    default: return launch_pdl(k_combine<8, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, oo);
+    case 1: return launch_pdl(k_combine<1, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, part, oo);
+    case 2: return launch_pdl(k_combine<2, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, part, oo);
+    case 4: return launch_pdl(k_combine<4, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, part, oo);
+    default: return launch_pdl(k_combine<8, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, part, oo);
     }
 }
 

@@ -70,15 +70,17 @@ ep_status_t derive_dims(const ep_config_t *c, Dims *d) {
     d->nhist = (d->ntiles + kRouteWarps - 1) / kRouteWarps;
     const int64_t per_cta = (int64_t)kRouteThreads * kAssignPer; // pairs per assignment CTA
     d->nassign = (int)(L > 0 ? (L + per_cta - 1) / per_cta : 1);
-    // cluster routing (plain layouts, batches small enough that each warp of a
-    // cluster of 8 takes at most kClusterMaxPairsPerWarp pairs: measured
-    // faster than the three-kernel path there, slower beyond)
-    if (!c->balanced) {
-        const int cs = 8;
+    // cluster routing: plain layouts and at most kClusterMaxPairs pairs
+    // (measured faster than the three-kernel path there, slower beyond). A
+    // cluster of 8 CTAs up to 16384 pairs; above that a cluster of 16 halves
+    // each SM's share of the warp votes (measured 13.2 vs 15.2 us at 32768
+    // pairs; at 8192 pairs 8 CTAs are faster).
+    if (!c->balanced && L <= kClusterMaxPairs) {
+        const int cs = L > 16384 ? 16 : 8;
         const int64_t ppw = ((L + (int64_t)cs * kClusterWarps - 1) / ((int64_t)cs * kClusterWarps) + 31) / 32 * 32;
         d->cl_size = cs;
         d->cl_ppw = (int)(ppw > 0 ? ppw : 32);
-        if (ppw > kClusterMaxPairsPerWarp || route_smem_cluster(*d) > (size_t)kMaxRouteSmem) d->cl_size = 0;
+        if (route_smem_cluster(*d) > (size_t)kMaxRouteSmem) d->cl_size = 0;
     }
     // the routing kernels keep their tables in one CTA's shared memory
     if (route_smem_layout(*d) > (size_t)kMaxRouteSmem || route_smem_assign(*d) > (size_t)kMaxRouteSmem ||

@@ -27,7 +27,7 @@ constexpr int kSmallMaxPairs = 1024;      // single-CTA routing up to this many 
 constexpr int kSmallMaxExperts = 512;     // ... and experts (plain layouts only)
 constexpr int kClusterThreads = 1024;     // one-launch cluster routing: threads per CTA
 constexpr int kClusterWarps = kClusterThreads / 32;
-constexpr int kClusterMaxPairsPerWarp = 128;
+constexpr int kClusterMaxPairs = 32768;  // ... up to this many (token, k) pairs
 
 // Device workspace of a handle: the routing state one ep_plan builds and the
 // later calls of the same forward/backward pass read.

@@ -13,7 +13,8 @@
 // Large batches, three kernels:
 //   k_route_hist    per warp tile of consecutive pairs: validate ids, give
 //                   each pair its rank among the tile's pairs of the same
-//                   expert (match_any), count the tile's pairs per expert
+//                   expert (a ballot per id bit), count the tile's pairs
+//                   per expert
 //   k_route_scan    per expert: exclusive scan of the tile counts over tiles;
 //                   with a balanced plan, the CTA that finishes last (a
 //                   ticket counter, no waiting) builds the plan
@@ -34,10 +35,12 @@
 
 namespace cg = cooperative_groups;
 
+
 namespace epb {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
+static_assert(kClusterWarps % 8 == 0, "the cluster kernel sums warp counts 8 at a time");
 constexpr int kSmallThreads = 1024;
 constexpr int kSmallWarps = kSmallThreads / 32;
 
@@ -45,6 +48,48 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     unsigned m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
+}
+
+// Bits of an expert id in [0, E).
+__device__ __forceinline__ int id_bits(int E) { return E > 1 ? 32 - __clz(E - 1) : 0; }
+
+// The lanes in `active` whose v (in [0, 2^bits)) equals this lane's: one
+// ballot per bit (a radix match), NB independent ballots issued back to back.
+// __match_any_sync did the same in several thousand cycles per call with 32
+// warps of a CTA calling it at once. Bits above `bits` are 0 for every lane in
+// `active`, so a larger NB gives the same mask.
+template <int NB>
+__device__ __forceinline__ unsigned warp_peers_n(int v, unsigned active) {
+    unsigned m = active;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const bool one = (v >> b) & 1;
+        const unsigned s = __ballot_sync(kFull, one);
+        m &= one ? s : ~s;
+    }
+    return m;
+}
+
+__device__ __forceinline__ unsigned warp_peers(int v, int bits, unsigned active) {
+    if (bits <= 4) return warp_peers_n<4>(v, active);
+    if (bits <= 8) return warp_peers_n<8>(v, active);
+    return warp_peers_n<12>(v, active); // kMaxExperts = 2^12
+}
+
+// A 32-pair warp step that holds whole tokens (K divides 32, the step starts
+// at a multiple of 32): a lane whose id repeats one of a lower lane of the
+// same token is dropped (e = -1) and flagged. Returns each kept lane's peers
+// among the kept lanes.
+__device__ __forceinline__ unsigned whole_token_peers(int &e, int K, int bits, uint32_t &fl) {
+    const int lane = threadIdx.x & 31;
+    const unsigned peers = warp_peers(e, bits, __ballot_sync(kFull, e >= 0));
+    const unsigned tok = K == 32 ? kFull : ((1u << K) - 1u) << (lane & ~(K - 1)); // K is a power of two
+    const bool dup = e >= 0 && (peers & tok & lanemask_lt()) != 0;
+    if (dup) {
+        fl |= EP_FLAG_DUP_EXPERT_ID;
+        e = -1;
+    }
+    return peers & ~__ballot_sync(kFull, dup);
 }
 
 // A pair is routed iff its id is in [0, E) and no earlier choice of the same
@@ -120,11 +165,11 @@ __device__ int block_exscan(int32_t *a, int n, int32_t *s_warp) {
 // adding the routed pairs of each expert to its own counters my[e].
 __device__ __forceinline__ void warp_count(const int32_t *s_ids, int lo, int hi, int K, int E, int32_t *my,
                                            uint32_t &fl) {
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, bits = id_bits(E);
     for (int base = lo; base < hi; base += 32) {
         const int p = base + lane;
         const int e = p < hi ? classify(s_ids, p, p % K, E, fl) : -1;
-        const unsigned peers = __match_any_sync(kFull, e >= 0 ? e : -1 - lane);
+        const unsigned peers = warp_peers(e, bits, __ballot_sync(kFull, e >= 0));
         if (e >= 0 && (peers & lanemask_lt()) == 0) my[e] += __popc(peers);
         __syncwarp();
     }
@@ -135,12 +180,12 @@ __device__ __forceinline__ void warp_count(const int32_t *s_ids, int lo, int hi,
 template <class Lookup>
 __device__ __forceinline__ void warp_assign(const int32_t *s_ids, int lo, int hi, int K, int E, int32_t *my,
                                             int32_t *__restrict__ dest_row, Lookup look) {
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, bits = id_bits(E);
     uint32_t fl = 0;
     for (int base = lo; base < hi; base += 32) {
         const int p = base + lane;
         const int e = p < hi ? classify(s_ids, p, p % K, E, fl) : -1;
-        const unsigned peers = __match_any_sync(kFull, e >= 0 ? e : -1 - lane);
+        const unsigned peers = warp_peers(e, bits, __ballot_sync(kFull, e >= 0));
         int dest = -1;
         if (e >= 0) dest = look(e, my[e] + __popc(peers & lanemask_lt()));
         __syncwarp();
@@ -187,11 +232,14 @@ __device__ void plain_outputs(const Dims &d, const Workspace &ws, const int32_t 
         ws.base0[e] = s_base[e];
         ws.recv_counts[e] = s_len[e];
     }
-    for (int r = tid; r < R; r += nth) {
+    for (int r = tid >> 5; r < R; r += nth >> 5) { // a warp per rank
         int s = 0;
-        for (int i = 0; i < g; ++i) s += s_len[r * g + i];
-        ws.rank_load[r] = s;
-        ws.rank_off[r] = ll ? r * g * d.cap : s_base[r * g];
+        for (int i = tid & 31; i < g; i += 32) s += s_len[r * g + i];
+        s = __reduce_add_sync(kFull, s);
+        if ((tid & 31) == 0) {
+            ws.rank_load[r] = s;
+            ws.rank_off[r] = ll ? r * g * d.cap : s_base[r * g];
+        }
     }
     if (tid == 0) {
         ws.rank_off[R] = ll ? E * d.cap : total;
@@ -571,8 +619,8 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const int32_t *__r
     // token are compared one by one; k, the lane's choice index, is kept up to
     // date in 32-bit arithmetic.
     const bool whole_tokens = (32 % K) == 0;
-    const int step_k = 32 % K;
-    int k = (int)(lo % K) + lane % K;
+    const int step_k = 32 % K, bits = id_bits(E);
+    int k = whole_tokens ? 0 : (int)lo % K + lane % K; // pair indices fit 31 bits
     if (k >= K) k -= K;
     for (int base = 0; base < n; base += 32) { // warp-uniform
         const int i = base + lane;
@@ -581,23 +629,22 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const int32_t *__r
             fl |= EP_FLAG_BAD_EXPERT_ID;
             e = -1;
         }
+        unsigned peers;
         if (whole_tokens) {
-            const unsigned tok = __match_any_sync(kFull, e >= 0 ? (e << 5) | (lane / K) : -1 - lane);
-            if (e >= 0 && (tok & lanemask_lt()) != 0) {
-                fl |= EP_FLAG_DUP_EXPERT_ID;
-                e = -1;
-            }
-        } else if (e >= 0) {
-            for (int k2 = 1; k2 <= k; ++k2) {
-                const int prev = i - k2 >= 0 ? ids[i - k2] : __ldg(idx + lo + i - k2); // token may start in the previous tile
-                if (prev == e) {
-                    fl |= EP_FLAG_DUP_EXPERT_ID;
-                    e = -1;
-                    break;
+            peers = whole_token_peers(e, K, bits, fl);
+        } else {
+            if (e >= 0) {
+                for (int k2 = 1; k2 <= k; ++k2) {
+                    const int prev = i - k2 >= 0 ? ids[i - k2] : __ldg(idx + lo + i - k2); // token may start in the previous tile
+                    if (prev == e) {
+                        fl |= EP_FLAG_DUP_EXPERT_ID;
+                        e = -1;
+                        break;
+                    }
                 }
             }
+            peers = warp_peers(e, bits, __ballot_sync(kFull, e >= 0));
         }
-        const unsigned peers = __match_any_sync(kFull, e >= 0 ? e : -1 - lane);
         const unsigned lower = peers & lanemask_lt();
         int packed = 0xffff;
         if (e >= 0) packed = e | ((my[e] + __popc(lower)) << 16);
@@ -810,8 +857,8 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     const int lo = w * ppw, hi = min(nc, lo + ppw);
     int32_t *my = s_wc + w * E;
     const bool whole_tokens = (32 % K) == 0; // ranges start at multiples of 32
-    const int step_k = 32 % K;
-    int k = (int)((c0 + lo) % K) + lane % K;
+    const int step_k = 32 % K, bits = id_bits(E);
+    int k = whole_tokens ? 0 : ((int)c0 + lo) % K + lane % K; // pair indices fit 31 bits
     if (k >= K) k -= K;
     uint32_t fl = 0;
     for (int base = lo; base < hi; base += 32) { // warp-uniform
@@ -821,23 +868,22 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
             fl |= EP_FLAG_BAD_EXPERT_ID;
             e = -1;
         }
+        unsigned peers;
         if (whole_tokens) {
-            const unsigned tok = __match_any_sync(kFull, e >= 0 ? (e << 5) | (lane / K) : -1 - lane);
-            if (e >= 0 && (tok & lanemask_lt()) != 0) {
-                fl |= EP_FLAG_DUP_EXPERT_ID;
-                e = -1;
-            }
-        } else if (e >= 0) {
-            for (int k2 = 1; k2 <= k; ++k2) {
-                const int prev = i - k2 >= 0 ? s_ids[i - k2] : __ldg(idx + c0 + i - k2);
-                if (prev == e) {
-                    fl |= EP_FLAG_DUP_EXPERT_ID;
-                    e = -1;
-                    break;
+            peers = whole_token_peers(e, K, bits, fl);
+        } else {
+            if (e >= 0) {
+                for (int k2 = 1; k2 <= k; ++k2) {
+                    const int prev = i - k2 >= 0 ? s_ids[i - k2] : __ldg(idx + c0 + i - k2);
+                    if (prev == e) {
+                        fl |= EP_FLAG_DUP_EXPERT_ID;
+                        e = -1;
+                        break;
+                    }
                 }
             }
+            peers = warp_peers(e, bits, __ballot_sync(kFull, e >= 0));
         }
-        const unsigned peers = __match_any_sync(kFull, e >= 0 ? e : -1 - lane);
         const unsigned lower = peers & lanemask_lt();
         if (i < hi) s_pk[i] = e >= 0 ? (e | ((my[e] + __popc(lower)) << 16)) : 0xffff;
         __syncwarp();
@@ -850,10 +896,15 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     __syncthreads();
     for (int e = tid; e < E; e += blockDim.x) { // per-warp bases and the CTA's totals
         int run = 0;
-        for (int ww = 0; ww < kClusterWarps; ++ww) {
-            const int v = s_wc[ww * E + e];
-            s_wc[ww * E + e] = run;
-            run += v;
+        for (int w0 = 0; w0 < kClusterWarps; w0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = s_wc[(w0 + u) * E + e];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                s_wc[(w0 + u) * E + e] = run;
+                run += v[u];
+            }
         }
         s_tot[e] = run;
     }
@@ -863,6 +914,7 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     //    each CTA's shared memory
     for (int e = tid; e < E; e += blockDim.x) {
         int before = 0, all = 0;
+#pragma unroll 8
         for (int q = 0; q < C; ++q) {
             const int v = cluster.map_shared_rank(s_tot, q)[e];
             if (q < r) before += v;

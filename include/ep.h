@@ -37,6 +37,13 @@
  *     read by ep_get_status.
  *   - A handle is not thread-safe; calls on one handle must be ordered by
  *     the caller (one stream, or explicit events).
+ *   - Kernels are launched with programmatic dependent launch. The routing
+ *     and router kernels let the next kernel of the stream start early, and
+ *     the dispatch kernels read their token rows x before waiting for the
+ *     kernels ahead of them. So a kernel of the caller's that writes x and is
+ *     itself launched with programmatic dependent launch must write x before
+ *     it triggers its dependents (kernels without that attribute need
+ *     nothing).
  */
 #ifndef EP_B200_H
 #define EP_B200_H
@@ -119,9 +126,11 @@ ep_status_t ep_recv_counts_len(const ep_config_t *cfg, int64_t *len);
 /* Device bytes ep_create will allocate for the handle's workspace. */
 ep_status_t ep_workspace_bytes(const ep_config_t *cfg, size_t *bytes);
 
-/* Number of kernels one ep_plan launches for this configuration (one for
- * small batches without a plan, else three); every other data call launches
- * one kernel. */
+/* Number of kernels one ep_plan launches for this configuration: one for
+ * batches of up to 1024 (token, k) pairs without a balanced plan, and for
+ * up to 32768 pairs when the current device can hold the routing cluster
+ * (asked of the device; reported as not holdable where there is no GPU),
+ * else three. Every other data call launches one kernel. */
 ep_status_t ep_plan_kernel_count(const ep_config_t *cfg, int32_t *count);
 
 /* "major.minor.patch" of the library. */

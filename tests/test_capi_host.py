@@ -87,6 +87,20 @@ def test_recv_rows_and_counts(L):
     assert L.ep_workspace_bytes(ctypes.byref(cfg), ctypes.byref(b)) == 0 and b.value > 0
 
 
+@pytest.mark.parametrize("kw,count", [
+    (dict(T=100, E=256, K=8, R=8), 1),            # 800 pairs: one CTA
+    (dict(T=32768, E=256, K=8, R=8), 3),          # 262144 pairs: three kernels
+    (dict(T=1024, E=256, K=8, R=8, balanced=True), 3),
+    (dict(T=100, E=256, K=8, R=8, balanced=True), 3),
+])
+def test_plan_kernel_count(L, kw, count):
+    """Counts that do not depend on the device (the cluster path, 1025 to
+    32768 pairs, asks the GPU whether its cluster fits)."""
+    n = ctypes.c_int32()
+    assert L.ep_plan_kernel_count(ctypes.byref(_cfg(**kw)), ctypes.byref(n)) == 0
+    assert n.value == count
+
+
 def test_null_arguments_rejected_without_gpu(L):
     assert L.ep_create(None, None) == 1
     assert L.ep_destroy(None) == 0

@@ -121,12 +121,54 @@ def test_several_tiles_ragged_tail(T, K):
     g.run_backward(r, seed=T)
 
 
-def test_long_rows_use_slab_loop():
-    """H = 20480 bf16 (2560 vectors) is longer than one CTA's registers hold."""
+@pytest.mark.parametrize("T,E,K,mode,cap", [(1100, 129, 6, "ht", 0), (4096, 256, 8, "ll", 100),
+                                             (2000, 1024, 5, "ht", 0), (1024, 384, 32, "ht", 0),
+                                             (3001, 200, 3, "ll", 64)])
+def test_cluster_routing_with_bad_and_repeated_ids(T, E, K, mode, cap):
+    """Batches of 1025..32768 pairs are routed by one launch of a cluster of
+    8 CTAs: expert counts that are not powers of two, top-k that does not
+    divide a warp (a token's earlier choices in the previous warp's range),
+    capacity drops, and masked, bad and repeated ids."""
     g = _gc()
-    r = g.run_forward(64, 20480, 16, 4, 4, seed=9)
+    H, R = 256, 4 if E % 4 == 0 else 1
+    x, idx, w = g.make_inputs(T, H, E, K, zipf_s=1.0, seed=T)
+    idx = idx.clone()
+    flat = idx.view(-1)
+    rng = np.random.default_rng(T)
+    # a repeat on a pair that starts a 32-pair word (its earlier choices sit
+    # in the previous word), elsewhere too
+    for p in list(range(32, T * K, 32 * 7)) + rng.integers(0, T * K, 40).tolist():
+        if p % K:
+            flat[p] = flat[p - 1]
+    flat[rng.integers(0, T * K, 25)] = -1
+    flat[rng.integers(0, T * K, 5)] = E + 3
+    h = ep.Ep(T, H, E, K, R, mode=mode, ll_capacity=cap)
+    assert ep.plan_launches(h) == 1
+    r = g.run_forward(T, H, E, K, R, mode=mode, cap=cap, idx=idx, w=w, x=x)
+    assert r["flags"] & oracle.FLAG_BAD_EXPERT_ID and r["flags"] & oracle.FLAG_DUP_EXPERT_ID
+    g.run_backward(r, seed=T)
+
+
+@pytest.mark.parametrize("T,H,fp8", [(1000, 7176, False), (1000, 7296, True), (300, 2056, False),
+                                      (64, 20480, False), (64, 40960, True)])
+def test_rows_split_across_ctas(T, H, fp8):
+    """Batches too small for several waves of one-row CTAs cut each row into
+    parts of whole warps of vectors, the last part ragged (897 vectors as
+    4 x 256 with 129 left over, 456 FP8 chunks as 256 + 200, 257 vectors)."""
+    g = _gc()
+    r = g.run_forward(T, H, 32, 4, 4, fp8=fp8, seed=H)
+    if not fp8:
+        g.run_backward(r, seed=H)
+
+
+def test_long_rows_use_slab_loop():
+    """Rows longer than one CTA's registers hold (2050 bf16 vectors, 2056 FP8
+    chunks) in a batch large enough to keep one CTA per row."""
+    g = _gc()
+    T = 40 * torch.cuda.get_device_properties(0).multi_processor_count
+    r = g.run_forward(T, 16400, 4, 1, 4, seed=9)
     g.run_backward(r, seed=9)
-    g.run_forward(64, 40960, 16, 4, 4, fp8=True, seed=9)
+    g.run_forward(T, 32896, 4, 1, 4, fp8=True, seed=9)
 
 
 # --------------------------------------------------------------- edge cases
