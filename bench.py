@@ -400,7 +400,7 @@ def run_native(args):
     avg = {k: sum(v) / len(v) for k, v in per.items()}
     peak, peak_kind = hbm_peak()
     dom = max((k for k in avg if k != "plan" or len(avg) == 1), key=lambda k: avg[k])
-    kname = KERNEL_OF.get(dom) or ("k_dispatch_fp8" if wl["fp8"] else "k_dispatch_bf16")
+    kname = KERNEL_OF.get(dom) or ("k_dispatch_fp8" if wl["fp8"] else "k_dispatch_bulk")
     achieved = nbytes[dom] / (avg[dom] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "call": dom, "kernel": kname, "achieved": round(achieved, 1), "peak": peak,
                 "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy)",

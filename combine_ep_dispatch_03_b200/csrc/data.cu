@@ -10,9 +10,11 @@
 // gradients of duplicated experts pass through a reduce buffer and are added
 // into the owner's gradients.
 //
-// Every kernel is a streaming row mover: one CTA per token row, 16-byte
-// vector loads/stores, each input row read once and each output row written
-// once, so the bytes moved are the algorithmic bytes.
+// Every kernel is a streaming row mover: one CTA per token row (or part of
+// one), each input row read once and each output row written once, so the
+// bytes moved are the algorithmic bytes. The bf16 dispatch moves its rows with
+// bulk copies (the TMA engine) through shared memory; the others use 16-byte
+// vector loads and stores from registers.
 #include <cuda_bf16.h>
 
 #include "ep_internal.cuh"
@@ -90,48 +92,129 @@ __device__ __forceinline__ void load_pairs(const uint4 *__restrict__ src, int c0
 }
 
 // ---------------------------------------------------------------------------
-// dispatch, bf16 payload: recv[dest_row[t,k]] = x[t]
+// Bulk copies (the TMA engine, no tensor map): cp.async.bulk between global
+// memory and this CTA's shared memory. Addresses and sizes are multiples of
+// 16 bytes (token rows are 16-byte aligned and H is a multiple of 8).
 // ---------------------------------------------------------------------------
-template <int VPT>
-__global__ void __launch_bounds__(256) k_dispatch_bf16(const uint4 *__restrict__ x, const int32_t *__restrict__ idx,
-                                                       const float *__restrict__ w,
-                                                       const int32_t *__restrict__ dest_row, int K, int nvec,
-                                                       int part, uint4 *__restrict__ recv, float *__restrict__ recv_w,
-                                                       int32_t *__restrict__ recv_expert,
-                                                       const int32_t *__restrict__ counts_src,
-                                                       int32_t *__restrict__ counts_dst, int counts_len) {
+constexpr uint64_t kWaitLimitNs = 2000000000ull; // a bounded wait gives up after 2 s
+constexpr int kBulkSlabVectors = 2048;             // 32 KB of shared memory per bulk-copy CTA
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// arm the barrier for `bytes` and start the load of global [src, src+bytes)
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// wait for phase `parity` of the barrier to complete, for at most kWaitLimitNs
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_test(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+
+// an L2 policy that marks lines evict-first (streamed output, as st.global.cs)
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes, uint64_t pol) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
+                 "r"(smem_u32(src)), "r"(bytes), "l"(pol)
+                 : "memory");
+}
+
+// every bulk store issued so far has finished reading shared memory
+__device__ __forceinline__ void bulk_stores_read() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+
+// ---------------------------------------------------------------------------
+// dispatch, bf16 payload, by bulk copies: one warp per (row, part); lane 0
+// loads the part into shared memory (before griddepcontrol.wait, as in
+// read_before_wait) and stores it to the K destination rows, a slab of at most
+// `slab` bytes at a time. The other lanes stage the routing.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) k_dispatch_bulk(const uint8_t *__restrict__ x, const int32_t *__restrict__ idx,
+                                                      const float *__restrict__ w,
+                                                      const int32_t *__restrict__ dest_row, int K, int row_bytes,
+                                                      int part_bytes, int slab, uint8_t *__restrict__ recv,
+                                                      float *__restrict__ recv_w, int32_t *__restrict__ recv_expert,
+                                                      const int32_t *__restrict__ counts_src,
+                                                      int32_t *__restrict__ counts_dst, int counts_len,
+                                                      uint32_t *__restrict__ status) {
+    extern __shared__ __align__(128) uint8_t s_row[];
+    __shared__ __align__(8) uint64_t s_bar;
     __shared__ int s_dest[kMaxTopk];
-    const int t = blockIdx.x;
-    const int64_t pb = (int64_t)t * K;
-    const int cb = blockIdx.y * part, n = min(part, nvec - cb); // this CTA's vectors of the row
-    const uint4 *src = x + (int64_t)t * nvec + cb;
-    const int step = VPT * blockDim.x;
-    uint4 v[VPT];
-    load_slab<VPT>(src, 0, n, v); // before the wait: see read_before_wait
+    const int t = blockIdx.x, lane = threadIdx.x;
+    const int cb = blockIdx.y * part_bytes, n = min(part_bytes, row_bytes - cb); // this CTA's bytes of the row
+    const uint8_t *src = x + (int64_t)t * row_bytes + cb;
+    if (lane == 0) {
+        mbar_init(&s_bar);
+        bulk_load(s_row, src, (uint32_t)min(n, slab), &s_bar);
+    }
     pdl_wait(); // no early trigger: measured slower for these multi-wave grids
-    if (threadIdx.x < K) {
-        const int dr = dest_row[pb + threadIdx.x];
-        s_dest[threadIdx.x] = dr;
+    const int64_t pb = (int64_t)t * K;
+    if (lane < K) {
+        const int dr = dest_row[pb + lane];
+        s_dest[lane] = dr;
         if (dr >= 0 && blockIdx.y == 0) {
-            if (recv_w) recv_w[dr] = w[pb + threadIdx.x];
-            if (recv_expert) recv_expert[dr] = idx[pb + threadIdx.x];
+            if (recv_w) recv_w[dr] = w[pb + lane];
+            if (recv_expert) recv_expert[dr] = idx[pb + lane];
         }
     }
     if (t == 0 && blockIdx.y == 0 && counts_dst)
-        for (int i = threadIdx.x; i < counts_len; i += blockDim.x) counts_dst[i] = counts_src[i];
-    for (int c0 = 0; c0 < n; c0 += step) {
-        if (c0 > 0) load_slab<VPT>(src, c0, n, v);
-        if (c0 == 0) __syncthreads();
+        for (int i = lane; i < counts_len; i += 32) counts_dst[i] = counts_src[i];
+    __syncwarp();
+    if (lane != 0) return;
+    uint32_t parity = 0;
+    for (int off = 0; off < n; off += slab, parity ^= 1u) {
+        const int len = min(slab, n - off);
+        if (off > 0) bulk_load(s_row, src + off, (uint32_t)len, &s_bar);
+        if (!mbar_wait(&s_bar, parity)) {
+            atomicOr(status, EP_FLAG_WAIT_TIMEOUT);
+            mbar_wait(&s_bar, parity); // the load in flight still writes s_row
+            return;
+        }
+        const uint64_t pol = policy_evict_first();
         for (int k = 0; k < K; ++k) {
             const int dr = s_dest[k];
             if (dr < 0) continue;
-            uint4 *dst = recv + (int64_t)dr * nvec + cb;
-#pragma unroll
-            for (int i = 0; i < VPT; ++i) {
-                const int c = c0 + threadIdx.x + i * blockDim.x;
-                if (c < n) __stcs(dst + c, v[i]);
-            }
+            bulk_store(recv + (int64_t)dr * row_bytes + cb + off, s_row, (uint32_t)len, pol);
         }
+        bulk_stores_read(); // before s_row is reloaded, and before the CTA exits
     }
 }
 
@@ -457,9 +540,10 @@ cudaError_t launch_dispatch(const Dims &d, const Workspace &ws, const void *x, c
         const int nvec = d.H / 8;
         const int part = row_part(d.T, nvec);
         const dim3 grid(d.T, (nvec + part - 1) / part);
-        pick_shape(part, &per, &threads);
-        EPB_SWITCH_VPT(per, k_dispatch_bf16, (const uint4 *)x, topk_idx, topk_w, ws.dest_row, d.K, nvec, part,
-                       (uint4 *)recv_x, recv_w, recv_expert, ws.recv_counts, recv_counts, d.counts_len);
+        const int slab = min(part, kBulkSlabVectors) * 16;
+        err = launch_pdl(k_dispatch_bulk, grid, dim3(32), (size_t)slab, st, (const uint8_t *)x, topk_idx, topk_w,
+                         ws.dest_row, d.K, nvec * 16, part * 16, slab, (uint8_t *)recv_x, recv_w, recv_expert,
+                         ws.recv_counts, recv_counts, d.counts_len, ws.flags);
     }
     return err;
 }

@@ -70,6 +70,8 @@ typedef enum ep_status {
 #define EP_FLAG_DUP_EXPERT_ID 0x2 /* a token chose the same expert twice */
 #define EP_FLAG_CAPACITY 0x4      /* LL: an expert received more than ll_capacity rows */
 #define EP_FLAG_PLAN_SLOTS 0x8    /* balanced plan ran out of replica slots */
+#define EP_FLAG_WAIT_TIMEOUT 0x10 /* a kernel's bounded wait for its own copy gave up
+                                     (after 2 s); that call's outputs are incomplete */
 
 typedef enum ep_mode { EP_MODE_LL = 0, EP_MODE_HT = 1 } ep_mode_t;
 
