@@ -22,11 +22,11 @@
 //                   destination row through the layout tables (each CTA
 //                   computes the plain layouts' expert offsets itself)
 // Batches up to 32768 pairs without a plan, one kernel:
-//   k_route_cluster a thread-block cluster of 8 CTAs; each CTA counts
-//                   and ranks its share of the pairs in shared memory, the
-//                   CTAs exchange per-expert totals through distributed
-//                   shared memory across two cluster barriers, and each then
-//                   assigns its own pairs
+//   k_route_cluster a thread-block cluster of 8 or 16 CTAs; each CTA counts
+//                   and ranks its share of the pairs in shared memory, stores
+//                   its per-expert totals into every CTA's shared memory
+//                   (distributed shared memory) before one cluster barrier,
+//                   and then assigns its own pairs
 // Tiny batches without a plan, one kernel:
 //   k_route_small   one CTA does all of the above in shared memory
 #include <cooperative_groups.h>
@@ -826,29 +826,30 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspac
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t *__restrict__ idx, Dims d,
                                                                     Workspace ws) {
+    // first phase of the cluster barrier: this CTA is running. Its wait, just
+    // before the first store into another CTA's shared memory, finds every
+    // CTA of the cluster started.
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     pdl_wait();
     pdl_launch_dependents();
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks(), r = (int)cluster.block_rank();
     extern __shared__ int32_t sm[];
     __shared__ int32_t s_warp[33];
-    __shared__ uint32_t s_fl, s_fl_all;
+    __shared__ uint32_t s_fl, s_flq[16]; // s_flq[q]: flags of CTA q (pushed by q)
     const int E = d.E, K = d.K, lane = threadIdx.x & 31, w = threadIdx.x >> 5, tid = threadIdx.x;
     const int ppw = d.cl_ppw, ppc = ppw * kClusterWarps;
     const int64_t c0 = (int64_t)r * ppc;
     const int nc = (int)max((int64_t)0, min((int64_t)ppc, d.L - c0));
     int32_t *s_wc = sm;                     // [warps][E]: per-warp counts, then per-warp bases
-    int32_t *s_tot = s_wc + kClusterWarps * E; // [E]: this CTA's totals (read by the other CTAs)
-    int32_t *s_cta = s_tot + E;             // [E]: pairs of each expert in lower-ranked CTAs
+    int32_t *s_all = s_wc + kClusterWarps * E; // [C][E]: every CTA's totals (pushed by each CTA)
+    int32_t *s_cta = s_all + C * E;         // [E]: pairs of each expert in lower-ranked CTAs
     int32_t *s_cnt = s_cta + E;             // [E]: routed pairs per expert (whole batch)
     int32_t *s_len = s_cnt + E;             // [E]: kept rows per expert
     int32_t *s_off = s_len + E;             // [E]: first row of each expert
     int32_t *s_ids = s_off + E;             // [ppc]: this CTA's expert ids
     int32_t *s_pk = s_ids + ppc;            // [ppc]: packed (expert, rank in warp range)
-    if (tid == 0) {
-        s_fl = 0;
-        s_fl_all = 0;
-    }
+    if (tid == 0) s_fl = 0;
     for (int i = tid; i < kClusterWarps * E; i += blockDim.x) s_wc[i] = 0;
     for (int i = tid; i < nc; i += blockDim.x) s_ids[i] = __ldg(idx + c0 + i);
     __syncthreads();
@@ -894,7 +895,9 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     }
     block_or(fl, &s_fl);
     __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) { // per-warp bases and the CTA's totals
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); // every CTA has started
+    if (tid < C) *cluster.map_shared_rank(&s_flq[r], tid) = s_fl;
+    for (int e = tid; e < E; e += blockDim.x) { // per-warp bases; the CTA's totals go to every CTA
         int run = 0;
         for (int w0 = 0; w0 < kClusterWarps; w0 += 8) {
             int v[8];
@@ -906,29 +909,30 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
                 run += v[u];
             }
         }
-        s_tot[e] = run;
+#pragma unroll 8
+        for (int q = 0; q < C; ++q) cluster.map_shared_rank(s_all, q)[r * E + e] = run;
     }
-    cluster.sync(); // every CTA's totals and flags are complete
+    // every CTA's stores into this CTA's shared memory are visible after the
+    // barrier, and no CTA touches another's shared memory after it
+    cluster.sync();
 
-    // 2. totals of the whole batch and of the lower-ranked CTAs, read from
-    //    each CTA's shared memory
+    // 2. totals of the whole batch and of the lower-ranked CTAs, all local now
     for (int e = tid; e < E; e += blockDim.x) {
         int before = 0, all = 0;
 #pragma unroll 8
         for (int q = 0; q < C; ++q) {
-            const int v = cluster.map_shared_rank(s_tot, q)[e];
+            const int v = s_all[q * E + e];
             if (q < r) before += v;
             all += v;
         }
         s_cta[e] = before;
         s_cnt[e] = all;
     }
-    if (tid < C) {
-        const uint32_t v = *cluster.map_shared_rank(&s_fl, tid);
-        if (v) atomicOr(&s_fl_all, v);
+    if (tid == 0) {
+        uint32_t f = 0;
+        for (int q = 0; q < C; ++q) f |= s_flq[q];
+        s_fl = f;
     }
-    cluster.sync(); // no remote reads after this point; s_fl_all complete
-    if (tid == 0) s_fl = s_fl_all;
     __syncthreads();
 
     // 3. layout (every CTA computes it; CTA 0 publishes it) and assignment
@@ -1019,7 +1023,7 @@ size_t route_smem_hist(const Dims &d) { return sizeof(int32_t) * (size_t)kRouteW
 size_t route_smem_small(const Dims &d) { return sizeof(int32_t) * ((size_t)(kSmallWarps + 3) * d.E + d.L); }
 
 size_t route_smem_cluster(const Dims &d) {
-    return sizeof(int32_t) * ((size_t)(kClusterWarps + 5) * d.E + 2 * (size_t)d.cl_ppw * kClusterWarps);
+    return sizeof(int32_t) * ((size_t)(kClusterWarps + 4 + d.cl_size) * d.E + 2 * (size_t)d.cl_ppw * kClusterWarps);
 }
 
 // Can a cluster of d.cl_size CTAs of this kernel be resident at once on this
