@@ -225,6 +225,33 @@ __global__ void __launch_bounds__(32) k_dispatch_bulk(const uint8_t *__restrict_
 // One thread owns 16 consecutive elements (two 16-byte loads, one 16-byte
 // store); the 8 threads of a 128-block are 8 consecutive lanes.
 // ---------------------------------------------------------------------------
+// One 16-element chunk (two 16-byte halves of bf16) to 16 e4m3 codes and its
+// block's scale. Every lane of the warp calls it at once: the block's amax is
+// reduced over the 8 lanes holding the block.
+__device__ __forceinline__ void quant_chunk(const uint4 &a, const uint4 &b, uint4 &q, float &sc) {
+    float f[16];
+    unpack8(a, f);
+    unpack8(b, f + 8);
+    float amax = 0.0f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) amax = fmaxf(amax, fabsf(f[u]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    const float s = __fdiv_rn(amax, 448.0f);
+    sc = s;
+    uint32_t wd[4] = {0u, 0u, 0u, 0u};
+    if (amax != 0.0f) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t lo = e4m3x2(__fdiv_rn(f[4 * u], s), __fdiv_rn(f[4 * u + 1], s));
+            const uint32_t hi = e4m3x2(__fdiv_rn(f[4 * u + 2], s), __fdiv_rn(f[4 * u + 3], s));
+            wd[u] = lo | (hi << 16);
+        }
+    }
+    q = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+}
+
 template <int CPT>
 __global__ void __launch_bounds__(256) k_dispatch_fp8(const uint4 *__restrict__ x, const int32_t *__restrict__ idx,
                                                       const float *__restrict__ w,
@@ -259,29 +286,7 @@ __global__ void __launch_bounds__(256) k_dispatch_fp8(const uint4 *__restrict__ 
         uint4 q[CPT];
         float sc[CPT];
 #pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-            float f[16];
-            unpack8(a[i], f);
-            unpack8(b[i], f + 8);
-            float amax = 0.0f;
-#pragma unroll
-            for (int u = 0; u < 16; ++u) amax = fmaxf(amax, fabsf(f[u]));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-            const float s = __fdiv_rn(amax, 448.0f);
-            sc[i] = s;
-            uint32_t wd[4] = {0u, 0u, 0u, 0u};
-            if (amax != 0.0f) {
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint32_t lo = e4m3x2(__fdiv_rn(f[4 * u], s), __fdiv_rn(f[4 * u + 1], s));
-                    const uint32_t hi = e4m3x2(__fdiv_rn(f[4 * u + 2], s), __fdiv_rn(f[4 * u + 3], s));
-                    wd[u] = lo | (hi << 16);
-                }
-            }
-            q[i] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-        }
+        for (int i = 0; i < CPT; ++i) quant_chunk(a[i], b[i], q[i], sc[i]);
         if (c0 == 0) __syncthreads();
         for (int k = 0; k < K; ++k) {
             const int dr = s_dest[k];
