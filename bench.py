@@ -325,12 +325,18 @@ class Step:
         return plan_launches(self.h) + len(self.calls) - 1
 
 
-def timed(step: Step, steps, warmup, stream, breakdown_steps=None):
+def timed(step: Step, steps, warmup, stream, breakdown_steps=None, graph=True):
     """Warm-up, then `steps` steps back to back between two CUDA events on the
     launching stream (the step time), then `breakdown_steps` more with an
     event between every two calls (the per-call split; events between calls
     stop consecutive kernels from overlapping their launches, so this loop
-    runs slightly slower). Returns (total_ms, {call: [ms per step]})."""
+    runs slightly slower). Returns (total_ms, {call: [ms per step]}).
+
+    With `graph`, the timed steps are replays of CUDA graphs captured from the
+    same calls (a graph of up to 10 steps, and one of a single step for the
+    remainder): the same kernels with the same programmatic launch edges,
+    without the host's per-launch cost, which otherwise bounds steps of a few
+    microseconds."""
     import torch
 
     with torch.cuda.stream(stream):
@@ -338,12 +344,36 @@ def timed(step: Step, steps, warmup, stream, breakdown_steps=None):
             step.run(stream)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for _ in range(steps):
-            step.run(stream)
-        end.record(stream)
-    torch.cuda.synchronize()
+    if graph:
+        chunk = min(steps, 10)
+        graphs = {}
+        for n in sorted({chunk, steps % chunk} - {0}):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(n):
+                    step.run(stream)
+            graphs[n] = g
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, warmup // chunk)):
+                graphs[chunk].replay()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(steps // chunk):
+                graphs[chunk].replay()
+            if steps % chunk:
+                graphs[steps % chunk].replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        del graphs
+    else:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(steps):
+                step.run(stream)
+            end.record(stream)
+        torch.cuda.synchronize()
     total = start.elapsed_time(end)
     nb = steps if breakdown_steps is None else breakdown_steps
     n = len(step.calls)
@@ -391,7 +421,7 @@ def run_native(args):
     barrier(world)
     torch.cuda.synchronize()
     sampler.start()
-    total_ms, per = timed(step, args.steps, args.warmup, stream, min(args.steps, 50))
+    total_ms, per = timed(step, args.steps, args.warmup, stream, min(args.steps, 50), graph=not args.no_graph)
     clocks = sampler.stop()
     barrier(world)
     value, ms_step = weak_scaling_value(step_bytes, total_ms / args.steps, world)
@@ -421,7 +451,8 @@ def run_native(args):
                                else "bf16 dispatch") + " -> bf16 combine (fp32 accumulation)",
                    "l2": ("no flush: the receive buffer (%.2f GB) and the expert rows exceed L2 (126 MB)"
                           % (big / 1e9)) if big > 2 * 126e6 else "working set partly L2-resident, no flush",
-                   "parallelism": f"{world} independent EP worlds (one per GPU), R logical ranks each"},
+                   "parallelism": f"{world} independent EP worlds (one per GPU), R logical ranks each",
+                   "launch": "stream" if args.no_graph else "CUDA graph replay of the captured step calls"},
         "tokens_per_s": round(world * wl["T"] / (ms_step * 1e-3), 1),
         "rows_per_s": round(world * step.placed / (ms_step * 1e-3), 1),
         "frac_of_hbm": round(step_bytes / (ms_step * 1e-3) / 1e9 / peak, 4),
@@ -637,6 +668,7 @@ def main():
     ap.add_argument("--zipf", type=float, default=None, help="override the router's Zipf bias s")
     ap.add_argument("--balanced", type=int, choices=[0, 1], default=None, help="override the balanced plan")
     ap.add_argument("--capacity", type=int, default=0, help="override the LL per-expert capacity (smaller buffers)")
+    ap.add_argument("--no-graph", action="store_true", help="time stream launches instead of CUDA-graph replays")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
