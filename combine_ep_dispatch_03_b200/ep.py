@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libep_b200.so")
 
 MODE_LL, MODE_HT = 0, 1
 FLAG_BAD_EXPERT_ID, FLAG_DUP_EXPERT_ID, FLAG_CAPACITY, FLAG_PLAN_SLOTS = 0x1, 0x2, 0x4, 0x8
+FLAG_WAIT_TIMEOUT = 0x10  # a bounded wait inside a kernel gave up; that call's outputs are incomplete
 (T_DEST_ROW, T_EXPERT_COUNTS, T_RECV_COUNTS, T_RANK_LOAD, T_RANK_OFFSET, T_REPLICA_EXPERT, T_DIRECT_COUNT,
  T_DIRECT_EXPERT, T_DIRECT_LEN) = range(9)
 
