@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(256) k_dispatch_fp8(const uint4 *__restrict__ 
             for (int i = 0; i < CPT; ++i) {
                 const int c = c0 + threadIdx.x + i * blockDim.x;
                 if (c < n) {
-                    __stcs(dst + c, q[i]);
+                    dst[c] = q[i]; // write-back: measured faster here than st.global.cs
                     if ((c & 7) == 0) scales[(int64_t)dr * nb + ((cb + c) >> 3)] = sc[i];
                 }
             }
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(256) k_dispatch_fp8(const uint4 *__restrict__ 
 // combine: out[t] = bf16(fold_k fmaf(w[t,k], y[dest_row[t,k]], acc)), k in
 // order, acc from +0; UNIT: unweighted fp32 sum (dispatch backward).
 // ---------------------------------------------------------------------------
-template <int CPT, bool UNIT>
+template <int CPT, bool UNIT, bool CS>
 __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, const float *__restrict__ w,
                                                  const int32_t *__restrict__ dest_row, int K, int nvec,
                                                  int part, uint4 *__restrict__ out) {
@@ -335,7 +335,8 @@ __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, co
                 for (int kk = 0; kk < 8; ++kk) {
                     const int k = k0 + kk;
                     const int dr = k < K ? s_dest[k] : -1;
-                    v[kk] = dr >= 0 ? __ldcs(yb + (int64_t)dr * nvec + c) : make_uint4(0, 0, 0, 0);
+                    const uint4 *p = yb + (int64_t)dr * nvec + c;
+                    v[kk] = dr >= 0 ? (CS ? __ldcs(p) : *p) : make_uint4(0, 0, 0, 0);
                 }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -353,7 +354,7 @@ __global__ void __launch_bounds__(256) k_combine(const uint4 *__restrict__ y, co
                     }
                 }
             }
-            __stcs(out + (int64_t)t * nvec + cb + c, pack8(acc));
+            out[(int64_t)t * nvec + cb + c] = pack8(acc); // write-back: measured faster than .cs
         }
     }
 }
@@ -473,12 +474,12 @@ __global__ void __launch_bounds__(kCopyThreads) k_prefetch(const uint4 *__restri
 #pragma unroll
         for (int u = 0; u < kCopyUnroll; ++u) {
             const int64_t i = base + (int64_t)u * kCopyThreads;
-            if (i < V) v[u] = __ldcs(src + i);
+            if (i < V) v[u] = src[i];
         }
 #pragma unroll
         for (int u = 0; u < kCopyUnroll; ++u) {
             const int64_t i = base + (int64_t)u * kCopyThreads;
-            if (i < V) __stcs(dst + i, v[u]);
+            if (i < V) dst[i] = v[u];
         }
     }
 }
@@ -578,21 +579,28 @@ cudaError_t launch_combine(const Dims &d, const Workspace &ws, const void *y, co
     const uint4 *yy = (const uint4 *)y;
     uint4 *oo = (uint4 *)out;
     const dim3 block(threads);
-    if (topk_w) {
-        switch (per) {
-        case 1: return launch_pdl(k_combine<1, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, part, oo);
-        case 2: return launch_pdl(k_combine<2, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, part, oo);
-        case 4: return launch_pdl(k_combine<4, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, part, oo);
-        default: return launch_pdl(k_combine<8, false>, grid, block, 0, st, yy, topk_w, ws.dest_row, d.K, nvec, part, oo);
-        }
-    }
+    // Streaming (evict-first) loads measured faster when rows are cut into parts
+    // (LL decode: combine 28.9 vs 31.7 us) and slower for whole rows (HT
+    // prefill: 646 vs 619 us), so they are used only for parts.
+    const bool cs = part < nvec;
     const float *none = nullptr;
-    switch (per) {
-    case 1: return launch_pdl(k_combine<1, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, part, oo);
-    case 2: return launch_pdl(k_combine<2, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, part, oo);
-    case 4: return launch_pdl(k_combine<4, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, part, oo);
-    default: return launch_pdl(k_combine<8, true>, grid, block, 0, st, yy, none, ws.dest_row, d.K, nvec, part, oo);
+#define EPB_COMBINE(C, U, S, W)                                                                                      \
+    return launch_pdl(k_combine<C, U, S>, grid, block, 0, st, yy, W, ws.dest_row, d.K, nvec, part, oo)
+#define EPB_COMBINE_CPT(U, S, W)                                                                                     \
+    switch (per) {                                                                                                   \
+    case 1: EPB_COMBINE(1, U, S, W);                                                                                 \
+    case 2: EPB_COMBINE(2, U, S, W);                                                                                 \
+    case 4: EPB_COMBINE(4, U, S, W);                                                                                 \
+    default: EPB_COMBINE(8, U, S, W);                                                                                \
     }
+    if (topk_w) {
+        if (cs) EPB_COMBINE_CPT(false, true, topk_w)
+        EPB_COMBINE_CPT(false, false, topk_w)
+    }
+    if (cs) EPB_COMBINE_CPT(true, true, none)
+    EPB_COMBINE_CPT(true, false, none)
+#undef EPB_COMBINE_CPT
+#undef EPB_COMBINE
 }
 
 cudaError_t launch_prefetch(const Dims &d, const Workspace &ws, const void *weights, int64_t bytes_per_expert,
