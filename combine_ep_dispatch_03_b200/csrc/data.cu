@@ -18,6 +18,7 @@
 #include <cuda_bf16.h>
 
 #include "ep_internal.cuh"
+#include "fast_div.cuh"
 
 namespace epb {
 namespace {
@@ -242,12 +243,22 @@ __device__ __forceinline__ void quant_chunk(const uint4 &a, const uint4 &b, uint
     sc = s;
     uint32_t wd[4] = {0u, 0u, 0u, 0u};
     if (amax != 0.0f) {
+        const float y = __frcp_rn(s);
+        float minnz = INFINITY;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const uint32_t lo = e4m3x2(__fdiv_rn(f[4 * u], s), __fdiv_rn(f[4 * u + 1], s));
-            const uint32_t hi = e4m3x2(__fdiv_rn(f[4 * u + 2], s), __fdiv_rn(f[4 * u + 3], s));
-            wd[u] = lo | (hi << 16);
+        for (int u = 0; u < 16; ++u) {
+            const float m = fabsf(f[u]);
+            minnz = fminf(minnz, m > 0.0f ? m : INFINITY);
         }
+        if (fast_group_ok(amax, minnz, y)) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) f[u] = div_by_scale_fast(f[u], s, y);
+        } else {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) f[u] = __fdiv_rn(f[u], s);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) wd[u] = e4m3x2(f[4 * u], f[4 * u + 1]) | (e4m3x2(f[4 * u + 2], f[4 * u + 3]) << 16);
     }
     q = make_uint4(wd[0], wd[1], wd[2], wd[3]);
 }

@@ -259,6 +259,34 @@ def test_zero_blocks_and_large_values_fp8():
     assert r["fp8_diff"] == 0
 
 
+def test_fp8_cast_across_the_bf16_range():
+    """Blocks scaled from 2^-133 to 2^120, with elements spread 2^40 below
+    the block's largest and some exact zeros of either sign. The cast's
+    division takes its reciprocal-and-correction path inside a range of
+    block scales and elements and the full division outside it; both must
+    give the oracle's e4m3 codes and scales bit for bit."""
+    g = _gc()
+    T, H, E, K, R = 256, 1024, 16, 2, 4
+    _, idx, w = g.make_inputs(T, H, E, K, seed=21)
+    rng = np.random.default_rng(21)
+    nb = T * H // 128
+    block_exp = rng.integers(-133, 121, nb).astype(np.float64)
+    spread = rng.uniform(-40.0, 0.0, (nb, 128))  # each element up to 2^40 below its block's top
+    mant = rng.uniform(1.0, 2.0, (nb, 128)) * rng.choice([-1.0, 1.0], (nb, 128))
+    vals = mant * np.exp2(block_exp[:, None] + np.floor(spread))
+    vals[rng.random((nb, 128)) < 0.02] = 0.0
+    neg0 = rng.random((nb, 128)) < 0.01
+    x = torch.from_numpy(vals.reshape(T, H)).to(torch.bfloat16)
+    x[torch.from_numpy(neg0.reshape(T, H))] = -0.0
+    assert torch.isfinite(x.float()).all()
+    r = g.run_forward(T, H, E, K, R, fp8=True, idx=idx, w=w, x=x, check_combine=False)
+    assert r["fp8_diff"] == 0
+    # byte for byte, so that a zero of the wrong sign shows too
+    ref = r["ref"]
+    codes = oracle.dispatch(x, idx, w, ref.dest_row, ref.recv_rows, fp8=True)[0]
+    np.testing.assert_array_equal(g.bits8(r["bufs"]["recv_x"])[r["rows"]], codes[r["rows"]])
+
+
 def test_plan_is_reused_by_backward_after_other_work():
     """Routing state lives in the handle from one ep_plan to the next (forward
     and backward share it); a second plan with new routing replaces it."""
