@@ -206,7 +206,9 @@ ep_status_t ep_plan(ep_handle_t *h, const int32_t *topk_idx, void *stream);
  * the rows per local slot. Rows no pair targets (LL padding) are not
  * written. x: device bf16 [T, H]. topk_idx must be the array given to the
  * last ep_plan (it may be NULL when recv_expert is NULL). recv_scales must
- * be non-NULL iff cfg.fp8. */
+ * be non-NULL iff cfg.fp8. The bf16 payload moves by bulk copies through
+ * shared memory; their completion wait is bounded, and a wait that runs out
+ * (2 s) sets EP_FLAG_WAIT_TIMEOUT instead of hanging. */
 ep_status_t ep_dispatch(ep_handle_t *h, const void *x, const int32_t *topk_idx, const float *topk_w,
                         void *recv_x, float *recv_scales, float *recv_w, int32_t *recv_expert,
                         int32_t *recv_counts, void *stream);
