@@ -25,7 +25,7 @@ constexpr int kRouterMaxExperts = 1024;   // ep_router_topk keeps a token's logi
 constexpr int kMaxRouteSmem = 200 * 1024; // dynamic shared memory cap of the routing kernels
 constexpr int kSmallMaxPairs = 1024;      // single-CTA routing up to this many pairs ...
 constexpr int kSmallMaxExperts = 512;     // ... and experts (plain layouts only)
-constexpr int kClusterThreads = 1024;     // one-launch cluster routing: threads per CTA
+constexpr int kClusterThreads = 1024;     // one-launch cluster routing: threads per CTA, at most
 constexpr int kClusterWarps = kClusterThreads / 32;
 constexpr int kClusterMaxPairs = 32768;  // ... up to this many (token, k) pairs
 
@@ -72,6 +72,7 @@ struct Dims {
     int ntiles, nhist;       // warp tiles, histogram CTAs
     int nassign;             // CTAs of the slot-assignment kernel
     int cl_size, cl_ppw;     // cluster routing: CTAs (8 or 16, 0 = not used), pairs per warp
+    int cl_warps;            // cluster routing: warps per CTA (16 or 32)
     int nx_max;              // bound on extra pieces (R*S + E with a plan, else 0)
     int counts_len;          // recv_counts entries
 };

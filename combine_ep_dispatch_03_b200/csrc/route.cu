@@ -40,7 +40,7 @@ namespace epb {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-static_assert(kClusterWarps % 8 == 0, "the cluster kernel sums warp counts 8 at a time");
+static_assert(kClusterWarps % 8 == 0, "the cluster kernel sums warp counts 8 at a time (16 or 32 warps)");
 constexpr int kSmallThreads = 1024;
 constexpr int kSmallWarps = kSmallThreads / 32;
 
@@ -838,11 +838,12 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     __shared__ int32_t s_warp[33];
     __shared__ uint32_t s_fl, s_flq[16]; // s_flq[q]: flags of CTA q (pushed by q)
     const int E = d.E, K = d.K, lane = threadIdx.x & 31, w = threadIdx.x >> 5, tid = threadIdx.x;
-    const int ppw = d.cl_ppw, ppc = ppw * kClusterWarps;
+    const int NW = d.cl_warps; // warps per CTA (blockDim.x / 32)
+    const int ppw = d.cl_ppw, ppc = ppw * NW;
     const int64_t c0 = (int64_t)r * ppc;
     const int nc = (int)max((int64_t)0, min((int64_t)ppc, d.L - c0));
     int32_t *s_wc = sm;                     // [warps][E]: per-warp counts, then per-warp bases
-    int32_t *s_all = s_wc + kClusterWarps * E; // [C][E]: every CTA's totals (pushed by each CTA)
+    int32_t *s_all = s_wc + NW * E;         // [C][E]: every CTA's totals (pushed by each CTA)
     int32_t *s_cta = s_all + C * E;         // [E]: pairs of each expert in lower-ranked CTAs
     int32_t *s_cnt = s_cta + E;             // [E]: routed pairs per expert (whole batch)
     int32_t *s_len = s_cnt + E;             // [E]: kept rows per expert
@@ -850,7 +851,7 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     int32_t *s_ids = s_off + E;             // [ppc]: this CTA's expert ids
     int32_t *s_pk = s_ids + ppc;            // [ppc]: packed (expert, rank in warp range)
     if (tid == 0) s_fl = 0;
-    for (int i = tid; i < kClusterWarps * E; i += blockDim.x) s_wc[i] = 0;
+    for (int i = tid; i < NW * E; i += blockDim.x) s_wc[i] = 0;
     for (int i = tid; i < nc; i += blockDim.x) s_ids[i] = __ldg(idx + c0 + i);
     __syncthreads();
 
@@ -899,7 +900,7 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     if (tid < C) *cluster.map_shared_rank(&s_flq[r], tid) = s_fl;
     for (int e = tid; e < E; e += blockDim.x) { // per-warp bases; the CTA's totals go to every CTA
         int run = 0;
-        for (int w0 = 0; w0 < kClusterWarps; w0 += 8) {
+        for (int w0 = 0; w0 < NW; w0 += 8) {
             int v[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) v[u] = s_wc[(w0 + u) * E + e];
@@ -1023,24 +1024,24 @@ size_t route_smem_hist(const Dims &d) { return sizeof(int32_t) * (size_t)kRouteW
 size_t route_smem_small(const Dims &d) { return sizeof(int32_t) * ((size_t)(kSmallWarps + 3) * d.E + d.L); }
 
 size_t route_smem_cluster(const Dims &d) {
-    return sizeof(int32_t) * ((size_t)(kClusterWarps + 4 + d.cl_size) * d.E + 2 * (size_t)d.cl_ppw * kClusterWarps);
+    return sizeof(int32_t) * ((size_t)(d.cl_warps + 4 + d.cl_size) * d.E + 2 * (size_t)d.cl_ppw * d.cl_warps);
 }
 
 // Can a cluster of d.cl_size CTAs of this kernel be resident at once on this
 // device? (Asked once per device and size.)
 static bool cluster_fits(const Dims &d) {
-    static signed char ok[64][2][64]; // [device][size 8/16][smem in 4 KB steps], 0 unknown, 1 yes, -1 no
+    static signed char ok[64][2][2][64]; // [device][size 8/16][16/32 warps][smem in 4 KB steps]: 0 unknown, 1 yes, -1 no
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     const size_t smem = route_smem_cluster(d);
-    const int si = d.cl_size == 16 ? 1 : 0, mi = (int)((smem + 4095) / 4096);
+    const int si = d.cl_size == 16 ? 1 : 0, wi = d.cl_warps == 32 ? 1 : 0, mi = (int)((smem + 4095) / 4096);
     if (mi >= 64) return false;
-    if (ok[dev][si][mi] == 0) {
+    if (ok[dev][si][wi][mi] == 0) {
         cudaFuncSetAttribute(k_route_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxRouteSmem);
         cudaFuncSetAttribute(k_route_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(d.cl_size);
-        cfg.blockDim = dim3(kClusterThreads);
+        cfg.blockDim = dim3(d.cl_warps * 32);
         cfg.dynamicSmemBytes = (size_t)mi * 4096;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1052,9 +1053,9 @@ static bool cluster_fits(const Dims &d) {
         int n = 0;
         const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, k_route_cluster, &cfg);
         if (e != cudaSuccess) cudaGetLastError();
-        ok[dev][si][mi] = (e == cudaSuccess && n >= 1) ? 1 : -1;
+        ok[dev][si][wi][mi] = (e == cudaSuccess && n >= 1) ? 1 : -1;
     }
-    return ok[dev][si][mi] == 1;
+    return ok[dev][si][wi][mi] == 1;
 }
 
 bool route_use_cluster(const Dims &d) {
@@ -1081,7 +1082,7 @@ cudaError_t launch_plan(const Dims &d, const Workspace &ws, const int32_t *topk_
     if (route_use_cluster(d)) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(d.cl_size);
-        cfg.blockDim = dim3(kClusterThreads);
+        cfg.blockDim = dim3(d.cl_warps * 32);
         cfg.dynamicSmemBytes = route_smem_cluster(d);
         cfg.stream = st;
         cudaLaunchAttribute attr[2];
