@@ -289,6 +289,53 @@ class Step:
         for _, f in self.calls:
             f(st)
 
+    def e2e_sets(self):
+        """Two sets of device inputs and outputs for the end-to-end leg, each
+        with the step's calls bound to it: (host->device copies, device
+        outputs, run(stream)). Set 0 is the step's own buffers; set 1 twins
+        them, so that one set's copies can run while the other's kernels do.
+        The handle, the receive buffers and the resident stand-ins are shared
+        (the kernels of consecutive steps run in order on one stream)."""
+        import torch
+
+        from combine_ep_dispatch_03_b200 import ep
+
+        def twin(t, b):
+            return t if b == 0 else torch.empty_like(t)
+
+        sets = []
+        for b in range(2):
+            if self.kind == "router":
+                lg, idx, w = twin(self.logits, b), twin(self.idx, b), twin(self.w, b)
+                K = self.K
+
+                def run(st, lg=lg, idx=idx, w=w):
+                    ep.router_topk(lg, K, idx, w, st)
+
+                sets.append(([(self.logits_host, lg)], [idx, w], run))
+                continue
+            h, bufs, back = self.h, self.bufs, self.wl["backward"]
+            xd, idxd, wd, out = twin(self.xd, b), twin(self.idxd, b), twin(self.wd, b), twin(self.out, b)
+            ins = [(self.x_host, xd), (self.idx_host, idxd), (self.w_host, wd)]
+            outs = [out]
+            gout = gx = None
+            if back:
+                gout, gx = twin(self.gout, b), twin(self.gx, b)
+                ins.append((self.gout_host, gout))
+                outs.append(gx)
+
+            def run(st, xd=xd, idxd=idxd, wd=wd, out=out, gout=gout, gx=gx):
+                h.plan(idxd, st)
+                h.dispatch(xd, idxd, wd, stream=st, **bufs)
+                h.combine(self.y, wd, out, st)
+                if back:
+                    h.combine_backward(gout, wd, self.gy, st)
+                    h.dispatch_backward(self.gy, gx, st)
+                    h.reduce_replica_grads(self.rep, self.owner, st)
+
+            sets.append((ins, outs, run))
+        return sets
+
     def measure_bytes(self, st):
         """Algorithmic bytes per call, from the routing of one untimed step."""
         self.run(st)
@@ -491,47 +538,44 @@ def run_e2e(step: Step, dev, stream, steps, world, step_bytes):
     host memory and its results (combined tokens, and the input gradient with
     a backward pass) read back to pinned host memory, inside the timed region.
 
-    Steps are pipelined over three streams: the host-to-device copies of step
-    i+1 run while the device-to-host copies of step i drain, since the two
-    PCIe directions are independent. Each step's copies and kernels are
-    ordered by events: a step's inputs are overwritten only after the previous
-    step's kernels have finished with them, and its outputs are written only
-    after the previous step's results have been read back."""
+    Steps are pipelined over three streams (uploads, kernels, read-backs) and
+    two sets of device inputs and outputs, used by alternate steps: step
+    i+1's inputs go up while step i's kernels run and step i-1's results come
+    down, so both directions of the link stay busy. Events order each step: a
+    set's inputs are overwritten only after the kernels of the step that last
+    used them have finished, and its outputs only after that step's results
+    have been read back."""
     import torch
 
-    if step.kind == "path":
-        ins = [(step.x_host, step.xd), (step.idx_host, step.idxd), (step.w_host, step.wd)]
-        if step.wl["backward"]:
-            ins.append((step.gout_host, step.gout))
-    else:
-        ins = step.ins
-    outs = [(o, torch.empty(o.shape, dtype=o.dtype).pin_memory()) for o in step.outputs]
+    sets = step.e2e_sets()
+    host_outs = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in sets[0][1]]
     h2d_st, d2h_st = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    state = {"computed": None, "drained": None}
+    computed, drained = [None, None], [None, None]
+    counter = [0]
 
     def one():
-        # inputs: wait until the previous step's kernels are done reading them
-        if state["computed"] is not None:
-            h2d_st.wait_event(state["computed"])
+        b = counter[0] % 2
+        counter[0] += 1
+        ins, outs, run = sets[b]
+        if computed[b] is not None:  # the kernels that last read this set's inputs
+            h2d_st.wait_event(computed[b])
         with torch.cuda.stream(h2d_st):
             for src, dst in ins:
                 dst.copy_(src, non_blocking=True)
         loaded = torch.cuda.Event()
         loaded.record(h2d_st)
-        # kernels: wait for this step's inputs and for the previous read-back
         stream.wait_event(loaded)
-        if state["drained"] is not None:
-            stream.wait_event(state["drained"])
-        step.run(stream)
-        computed = torch.cuda.Event()
-        computed.record(stream)
-        d2h_st.wait_event(computed)
+        if drained[b] is not None:  # the read-back of this set's last outputs
+            stream.wait_event(drained[b])
+        run(stream)
+        computed[b] = torch.cuda.Event()
+        computed[b].record(stream)
+        d2h_st.wait_event(computed[b])
         with torch.cuda.stream(d2h_st):
-            for src, dst in outs:
+            for src, dst in zip(outs, host_outs):
                 dst.copy_(src, non_blocking=True)
-        drained = torch.cuda.Event()
-        drained.record(d2h_st)
-        state["computed"], state["drained"] = computed, drained
+        drained[b] = torch.cuda.Event()
+        drained[b].record(d2h_st)
 
     for _ in range(2):
         one()
@@ -539,16 +583,18 @@ def run_e2e(step: Step, dev, stream, steps, world, step_bytes):
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record(stream)
     h2d_st.wait_event(s)
-    state["computed"] = state["drained"] = s
+    d2h_st.wait_event(s)
     for _ in range(steps):
         one()
-    stream.wait_event(state["drained"])
+    stream.wait_event(drained[0])
+    stream.wait_event(drained[1])
     e.record(stream)
     torch.cuda.synchronize()
     value, ms = weak_scaling_value(step_bytes, s.elapsed_time(e) / steps, world)
-    h2d = sum(src.numel() * src.element_size() for src, _ in ins)
-    d2h = sum(src.numel() * src.element_size() for src, _ in outs)
-    return {"value": round(value, 2), "unit": "GB/s", "pipelined": True,
+    h2d = sum(src.numel() * src.element_size() for src, _ in sets[0][0])
+    d2h = sum(o.numel() * o.element_size() for o in sets[0][1])
+    del sets
+    return {"value": round(value, 2), "unit": "GB/s", "pipelined": True, "device_buffer_sets": 2,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": steps}
 
 
