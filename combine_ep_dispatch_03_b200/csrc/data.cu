@@ -514,7 +514,7 @@ void pick_shape(int n, int *per_thread, int *threads) {
 // idle while it drains; such rows are cut into parts (whole warps of vectors,
 // at least kSplitMinVectors each) until the grid has about kSplitCtasPerSm
 // CTAs per SM. Large batches keep one CTA per row.
-constexpr int kSplitCtasPerSm = 32, kSplitMinVectors = 128;
+constexpr int kSplitCtasPerSm = 32, kSplitMinVectors = 64;
 
 int row_part(int T, int nvec) {
     const int64_t want = (int64_t)kSplitCtasPerSm * num_sms();

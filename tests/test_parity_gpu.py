@@ -154,7 +154,8 @@ def test_cluster_routing_with_bad_and_repeated_ids(T, E, K, mode, cap):
 def test_rows_split_across_ctas(T, H, fp8):
     """Batches too small for several waves of one-row CTAs cut each row into
     parts of whole warps of vectors, the last part ragged (897 vectors as
-    4 x 256 with 129 left over, 456 FP8 chunks as 256 + 200, 257 vectors)."""
+    7 x 128 and 1 left over, 456 FP8 chunks as 3 x 128 + 72, 257 vectors as
+    96 + 96 + 65)."""
     g = _gc()
     r = g.run_forward(T, H, 32, 4, 4, fp8=fp8, seed=H)
     if not fp8:
