@@ -149,6 +149,17 @@ def test_cluster_routing_with_bad_and_repeated_ids(T, E, K, mode, cap):
     g.run_backward(r, seed=T)
 
 
+@pytest.mark.parametrize("T,K", [(1025, 1), (8192, 1), (8193, 1), (2048, 8), (16385, 1), (32767, 1),
+                                 (4096, 8), (32769, 1)])
+def test_routing_shape_boundaries(T, K):
+    """Batches on either side of each switch of the routing's shape: one CTA
+    up to 1024 pairs; a cluster of 8 CTAs x 16 warps up to 8192; 16 x 16 up
+    to 16384; 16 x 32 up to 32768; three kernels beyond."""
+    g = _gc()
+    r = g.run_forward(T, 128, 64, K, 4, seed=T + K, check_combine=False)
+    assert r["flags"] == 0
+
+
 @pytest.mark.parametrize("T,H,fp8", [(1000, 7176, False), (1000, 7296, True), (300, 2056, False),
                                       (64, 20480, False), (64, 40960, True)])
 def test_rows_split_across_ctas(T, H, fp8):
