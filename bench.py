@@ -37,7 +37,7 @@ FALLBACK_HBM_GBS = 6650.0
 def algorithmic_bytes(T, H, K, rows_placed, fp8):
     """Minimum bytes each call must move (per step), by call."""
     L = T * K
-    plan = 4 * L + 4 * L                                    # topk_idx read, dest_row written
+    plan = 4 * L + 4 * L + 4 * rows_placed                  # topk_idx read; dest_row, src_row written
     payload = rows_placed * H * (1 if fp8 else 2)
     scales = rows_placed * (H // 128) * 4 if fp8 else 0
     dispatch = 2 * T * H + payload + scales + 12 * L + 8 * rows_placed  # x, rows, scales, idx+w+dest, recv_w+recv_expert

@@ -97,6 +97,7 @@ static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 // every array is placed on a 256-byte boundary
 #define EPB_WS_FIELDS(X)                                                                                             \
     X(dest_row, d.L > 0 ? d.L : 1)                                                                                    \
+    X(src_row, d.rows > 0 ? d.rows : 1)                                                                               \
     X(packed, d.L > 0 ? d.L : 1)                                                                                      \
     X(blk, (int64_t)d.E * (d.ntiles > 0 ? d.ntiles : 1))                                                              \
     X(blk_cta, (int64_t)d.E * (d.nhist > 0 ? d.nhist : 1))                                                            \
@@ -162,6 +163,27 @@ ep_status_t ep_recv_rows(const ep_config_t *cfg, int64_t *rows) {
     const ep_status_t s = derive_dims(cfg, &d);
     if (s != EP_OK) return s;
     *rows = d.rows;
+    return EP_OK;
+}
+
+ep_status_t ep_output_shape(const ep_config_t *cfg, int64_t dims[4], int32_t *ndim) {
+    Dims d;
+    if (!dims || !ndim) return EP_ERR_INVALID_ARG;
+    const ep_status_t s = derive_dims(cfg, &d);
+    if (s != EP_OK) return s;
+    if (d.mode == EP_MODE_LL) {
+        *ndim = 4;
+        dims[0] = d.R;
+        dims[1] = d.g;
+        dims[2] = d.cap;
+        dims[3] = d.H;
+    } else {
+        *ndim = 2;
+        dims[0] = d.rows;
+        dims[1] = d.H;
+        dims[2] = 1;
+        dims[3] = 1;
+    }
     return EP_OK;
 }
 
@@ -377,6 +399,7 @@ ep_status_t ep_get_tensor(const ep_handle_t *h, ep_tensor_t which, const void **
     case EP_T_DIRECT_COUNT: *dptr = h->ws.direct_n; *numel = d.direct ? d.R : 0; break;
     case EP_T_DIRECT_EXPERT: *dptr = h->ws.direct_expert; *numel = d.direct ? (int64_t)d.R * d.E : 0; break;
     case EP_T_DIRECT_LEN: *dptr = h->ws.direct_len; *numel = d.direct ? (int64_t)d.R * d.E : 0; break;
+    case EP_T_SRC_ROW: *dptr = h->ws.src_row; *numel = d.rows; break;
     default: return EP_ERR_INVALID_ARG;
     }
     return EP_OK;

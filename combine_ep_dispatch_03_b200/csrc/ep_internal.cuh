@@ -33,6 +33,7 @@ constexpr int kClusterMaxPairs = 32768;  // ... up to this many (token, k) pairs
 // later calls of the same forward/backward pass read.
 struct Workspace {
     int32_t *dest_row;       // [T*K]: receive-buffer row of each pair, -1 if none
+    int32_t *src_row;        // [rows]: pair index of each targeted row (NULL: not kept)
     int32_t *packed;         // [T*K]: expert | rank-in-tile << 16, 0xffff if not routed
     int32_t *blk;            // [ntiles][E]: each tile's base within its CTA's tiles
     int32_t *blk_cta;        // [nhist][E]: per-CTA counts, then bases over CTAs

@@ -179,7 +179,8 @@ __device__ __forceinline__ void warp_count(const int32_t *s_ids, int lo, int hi,
 // warp's first pair of expert e; each pair's index j goes through `look`.
 template <class Lookup>
 __device__ __forceinline__ void warp_assign(const int32_t *s_ids, int lo, int hi, int K, int E, int32_t *my,
-                                            int32_t *__restrict__ dest_row, Lookup look) {
+                                            int32_t *__restrict__ dest_row, int32_t *__restrict__ src_row,
+                                            Lookup look) {
     const int lane = threadIdx.x & 31, bits = id_bits(E);
     uint32_t fl = 0;
     for (int base = lo; base < hi; base += 32) {
@@ -192,6 +193,7 @@ __device__ __forceinline__ void warp_assign(const int32_t *s_ids, int lo, int hi
         if (e >= 0 && (peers & lanemask_lt()) == 0) my[e] += __popc(peers);
         __syncwarp();
         if (p < hi) dest_row[p] = dest;
+        if (dest >= 0 && src_row) src_row[dest] = p;
     }
 }
 
@@ -818,6 +820,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspac
             }
         }
         ws.dest_row[p] = dest;
+        if (dest >= 0 && ws.src_row) ws.src_row[dest] = (int32_t)p;
     }
 }
 
@@ -953,6 +956,7 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
             if (j < s_len[e]) dest = s_off[e] + j;
         }
         ws.dest_row[c0 + i] = dest;
+        if (dest >= 0 && ws.src_row) ws.src_row[dest] = (int32_t)(c0 + i);
     }
 }
 
@@ -998,7 +1002,7 @@ __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__
     __syncthreads();
     const int total = plain_tables(d, s_cnt, s_len, s_base, s_warp, &s_fl);
     plain_outputs(d, ws, s_len, s_base, total);
-    warp_assign(s_ids, lo, hi, K, E, my, ws.dest_row,
+    warp_assign(s_ids, lo, hi, K, E, my, ws.dest_row, ws.src_row,
                 [&](int e, int j) { return j < s_len[e] ? s_base[e] + j : -1; });
     __syncthreads();
     if (threadIdx.x == 0) *ws.flags = s_fl;

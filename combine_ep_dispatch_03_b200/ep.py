@@ -20,7 +20,7 @@ MODE_LL, MODE_HT = 0, 1
 FLAG_BAD_EXPERT_ID, FLAG_DUP_EXPERT_ID, FLAG_CAPACITY, FLAG_PLAN_SLOTS = 0x1, 0x2, 0x4, 0x8
 FLAG_WAIT_TIMEOUT = 0x10  # a bounded wait inside a kernel gave up; that call's outputs are incomplete
 (T_DEST_ROW, T_EXPERT_COUNTS, T_RECV_COUNTS, T_RANK_LOAD, T_RANK_OFFSET, T_REPLICA_EXPERT, T_DIRECT_COUNT,
- T_DIRECT_EXPERT, T_DIRECT_LEN) = range(9)
+ T_DIRECT_EXPERT, T_DIRECT_LEN, T_SRC_ROW) = range(10)
 
 
 class EpConfig(ctypes.Structure):
@@ -52,6 +52,7 @@ _CFG = ctypes.POINTER(EpConfig)
 SIGNATURES = {
     "ep_validate_config": (ctypes.c_int, [_CFG]),
     "ep_recv_rows": (ctypes.c_int, [_CFG, ctypes.POINTER(_I64)]),
+    "ep_output_shape": (ctypes.c_int, [_CFG, ctypes.POINTER(_I64), ctypes.POINTER(ctypes.c_int32)]),
     "ep_recv_counts_len": (ctypes.c_int, [_CFG, ctypes.POINTER(_I64)]),
     "ep_workspace_bytes": (ctypes.c_int, [_CFG, ctypes.POINTER(ctypes.c_size_t)]),
     "ep_plan_kernel_count": (ctypes.c_int, [_CFG, ctypes.POINTER(_I32)]),
@@ -114,6 +115,14 @@ def make_config(T: int, H: int, E: int, K: int, R: int, mode: str = "ht", ll_cap
 
 def validate(cfg: EpConfig) -> int:
     return lib().ep_validate_config(ctypes.byref(cfg))
+
+
+def output_shape(cfg: "EpConfig") -> tuple:
+    """Receive-buffer shape in elements: (rows, H) in HT, (R, E/R, cap, H) in LL."""
+    dims = (_I64 * 4)()
+    nd = ctypes.c_int32()
+    _check("ep_output_shape", lib().ep_output_shape(ctypes.byref(cfg), dims, ctypes.byref(nd)))
+    return tuple(dims[i] for i in range(nd.value))
 
 
 def plan_launches(h: "Ep") -> int:

@@ -85,7 +85,10 @@ typedef enum ep_tensor {
     EP_T_REPLICA_EXPERT = 5, /* int32 [R*S]: expert held by replica slot (r,s), -1 empty */
     EP_T_DIRECT_COUNT = 6,   /* int32 [R]: direct-read pieces of each rank (direct_overflow) */
     EP_T_DIRECT_EXPERT = 7,  /* int32 [R*E]: expert of direct piece i of rank r at [r*E+i], -1 unused */
-    EP_T_DIRECT_LEN = 8      /* int32 [R*E]: rows of that piece */
+    EP_T_DIRECT_LEN = 8,     /* int32 [R*E]: rows of that piece */
+    EP_T_SRC_ROW = 9         /* int32 [rows]: for each receive row that a pair targets, that
+                                pair's index t*K+k (the inverse of EP_T_DEST_ROW); rows no
+                                pair targets hold unspecified values */
 } ep_tensor_t;
 
 /* One EP configuration: fixed for the lifetime of a handle (static shapes,
@@ -124,6 +127,13 @@ ep_status_t ep_recv_rows(const ep_config_t *cfg, int64_t *rows);
  * own experts in id order, then its S replica slots; S = 0 without a
  * balanced plan, giving the per-expert counts [E]), E in LL. */
 ep_status_t ep_recv_counts_len(const ep_config_t *cfg, int64_t *len);
+
+/* Shape of the receive buffer in elements (NCCL EP Table III): HT *ndim = 2,
+ * dims = {rows, H} (rows = T*K, one per (token, k) pair, grouped by expert;
+ * "2D with token counts"); LL *ndim = 4, dims = {R, E/R, ll_capacity, H}
+ * ("3D expert-major"). An FP8 payload has the same shape in bytes, plus
+ * scales [rows, H/128]. dims[i] for i >= *ndim are set to 1. */
+ep_status_t ep_output_shape(const ep_config_t *cfg, int64_t dims[4], int32_t *ndim);
 
 /* Device bytes ep_create will allocate for the handle's workspace. */
 ep_status_t ep_workspace_bytes(const ep_config_t *cfg, size_t *bytes);

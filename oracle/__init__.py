@@ -172,6 +172,16 @@ class Routing:
     recv_counts: np.ndarray  # HT: [E] or [R, g+S] under a plan; LL: [E] rows kept
     plan: dict | None = None
 
+    @property
+    def src_row(self) -> np.ndarray:
+        """[recv_rows]: the pair index t*K+k placed in each receive row, -1 for
+        rows no pair targets. By definition the inverse of dest_row, which is
+        one-to-one on the placed pairs."""
+        src = np.full(self.recv_rows, -1, np.int64)
+        placed = np.nonzero(self.dest_row >= 0)[0]
+        src[self.dest_row[placed]] = placed
+        return src.astype(np.int32)
+
 
 def route(idx, E: int, R: int, mode: str = "ht", cap: int = 0, balanced: bool = False,
           slots: int | None = None, direct: bool = False) -> Routing:

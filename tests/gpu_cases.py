@@ -87,6 +87,8 @@ def run_forward(T, H, E, K, R, mode="ht", cap=0, fp8=False, balanced=False, slot
     np.testing.assert_array_equal(dest, ref.dest_row)
     np.testing.assert_array_equal(h.tensor(ep.T_EXPERT_COUNTS).cpu().numpy(), ref.cnt)
     np.testing.assert_array_equal(bufs["recv_counts"].cpu().numpy(), ref.recv_counts.reshape(-1))
+    placed_rows = np.unique(ref.dest_row[ref.dest_row >= 0])
+    np.testing.assert_array_equal(h.tensor(ep.T_SRC_ROW).cpu().numpy()[placed_rows], ref.src_row[placed_rows])
     if balanced:
         rep, load = h.get_plan()
         np.testing.assert_array_equal(np.array(rep), ref.plan["replica_expert"].reshape(-1))

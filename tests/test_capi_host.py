@@ -87,6 +87,18 @@ def test_recv_rows_and_counts(L):
     assert L.ep_workspace_bytes(ctypes.byref(cfg), ctypes.byref(b)) == 0 and b.value > 0
 
 
+def test_output_shape(L):
+    """HT: one row per (token, k) pair, [T*K, H]; LL: [R, E/R, cap, H]."""
+    from combine_ep_dispatch_03_b200 import ep
+
+    assert ep.output_shape(_cfg()) == (256, 1024)
+    assert ep.output_shape(_cfg(fp8=True)) == (256, 1024)
+    assert ep.output_shape(_cfg(mode="ll", ll_capacity=100)) == (4, 4, 100, 1024)
+    dims, nd = (ctypes.c_int64 * 4)(), ctypes.c_int32()
+    assert L.ep_output_shape(ctypes.byref(_cfg(E=18)), dims, ctypes.byref(nd)) == 1  # E % R != 0
+    assert L.ep_output_shape(ctypes.byref(_cfg()), None, ctypes.byref(nd)) == 1
+
+
 @pytest.mark.parametrize("kw,count", [
     (dict(T=100, E=256, K=8, R=8), 1),            # 800 pairs: one CTA
     (dict(T=32768, E=256, K=8, R=8), 3),          # 262144 pairs: three kernels

@@ -314,6 +314,23 @@ def test_direct_plan_invariants(orc, E, R, S):
         assert sorted(r.dest_row.tolist()) == list(range(L))
 
 
+@pytest.mark.parametrize("mode,cap,balanced", [("ht", 0, False), ("ll", 3, False), ("ht", 0, True)])
+def test_src_row_inverts_dest_row(orc, mode, cap, balanced):
+    """Every placed pair's row maps back to that pair, and no other row holds
+    a pair: checked pair by pair, with LL capacity drops and under a plan."""
+    from combine_ep_dispatch_03_b200 import synth
+
+    idx, _ = synth.routing(300, 16, 4, zipf_s=1.5, seed=7)
+    ref = orc.route(idx, E=16, R=4, mode=mode, cap=cap, balanced=balanced)
+    src = ref.src_row
+    placed = [p for p in range(ref.dest_row.size) if ref.dest_row[p] >= 0]
+    for p in placed:
+        assert src[ref.dest_row[p]] == p
+    assert int((src >= 0).sum()) == len(placed) == len(set(int(ref.dest_row[p]) for p in placed))
+    if mode == "ll":
+        assert len(placed) < ref.dest_row.size  # capacity 3 drops pairs under this skew
+
+
 def test_plan_balances_zipf_routing(orc):
     """Imbalance sweep shape: per-rank load flat across skew under the plan."""
     E, R, K, T = 128, 8, 8, 4096
