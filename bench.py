@@ -30,6 +30,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "dispatch+combine GB/s and tokens/s on 1 B200; % of HBM roofline vs skew"
 FALLBACK_HBM_GBS = 6650.0
+NVLINK_PEER_GBS = 770.0  # measured peer copy per direction per GPU on this B200 type (context only)
 
 
 # ------------------------------------------------------------------ bytes
@@ -615,8 +616,14 @@ def run_sweep(dev, stream, seed, peak, steps=10, warmup=3):
             load = step.h.tensor(ep.T_RANK_LOAD).cpu().tolist()
             mean = sum(load) / len(load)
             gbs = sum(nb.values()) / (ms * 1e-3) / 1e9
+            # What the skew would cost on R real GPUs: the busiest rank receives
+            # max(load) rows and sends as many back, over a peer link of the
+            # measured 770 GB/s per direction.
+            row_bytes = wl["H"] * (1 if wl["fp8"] else 2)
+            modelled_ms = 2 * max(load) * row_bytes / NVLINK_PEER_GBS / 1e6
             rows.append({"zipf_s": s, "balanced": balanced, "ms": round(ms, 4), "gbs": round(gbs, 1),
                          "frac": round(gbs / peak, 4), "load_max_over_mean": round(max(load) / mean, 4),
+                         "modelled_ep_exchange_ms": round(modelled_ms, 3),
                          "plan_us": round(1e3 * sum(per["plan"]) / steps, 2), "flags": step.h.status(stream)})
             step.h.close()
             del step
