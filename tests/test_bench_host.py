@@ -1,0 +1,49 @@
+"""Host-side arithmetic of the benchmark (no GPU): the algorithmic bytes each
+call must move, counted here term by term for a small case, and the guard
+that ties a committed DRAM traffic figure to the source it was measured on."""
+import sys
+
+from conftest import ROOT
+
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_algorithmic_bytes_bf16_by_hand():
+    T, H, K, P = 4, 128, 2, 7  # 8 pairs, 7 of them placed
+    b = bench.algorithmic_bytes(T, H, K, P, fp8=False)
+    L = T * K
+    # plan: ids read (4 B each), dest_row written for every pair, src_row for placed ones
+    assert b["plan"] == 4 * L + 4 * L + 4 * P
+    # dispatch: x read once (bf16), every placed row written once, idx + w + dest read,
+    # recv_w and recv_expert written per placed row
+    assert b["dispatch"] == 2 * T * H + 2 * P * H + 12 * L + 8 * P
+    # combine: every placed expert row read once, out written once, w + dest read
+    assert b["combine"] == 2 * P * H + 2 * T * H + 8 * L
+
+
+def test_algorithmic_bytes_fp8_by_hand():
+    T, H, K, P = 4, 256, 2, 8
+    b = bench.algorithmic_bytes(T, H, K, P, fp8=True)
+    L = T * K
+    # one byte per element and one fp32 scale per 128-element block of each placed row
+    assert b["dispatch"] == 2 * T * H + P * H + P * (H // 128) * 4 + 12 * L + 8 * P
+    assert b["combine"] == 2 * P * H + 2 * T * H + 8 * L
+
+
+def test_ht_prefill_step_bytes_match_the_documented_total():
+    # the HT prefill step with every pair placed: 6.64 GB
+    wl = bench.WORKLOADS["ht_prefill"]
+    T, H, K = wl["T"], wl["H"], wl["K"]
+    b = bench.algorithmic_bytes(T, H, K, T * K, fp8=True)
+    assert abs(sum(b.values()) / 1e9 - 6.645) < 0.002
+
+
+def test_committed_traffic_is_tied_to_its_workload_and_source():
+    assert bench.committed_traffic("k_combine", "not_a_workload") is None
+    assert bench.committed_traffic("no_such_kernel", "ht_prefill") is None
+
+
+def test_weak_scaling_value_single_rank():
+    value, ms = bench.weak_scaling_value(2.0e9, 1.0, 1)
+    assert ms == 1.0 and abs(value - 2000.0) < 1e-9
