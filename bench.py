@@ -20,6 +20,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -56,16 +57,28 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def code_sha(paths) -> str:
+    """sha256[:16] of the C/CUDA code in `paths` (repo-relative), with comments
+    removed and whitespace collapsed: an edit to a comment keeps a committed
+    counter record valid, while any change to the code voids it."""
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel)) as f:
+            s = f.read()
+        s = re.sub(r"/\*.*?\*/", " ", s, flags=re.S)
+        s = re.sub(r"//[^\n]*", "", s)
+        h.update((rel + "\0" + " ".join(s.split()) + "\0").encode())
+    return h.hexdigest()[:16]
+
+
 def committed_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current source of the kernel's file (else None)."""
+    on the current code of the kernel's sources (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f)[kernel]
-        src = os.path.join(ROOT, rec["source"])
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if sha != rec["source_sha"] or rec["workload"] != workload:
+        if code_sha(rec["sources"]) != rec["code_sha"] or rec["workload"] != workload:
             return None
         return int(rec["dram_bytes_per_launch"])
     except Exception:

@@ -2,8 +2,8 @@
 // cast), combine (gather + fp32 weighted reduce), their backward twins, and
 // the replica-gradient reduce.
 //
-// NCCL EP paper (arXiv 2603.13606): dispatch(x, topk_i, topk_w, handle) ->
-// recv_x, recv_i, recv_w (Table V); FP8 quantization scales as a tensor role
+// NCCL EP paper (arXiv 2603.13606): dispatch takes tokens, top-k ids and
+// weights and a handle, and yields received rows, ids and weights (Table V); FP8 quantization scales as a tensor role
 // (Table IV); combine gathers expert outputs and reduces them to the original
 // token order (Table II), per token at the receiver (Table III); the backward
 // pass reuses the forward routing state (Fig. 5). MoonEP article, para. 5:

@@ -9,8 +9,9 @@
  *     expert-major output and HT mode with a 2D concatenated output plus
  *     per-expert token counts (Table III, Figs. 3-4); the tensor roles
  *     TOKENS, TOPK_IDX, TOPK_WEIGHTS and FP8 quantization scales (Table IV);
- *     dispatch(x, topk_i, topk_w, handle) -> recv_x, recv_i, recv_w
- *     (Table V); combine gathers expert outputs and reduces them to the
+ *     a dispatch call that takes the tokens, the top-k ids and weights and
+ *     the handle, and returns the received rows, their expert ids and
+ *     their weights (Table V); combine gathers expert outputs and reduces them to the
  *     original token order (Table II); routing state shared by the forward
  *     and backward passes (Fig. 5).
  *   - MoonEP news article (opensourceforu.com): a GPU planner that

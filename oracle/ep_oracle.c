@@ -252,8 +252,9 @@ int orc_layout_ll(int T, int K, int cap, const int32_t *idx, const int32_t *j, i
  * replica_expert[R*S] (-1 = empty), slot_start[R*S] (first stable index the
  * slot holds), slot_len[R*S], rank_load[R], rank_off[R+1].
  */
-/* Inference variant [MoonEP para 5: "a small fixed number of slots while
- * handling overflow via direct symmetric-memory reads"], reading taken: with
+/* Inference variant [MoonEP para 5: at inference a rank keeps only a few
+ * prefetch slots and rows past them read the owner's weights in place],
+ * reading taken: with
  * `direct` set, step 5 no longer skips a receiver that has a deficit but no
  * free slot; the piece goes to it as a *direct* piece, whose rows are computed
  * with the owner's weights read in place, so every spilled row is placed and

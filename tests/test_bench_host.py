@@ -47,3 +47,23 @@ def test_committed_traffic_is_tied_to_its_workload_and_source():
 def test_weak_scaling_value_single_rank():
     value, ms = bench.weak_scaling_value(2.0e9, 1.0, 1)
     assert ms == 1.0 and abs(value - 2000.0) < 1e-9
+
+
+def test_code_sha_ignores_comments_but_not_code(tmp_path):
+    a = tmp_path / "a.cu"
+    a.write_text("// row mover\n__global__ void k(int* p) { p[0] = 1; /* store */ }\n")
+    base = bench.code_sha([str(a)])
+    a.write_text("/* another\n comment */ __global__ void k(int* p) {\n  p[0] = 1;  // same store\n}\n")
+    assert bench.code_sha([str(a)]) == base
+    a.write_text("__global__ void k(int* p) { p[0] = 2; }\n")
+    assert bench.code_sha([str(a)]) != base
+
+
+def test_committed_traffic_records_name_existing_sources():
+    import json
+    import os
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        recs = json.load(f)
+    for rec in recs.values():
+        assert rec["sources"] and all(os.path.exists(os.path.join(ROOT, s)) for s in rec["sources"])
+        assert len(rec["code_sha"]) == 16 and rec["dram_bytes_per_launch"] > 0
