@@ -363,14 +363,11 @@ ep_status_t ep_get_plan(ep_handle_t *h, int32_t *replica_expert_host, int32_t *r
     if (!h) return EP_ERR_INVALID_ARG;
     if (!h->planned) return EP_ERR_NOT_PLANNED;
     if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return EP_ERR_CUDA;
-    if (replica_expert_host) {
-        if (h->d.S == 0) {
-            for (int r = 0; r < h->d.R; ++r) replica_expert_host[r] = -1;
-        } else if (cudaMemcpy(replica_expert_host, h->ws.replica_expert, sizeof(int32_t) * h->d.R * h->d.S,
-                              cudaMemcpyDeviceToHost) != cudaSuccess) {
-            return EP_ERR_CUDA;
-        }
-    }
+    // without a plan there are no slots (R*S = 0) and nothing is written
+    if (replica_expert_host && h->d.S > 0 &&
+        cudaMemcpy(replica_expert_host, h->ws.replica_expert, sizeof(int32_t) * h->d.R * h->d.S,
+                   cudaMemcpyDeviceToHost) != cudaSuccess)
+        return EP_ERR_CUDA;
     if (rank_load_host &&
         cudaMemcpy(rank_load_host, h->ws.rank_load, sizeof(int32_t) * h->d.R, cudaMemcpyDeviceToHost) != cudaSuccess)
         return EP_ERR_CUDA;

@@ -282,7 +282,10 @@ class Ep:
     def prefetch_replica_weights(self, expert_weights, prefetch_slots, stream=None) -> None:
         """Copy each filled replica slot's expert weights into it: expert_weights
         [E, ...] and prefetch_slots [R, S, ...] of the same row size in bytes."""
-        nbytes = expert_weights.numel() * expert_weights.element_size() // self.E
+        total = expert_weights.numel() * expert_weights.element_size()
+        if total % self.E:
+            raise ValueError("expert_weights must hold E rows of equal size")
+        nbytes = total // self.E
         if prefetch_slots.numel() * prefetch_slots.element_size() != self.R * max(self.S, 1) * nbytes:
             raise ValueError("prefetch_slots must hold R*S rows of one expert's weights")
         _check("ep_prefetch_replica_weights", lib().ep_prefetch_replica_weights(
@@ -290,12 +293,11 @@ class Ep:
 
     # -- inspection
     def get_plan(self, stream=None) -> tuple[list[int], list[int]]:
-        S = max(self.S, 1)
-        rep = (ctypes.c_int32 * (self.R * S))()
+        rep = (ctypes.c_int32 * (self.R * self.S))()
         load = (ctypes.c_int32 * self.R)()
-        _check("ep_get_plan", lib().ep_get_plan(self._h, ctypes.cast(rep, _P), ctypes.cast(load, _P),
-                                                _stream(stream)))
-        return list(rep)[: self.R * self.S], list(load)
+        rep_p = ctypes.cast(rep, _P) if self.S > 0 else None
+        _check("ep_get_plan", lib().ep_get_plan(self._h, rep_p, ctypes.cast(load, _P), _stream(stream)))
+        return list(rep), list(load)
 
     def status(self, stream=None) -> int:
         f = ctypes.c_int32()

@@ -269,7 +269,8 @@ ep_status_t ep_prefetch_replica_weights(ep_handle_t *h, const void *expert_weigh
 /* ---- inspection (these synchronise the stream) ------------------------- */
 
 /* Wait for `stream`, then copy the plan to host memory: replica_expert
- * [R*S] (-1 = empty slot; may be NULL) and rank_load [R] (may be NULL). */
+ * [R*S] (-1 = empty slot; may be NULL; nothing is written when the handle
+ * has no plan, S = 0) and rank_load [R] (may be NULL). */
 ep_status_t ep_get_plan(ep_handle_t *h, int32_t *replica_expert_host, int32_t *rank_load_host, void *stream);
 
 /* Wait for `stream`, then read the device status word (EP_FLAG_* bits set
