@@ -72,6 +72,16 @@ def test_router_topk_ties():
     _check_router(logits.contiguous(), 8)
 
 
+@pytest.mark.parametrize("T,E,K", [(3000, 256, 8), (200, 1024, 32), (500, 40, 5)])
+def test_router_topk_near_ties(T, E, K):
+    """Each token's logits agree in all but their lowest 11 mantissa bits: the
+    choices and their order must follow the full fp32 values."""
+    g = torch.Generator().manual_seed(T + E)
+    base = torch.randn(T, 1, generator=g).expand(T, E).contiguous()
+    low = torch.randint(0, 1 << 11, (T, E), generator=g, dtype=torch.int32)
+    _check_router((base.view(torch.int32) ^ low).view(torch.float32).contiguous(), K)
+
+
 def test_router_feeds_plan_dispatch_combine():
     """Router -> plan -> dispatch -> combine on the GPU equals the oracle chain."""
     import gpu_cases
