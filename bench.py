@@ -5,8 +5,10 @@ One step = one pass of the hot path over one batch: ep_plan (routing
 histogram, scan, layout/plan, stable slots) + ep_dispatch + ep_combine.
 Default workload: HT prefill (T=32768, H=7168, E=256, top-8, R=8 logical ranks,
 FP8 e4m3 dispatch with per-128 scales, bf16 combine with fp32 accumulation),
-seeded synthetic routing. Every buffer is larger than L2 (126 MB), so no L2
-flush is needed between steps.
+seeded synthetic routing. Its step moves 6.6 GB, far more than L2 (126 MB), so
+no L2 flush is needed between its steps; workloads whose step moves at most four
+times the L2 (LL decode, tiny, router) are timed one step at a time, each after
+a write of a buffer twice the L2's size.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 
@@ -386,7 +388,23 @@ class Step:
         return plan_launches(self.h) + len(self.calls) - 1
 
 
-def timed(step: Step, steps, warmup, stream, breakdown_steps=None, graph=True):
+L2_FALLBACK_BYTES = 126 * 2**20
+
+
+def l2_bytes(dev) -> int:
+    import torch
+
+    return int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or L2_FALLBACK_BYTES)
+
+
+def needs_l2_flush(step_bytes: int, l2: int) -> bool:
+    """A step that moves less than four times the L2 could find a good part of
+    its inputs still in L2 from the step before, so such steps are timed one by
+    one, each after a write of a buffer twice the L2's size."""
+    return step_bytes <= 4 * l2
+
+
+def timed(step: Step, steps, warmup, stream, breakdown_steps=None, graph=True, flush=None):
     """Warm-up, then `steps` steps back to back between two CUDA events on the
     launching stream (the step time), then `breakdown_steps` more with an
     event between every two calls (the per-call split; events between calls
@@ -397,8 +415,16 @@ def timed(step: Step, steps, warmup, stream, breakdown_steps=None, graph=True):
     same calls (a graph of up to 10 steps, and one of a single step for the
     remainder): the same kernels with the same programmatic launch edges,
     without the host's per-launch cost, which otherwise bounds steps of a few
-    microseconds."""
+    microseconds.
+
+    With a `flush` buffer (larger than L2), every timed step, and every step
+    of the per-call loop, follows a write of that buffer outside its events:
+    the step is timed alone (a replay of a one-step graph, with `graph`), on
+    cold L2, and the step time is the sum of the steps' own times."""
     import torch
+
+    if flush is not None:
+        return _timed_flushed(step, steps, warmup, stream, breakdown_steps, graph, flush)
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):
@@ -450,6 +476,50 @@ def timed(step: Step, steps, warmup, stream, breakdown_steps=None, graph=True):
     return total, per
 
 
+def _timed_flushed(step: Step, steps, warmup, stream, breakdown_steps, graph, flush):
+    import torch
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step.run(stream)
+    torch.cuda.synchronize()
+    g = None
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step.run(stream)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            g.replay()  # untimed: a graph's first replay may carry one-time set-up
+        torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            flush.fill_(i & 0x7F)
+            ev[i][0].record(stream)
+            if g is not None:
+                g.replay()
+            else:
+                step.run(stream)
+            ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    total = sum(a.elapsed_time(b) for a, b in ev)
+    del g
+    nb = steps if breakdown_steps is None else breakdown_steps
+    n = len(step.calls)
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(nb)]
+    with torch.cuda.stream(stream):
+        for s in range(nb):
+            flush.fill_(s & 0x7F)
+            pev[s][0].record(stream)
+            for i, (_, f) in enumerate(step.calls):
+                f(stream)
+                pev[s][i + 1].record(stream)
+    torch.cuda.synchronize()
+    per = {name: [e[i].elapsed_time(e[i + 1]) for e in pev] for i, (name, _) in enumerate(step.calls)}
+    return total, per
+
+
 def run_native(args):
     import torch
 
@@ -478,11 +548,16 @@ def run_native(args):
     step_bytes = sum(nbytes.values())
     torch.cuda.synchronize()
 
+    l2 = l2_bytes(dev)
+    flush = None
+    if not args.no_flush and needs_l2_flush(step_bytes, l2):
+        flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
     barrier(world)
     torch.cuda.synchronize()
     sampler.start()
-    total_ms, per = timed(step, args.steps, args.warmup, stream, min(args.steps, 50), graph=not args.no_graph)
+    total_ms, per = timed(step, args.steps, args.warmup, stream, min(args.steps, 50), graph=not args.no_graph,
+                          flush=flush)
     clocks = sampler.stop()
     barrier(world)
     value, ms_step = weak_scaling_value(step_bytes, total_ms / args.steps, world)
@@ -499,7 +574,16 @@ def run_native(args):
 
     e2e = None if (args.no_e2e or step.kind == "prefetch") else run_e2e(step, dev, stream, max(3, min(args.steps, 20)),
                                                                         world, step_bytes)
-    big = (step.h.recv_rows * step.H * (1 if wl["fp8"] else 2)) if step.kind == "path" else 4 * wl["T"] * wl["E"]
+    if flush is not None:
+        l2_note = (f"flushed: each step moves {step_bytes / 1e6:.1f} MB, at most 4x L2 ({l2 / 2**20:.0f} MiB), so "
+                   f"a {2 * l2 / 2**20:.0f} MiB buffer is written before every timed step and the steps are "
+                   "timed one by one")
+    elif needs_l2_flush(step_bytes, l2):
+        l2_note = "not flushed (--no-flush): the working set is partly L2-resident"
+    else:
+        l2_note = (f"no flush: each step moves {step_bytes / 1e9:.2f} GB, more than 4x L2 "
+                   f"({l2 / 2**20:.0f} MiB)")
+    del flush
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -510,10 +594,10 @@ def run_native(args):
                    "balanced_plan": wl["balanced"], "zipf_s": wl["s"], "backward": wl["backward"],
                    "payload": ("bf16 x -> fp8 e4m3 dispatch (per-128 fp32 scales)" if wl["fp8"]
                                else "bf16 dispatch") + " -> bf16 combine (fp32 accumulation)",
-                   "l2": ("no flush: the receive buffer (%.2f GB) and the expert rows exceed L2 (126 MB)"
-                          % (big / 1e9)) if big > 2 * 126e6 else "working set partly L2-resident, no flush",
+                   "l2": l2_note,
                    "parallelism": f"{world} independent EP worlds (one per GPU), R logical ranks each",
-                   "launch": "stream" if args.no_graph else "CUDA graph replay of the captured step calls"},
+                   "launch": ("stream" if args.no_graph else "CUDA graph replay of the captured step calls")
+                             + (", one step per timed interval" if l2_note.startswith("flushed") else "")},
         "tokens_per_s": round(world * wl["T"] / (ms_step * 1e-3), 1),
         "rows_per_s": round(world * step.placed / (ms_step * 1e-3), 1),
         "frac_of_hbm": round(step_bytes / (ms_step * 1e-3) / 1e9 / peak, 4),
@@ -737,6 +821,8 @@ def main():
     ap.add_argument("--balanced", type=int, choices=[0, 1], default=None, help="override the balanced plan")
     ap.add_argument("--capacity", type=int, default=0, help="override the LL per-expert capacity (smaller buffers)")
     ap.add_argument("--no-graph", action="store_true", help="time stream launches instead of CUDA-graph replays")
+    ap.add_argument("--no-flush", action="store_true",
+                    help="never flush L2 between timed steps (by default steps moving at most 4x L2 are flushed)")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

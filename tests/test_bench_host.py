@@ -67,3 +67,16 @@ def test_committed_traffic_records_name_existing_sources():
     for rec in recs.values():
         assert rec["sources"] and all(os.path.exists(os.path.join(ROOT, s)) for s in rec["sources"])
         assert len(rec["code_sha"]) == 16 and rec["dram_bytes_per_launch"] > 0
+
+
+def test_l2_flush_decision():
+    l2 = bench.L2_FALLBACK_BYTES
+    # HT prefill moves 6.6 GB a step: far beyond L2, no flush
+    wl = bench.WORKLOADS["ht_prefill"]
+    b = bench.algorithmic_bytes(wl["T"], wl["H"], wl["K"], wl["T"] * wl["K"], fp8=True)
+    assert not bench.needs_l2_flush(sum(b.values()), l2)
+    # LL decode moves about 265 MB (about 2x L2), the router 36 MB: flushed
+    wl = bench.WORKLOADS["ll_decode"]
+    b = bench.algorithmic_bytes(wl["T"], wl["H"], wl["K"], wl["T"] * wl["K"], fp8=False)
+    assert bench.needs_l2_flush(sum(b.values()), l2)
+    assert bench.needs_l2_flush(4 * 32768 * 256 + 8 * 32768 * 8, l2)
