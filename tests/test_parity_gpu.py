@@ -175,12 +175,14 @@ def test_rows_split_across_ctas(T, H, fp8):
 
 def test_long_rows_use_slab_loop():
     """Rows longer than one CTA's registers hold (2050 bf16 vectors, 2056 FP8
-    chunks) in a batch large enough to keep one CTA per row."""
+    chunks) in a batch large enough to keep one CTA per row, and FP8 rows of
+    768 chunks, four a thread (the instance rows of 8193..16384 elements use)."""
     g = _gc()
     T = 40 * torch.cuda.get_device_properties(0).multi_processor_count
     r = g.run_forward(T, 16400, 4, 1, 4, seed=9)
     g.run_backward(r, seed=9)
     g.run_forward(T, 32896, 4, 1, 4, fp8=True, seed=9)
+    g.run_forward(T, 12288, 4, 1, 4, fp8=True, seed=10)
 
 
 # --------------------------------------------------------------- edge cases
