@@ -3,21 +3,24 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "ep_internal.cuh"
 
 namespace epb {
 
 int num_sms() {
-    static int cached[64] = {0};
+    // per device, filled on first use; threads that race to fill it store the same value
+    static std::atomic<int> cached[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
-    if (cached[dev] == 0) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 ep_status_t derive_dims(const ep_config_t *c, Dims *d) {

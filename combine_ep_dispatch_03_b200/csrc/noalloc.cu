@@ -8,6 +8,8 @@
 // outputs point at the caller's buffers.
 #include <string.h>
 
+#include <atomic>
+
 #include "ep_internal.cuh"
 
 namespace epb {
@@ -18,8 +20,9 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[EP_NOALLOC_SCRATCH_BYTES];
 
 // Device address of g_noalloc_scratch per device, looked up once per device
-// with that device current (host code cannot use the symbol itself).
-void *g_scratch_ptr[64] = {nullptr};
+// with that device current (host code cannot use the symbol itself); threads
+// that race to look it up store the same address.
+std::atomic<void *> g_scratch_ptr[64];
 
 size_t al256(size_t n) { return (n + 255) & ~(size_t)255; }
 
@@ -60,13 +63,15 @@ extern "C" ep_status_t ep_route_noalloc(const int32_t *topk_idx, int32_t num_tok
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ERR_CUDA;
-    if (!g_scratch_ptr[dev]) { // set-up: once per device, with that device current
+    void *base = g_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (!base) { // set-up: once per device, with that device current
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
             cudaGetLastError();
             return EP_ERR_CUDA;
         }
-        g_scratch_ptr[dev] = p;
+        g_scratch_ptr[dev].store(p, std::memory_order_release);
+        base = p;
     }
 
     // Every scratch word a kernel reads is written earlier in the same call
@@ -74,7 +79,7 @@ extern "C" ep_status_t ep_route_noalloc(const int32_t *topk_idx, int32_t num_tok
     // assignment kernel), so nothing needs clearing between calls.
     Workspace ws;
     memset(&ws, 0, sizeof ws);
-    char *p = (char *)g_scratch_ptr[dev];
+    char *p = (char *)base;
     auto take = [&p](size_t n) {
         char *q = p;
         p += al256(n);

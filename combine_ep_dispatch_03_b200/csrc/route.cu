@@ -29,6 +29,8 @@
 //                   and then assigns its own pairs
 // Tiny batches without a plan, one kernel:
 //   k_route_small   one CTA does all of the above in shared memory
+#include <atomic>
+
 #include <cooperative_groups.h>
 
 #include "ep_internal.cuh"
@@ -1034,13 +1036,16 @@ size_t route_smem_cluster(const Dims &d) {
 // Can a cluster of d.cl_size CTAs of this kernel be resident at once on this
 // device? (Asked once per device and size.)
 static bool cluster_fits(const Dims &d) {
-    static signed char ok[64][2][2][64]; // [device][size 8/16][16/32 warps][smem in 4 KB steps]: 0 unknown, 1 yes, -1 no
+    // [device][size 8/16][16/32 warps][smem in 4 KB steps]: 0 unknown, 1 yes, -1 no;
+    // threads that race to fill an entry store the same answer
+    static std::atomic<signed char> ok[64][2][2][64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     const size_t smem = route_smem_cluster(d);
     const int si = d.cl_size == 16 ? 1 : 0, wi = d.cl_warps == 32 ? 1 : 0, mi = (int)((smem + 4095) / 4096);
     if (mi >= 64) return false;
-    if (ok[dev][si][wi][mi] == 0) {
+    signed char known = ok[dev][si][wi][mi].load(std::memory_order_relaxed);
+    if (known == 0) {
         cudaFuncSetAttribute(k_route_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxRouteSmem);
         cudaFuncSetAttribute(k_route_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         cudaLaunchConfig_t cfg = {};
@@ -1057,9 +1062,10 @@ static bool cluster_fits(const Dims &d) {
         int n = 0;
         const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, k_route_cluster, &cfg);
         if (e != cudaSuccess) cudaGetLastError();
-        ok[dev][si][wi][mi] = (e == cudaSuccess && n >= 1) ? 1 : -1;
+        known = (e == cudaSuccess && n >= 1) ? 1 : -1;
+        ok[dev][si][wi][mi].store(known, std::memory_order_relaxed);
     }
-    return ok[dev][si][wi][mi] == 1;
+    return known == 1;
 }
 
 bool route_use_cluster(const Dims &d) {
@@ -1071,16 +1077,17 @@ bool route_use_small(const Dims &d) {
 }
 
 cudaError_t launch_plan(const Dims &d, const Workspace &ws, const int32_t *topk_idx, cudaStream_t st) {
-    static bool attrs_set[64] = {false};
+    // per-device function attributes, set once; the flag is published after them
+    static std::atomic<bool> attrs_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attrs_set[dev]) { // per-device function attributes, set once
+    if (dev >= 0 && dev < 64 && !attrs_set[dev].load(std::memory_order_acquire)) {
         const int max_dyn = kMaxRouteSmem;
         cudaFuncSetAttribute(k_route_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
         cudaFuncSetAttribute(k_route_assign, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
         cudaFuncSetAttribute(k_route_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
         cudaFuncSetAttribute(k_route_small, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
-        attrs_set[dev] = true;
+        attrs_set[dev].store(true, std::memory_order_release);
     }
     cudaError_t err;
     if (route_use_cluster(d)) {
