@@ -67,3 +67,11 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["higher_is_better"] is True
+    required = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"}
+    assert required <= set(line)
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert line["metric"] == bench.METRIC and line["unit"] == "GB/s" and line["steps"] == 1
+    assert line["config"]["workload"] == "ht_prefill" and line["e2e"]["value"] == line["value"] > 0
