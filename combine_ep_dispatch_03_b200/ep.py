@@ -133,11 +133,13 @@ def plan_launches(h: "Ep") -> int:
 
 
 def _ptr(t: torch.Tensor | None, dtype: torch.dtype | None = None, numel: int | None = None,
-         name: str = "tensor") -> ctypes.c_void_p | None:
+         name: str = "tensor", device: int | None = None) -> ctypes.c_void_p | None:
     if t is None:
         return None
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device.index != device:
+        raise ValueError(f"{name} is on cuda:{t.device.index}, the handle on cuda:{device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
@@ -196,6 +198,7 @@ class Ep:
         self.mode, self.fp8, self.balanced = mode, fp8, balanced
         self.S = (replica_slots or E // R) if balanced else 0
         self.G = grad_elems_per_expert
+        self.device = torch.cuda.current_device()  # ep_create allocates on the current device
         rows, clen = ctypes.c_int64(), ctypes.c_int64()
         _check("ep_recv_rows", L.ep_recv_rows(ctypes.byref(self.cfg), ctypes.byref(rows)))
         _check("ep_recv_counts_len", L.ep_recv_counts_len(ctypes.byref(self.cfg), ctypes.byref(clen)))
@@ -222,6 +225,10 @@ class Ep:
     def __exit__(self, *exc):
         self.close()
 
+    def _p(self, t, dtype=None, numel=None, name="tensor"):
+        """A tensor's device pointer, checked to be on this handle's device."""
+        return _ptr(t, dtype, numel, name, device=self.device)
+
     # -- output allocation helpers (plumbing)
     def empty_recv(self, device="cuda") -> dict:
         rows, H = self.recv_rows, self.H
@@ -237,7 +244,7 @@ class Ep:
 
     # -- forward
     def plan(self, topk_idx: torch.Tensor, stream=None) -> None:
-        _check("ep_plan", lib().ep_plan(self._h, _ptr(topk_idx, torch.int32, self.T * self.K, "topk_idx"),
+        _check("ep_plan", lib().ep_plan(self._h, self._p(topk_idx, torch.int32, self.T * self.K, "topk_idx"),
                                         _stream(stream)))
 
     def dispatch(self, x, topk_idx, topk_w, recv_x, recv_scales=None, recv_w=None, recv_expert=None,
@@ -246,38 +253,38 @@ class Ep:
         caller's receive buffers (see empty_recv)."""
         rows, H = self.recv_rows, self.H
         _check("ep_dispatch", lib().ep_dispatch(
-            self._h, _ptr(x, torch.bfloat16, self.T * H, "x"),
-            _ptr(topk_idx, torch.int32, self.T * self.K, "topk_idx"),
-            _ptr(topk_w, torch.float32, self.T * self.K, "topk_w"),
-            _ptr(recv_x, torch.float8_e4m3fn if self.fp8 else torch.bfloat16, rows * H, "recv_x"),
-            _ptr(recv_scales, torch.float32, rows * (H // 128), "recv_scales"),
-            _ptr(recv_w, torch.float32, rows, "recv_w"),
-            _ptr(recv_expert, torch.int32, rows, "recv_expert"),
-            _ptr(recv_counts, torch.int32, self.counts_len, "recv_counts"),
+            self._h, self._p(x, torch.bfloat16, self.T * H, "x"),
+            self._p(topk_idx, torch.int32, self.T * self.K, "topk_idx"),
+            self._p(topk_w, torch.float32, self.T * self.K, "topk_w"),
+            self._p(recv_x, torch.float8_e4m3fn if self.fp8 else torch.bfloat16, rows * H, "recv_x"),
+            self._p(recv_scales, torch.float32, rows * (H // 128), "recv_scales"),
+            self._p(recv_w, torch.float32, rows, "recv_w"),
+            self._p(recv_expert, torch.int32, rows, "recv_expert"),
+            self._p(recv_counts, torch.int32, self.counts_len, "recv_counts"),
             _stream(stream)))
 
     def combine(self, expert_out, topk_w, out, stream=None) -> None:
         _check("ep_combine", lib().ep_combine(
-            self._h, _ptr(expert_out, torch.bfloat16, self.recv_rows * self.H, "expert_out"),
-            _ptr(topk_w, torch.float32, self.T * self.K, "topk_w"),
-            _ptr(out, torch.bfloat16, self.T * self.H, "out"), _stream(stream)))
+            self._h, self._p(expert_out, torch.bfloat16, self.recv_rows * self.H, "expert_out"),
+            self._p(topk_w, torch.float32, self.T * self.K, "topk_w"),
+            self._p(out, torch.bfloat16, self.T * self.H, "out"), _stream(stream)))
 
     # -- backward
     def combine_backward(self, grad_out, topk_w, grad_expert_out, stream=None) -> None:
         _check("ep_combine_backward", lib().ep_combine_backward(
-            self._h, _ptr(grad_out, torch.bfloat16, self.T * self.H, "grad_out"),
-            _ptr(topk_w, torch.float32, self.T * self.K, "topk_w"),
-            _ptr(grad_expert_out, torch.bfloat16, self.recv_rows * self.H, "grad_expert_out"), _stream(stream)))
+            self._h, self._p(grad_out, torch.bfloat16, self.T * self.H, "grad_out"),
+            self._p(topk_w, torch.float32, self.T * self.K, "topk_w"),
+            self._p(grad_expert_out, torch.bfloat16, self.recv_rows * self.H, "grad_expert_out"), _stream(stream)))
 
     def dispatch_backward(self, grad_recv, grad_x, stream=None) -> None:
         _check("ep_dispatch_backward", lib().ep_dispatch_backward(
-            self._h, _ptr(grad_recv, torch.bfloat16, self.recv_rows * self.H, "grad_recv"),
-            _ptr(grad_x, torch.bfloat16, self.T * self.H, "grad_x"), _stream(stream)))
+            self._h, self._p(grad_recv, torch.bfloat16, self.recv_rows * self.H, "grad_recv"),
+            self._p(grad_x, torch.bfloat16, self.T * self.H, "grad_x"), _stream(stream)))
 
     def reduce_replica_grads(self, replica_grad, owner_grad, stream=None) -> None:
         _check("ep_reduce_replica_grads", lib().ep_reduce_replica_grads(
-            self._h, _ptr(replica_grad, torch.float32, self.R * max(self.S, 1) * self.G, "replica_grad"),
-            _ptr(owner_grad, torch.float32, self.E * self.G, "owner_grad"), _stream(stream)))
+            self._h, self._p(replica_grad, torch.float32, self.R * max(self.S, 1) * self.G, "replica_grad"),
+            self._p(owner_grad, torch.float32, self.E * self.G, "owner_grad"), _stream(stream)))
 
     def prefetch_replica_weights(self, expert_weights, prefetch_slots, stream=None) -> None:
         """Copy each filled replica slot's expert weights into it: expert_weights
@@ -289,7 +296,7 @@ class Ep:
         if prefetch_slots.numel() * prefetch_slots.element_size() != self.R * max(self.S, 1) * nbytes:
             raise ValueError("prefetch_slots must hold R*S rows of one expert's weights")
         _check("ep_prefetch_replica_weights", lib().ep_prefetch_replica_weights(
-            self._h, _ptr(expert_weights), nbytes, _ptr(prefetch_slots), _stream(stream)))
+            self._h, self._p(expert_weights), nbytes, self._p(prefetch_slots), _stream(stream)))
 
     # -- inspection
     def get_plan(self, stream=None) -> tuple[list[int], list[int]]:

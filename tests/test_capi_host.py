@@ -118,3 +118,37 @@ def test_null_arguments_rejected_without_gpu(L):
     assert L.ep_destroy(None) == 0
     assert L.ep_plan(None, None, None) == 1
     assert L.ep_get_status(None, None, None) == 1
+
+
+class _FakeCudaTensor:
+    """Stands in for a CUDA tensor (no GPU here): only what the binding's
+    pointer marshalling reads."""
+
+    def __init__(self, index):
+        import torch
+
+        self.is_cuda = True
+        self.device = type("D", (), {"index": index})()
+        self.dtype = torch.float32
+
+    def is_contiguous(self):
+        return True
+
+    def numel(self):
+        return 4
+
+    def data_ptr(self):
+        return 4096
+
+
+def test_binding_rejects_a_tensor_on_another_device():
+    import torch
+
+    from combine_ep_dispatch_03_b200 import ep
+
+    with pytest.raises(ValueError, match="cuda:1, the handle on cuda:0"):
+        ep._ptr(_FakeCudaTensor(1), torch.float32, 4, "x", device=0)
+    assert ep._ptr(_FakeCudaTensor(1), torch.float32, 4, "x", device=1).value == 4096
+    assert ep._ptr(_FakeCudaTensor(1), torch.float32, 4, "x").value == 4096  # no handle: no device to match
+    with pytest.raises(ValueError, match="must have 8 elements"):
+        ep._ptr(_FakeCudaTensor(0), torch.float32, 8, "x", device=0)
