@@ -3,9 +3,10 @@
 // the replica-gradient reduce.
 //
 // NCCL EP paper (arXiv 2603.13606): dispatch takes tokens, top-k ids and
-// weights and a handle, and yields received rows, ids and weights (Table V); FP8 quantization scales as a tensor role
-// (Table IV); combine gathers expert outputs and reduces them to the original
-// token order (Table II), per token at the receiver (Table III); the backward
+// weights and a handle, and yields received rows, ids and weights (Table V);
+// FP8 quantization scales as a tensor role (Table IV); combine collects each
+// token's expert results and sums them back into that token's row (Table II),
+// per token at the receiver (Table III); the backward
 // pass reuses the forward routing state (Fig. 5). MoonEP article, para. 5:
 // gradients of duplicated experts pass through a reduce buffer and are added
 // into the owner's gradients.

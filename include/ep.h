@@ -11,9 +11,9 @@
  *     TOKENS, TOPK_IDX, TOPK_WEIGHTS and FP8 quantization scales (Table IV);
  *     a dispatch call that takes the tokens, the top-k ids and weights and
  *     the handle, and returns the received rows, their expert ids and
- *     their weights (Table V); combine gathers expert outputs and reduces them to the
- *     original token order (Table II); routing state shared by the forward
- *     and backward passes (Fig. 5).
+ *     their weights (Table V); combine collects each token's expert results
+ *     and sums them back into that token's row (Table II); routing state
+ *     shared by the forward and backward passes (Fig. 5).
  *   - MoonEP news article (opensourceforu.com): a GPU planner that
  *     replicates hot experts online so that every rank receives a
  *     predictable load (para. 3), placement straight into expert-grouped rank
@@ -192,8 +192,8 @@ ep_status_t ep_router_topk(const float *logits, int32_t num_tokens, int32_t num_
  *            receives floor or ceil of L/R rows (L = routed pairs), hot
  *            experts spilling into at most S replica slots per rank
  *            (MoonEP article paras. 3 and 5). With cfg.direct_overflow (the
- *            inference plan, MoonEP para. 5: a small fixed number of slots,
- *            overflow served by direct reads of the owner's memory), a rank
+ *            inference plan, MoonEP para. 5: only a few slots per rank, and
+ *            rows past them read the owner's weights in place), a rank
  *            with rows to take but no free slot takes them as a direct piece:
  *            its rows are computed with the owner's weights read in place,
  *            and it follows the rank's slots in its region (EP_T_DIRECT_*);
