@@ -696,6 +696,13 @@ def run_e2e(step: Step, dev, stream, steps, world, step_bytes):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": steps}
 
 
+def modelled_exchange_ms(rank_loads, row_bytes: int, link_gbs: float = NVLINK_PEER_GBS) -> float:
+    """What the skew would cost on R real GPUs: the busiest rank receives
+    max(load) rows in dispatch and sends as many back in combine, each over a
+    peer link of `link_gbs` per direction, one phase after the other."""
+    return 2 * max(rank_loads) * row_bytes / link_gbs / 1e6
+
+
 def run_sweep(dev, stream, seed, peak, steps=10, warmup=3):
     """Imbalance sweep: T=32768, H=4096, E=128, top-8, R=8, Zipf s, plan off/on."""
     import torch
@@ -713,11 +720,7 @@ def run_sweep(dev, stream, seed, peak, steps=10, warmup=3):
             load = step.h.tensor(ep.T_RANK_LOAD).cpu().tolist()
             mean = sum(load) / len(load)
             gbs = sum(nb.values()) / (ms * 1e-3) / 1e9
-            # What the skew would cost on R real GPUs: the busiest rank receives
-            # max(load) rows and sends as many back, over a peer link of the
-            # measured 770 GB/s per direction.
-            row_bytes = wl["H"] * (1 if wl["fp8"] else 2)
-            modelled_ms = 2 * max(load) * row_bytes / NVLINK_PEER_GBS / 1e6
+            modelled_ms = modelled_exchange_ms(load, wl["H"] * (1 if wl["fp8"] else 2))
             rows.append({"zipf_s": s, "balanced": balanced, "ms": round(ms, 4), "gbs": round(gbs, 1),
                          "frac": round(gbs / peak, 4), "load_max_over_mean": round(max(load) / mean, 4),
                          "modelled_ep_exchange_ms": round(modelled_ms, 3),

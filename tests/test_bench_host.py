@@ -80,3 +80,30 @@ def test_l2_flush_decision():
     b = bench.algorithmic_bytes(wl["T"], wl["H"], wl["K"], wl["T"] * wl["K"], fp8=False)
     assert bench.needs_l2_flush(sum(b.values()), l2)
     assert bench.needs_l2_flush(4 * 32768 * 256 + 8 * 32768 * 8, l2)
+
+
+def test_modelled_exchange_stays_flat_under_the_balanced_plan():
+    """The sweep's derived column on the oracle's routing at the sweep's full
+    size: with the balanced plan the busiest rank holds ceil(L/R) rows at
+    every skew, so the modelled exchange time does not move; without it, it
+    grows with the skew."""
+    import numpy as np
+
+    import oracle
+    from combine_ep_dispatch_03_b200 import synth
+
+    oracle.build()
+    wl = bench.SWEEP
+    T, H, E, K, R = wl["T"], wl["H"], wl["E"], wl["K"], wl["R"]
+    L = T * K
+    flat, plain = [], []
+    for s in (0.0, 0.5, 1.0, 1.5):
+        idx, _ = synth.routing(T, E, K, zipf_s=s, seed=11)
+        bal = oracle.route(idx, E=E, R=R, balanced=True)
+        assert bal.flags == 0 and max(bal.plan["rank_load"]) == -(-L // R)
+        flat.append(bench.modelled_exchange_ms(bal.plan["rank_load"], 2 * H))
+        loads = oracle.route(idx, E=E, R=R).cnt.reshape(R, E // R).sum(axis=1)
+        plain.append(bench.modelled_exchange_ms(loads, 2 * H))
+    assert flat == [flat[0]] * 4
+    assert abs(flat[0] - 2 * (L // R) * 2 * H / 770e9 * 1e3) < 1e-9
+    assert np.all(np.diff(plain) > 0) and plain[-1] > 5 * flat[0]
