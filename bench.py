@@ -535,6 +535,8 @@ def run_native(args):
     wl = dict(WORKLOADS[args.workload])
     if args.tokens:
         wl["T"] = args.tokens
+    if args.hidden:
+        wl["H"] = args.hidden
     if args.zipf is not None:
         wl["s"] = args.zipf
     if args.balanced is not None:
@@ -820,6 +822,7 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="ht_prefill")
     ap.add_argument("--tokens", type=int, default=0, help="override T (smaller cases for profiling)")
+    ap.add_argument("--hidden", type=int, default=0, help="override H (a multiple of 8; of 128 with FP8)")
     ap.add_argument("--zipf", type=float, default=None, help="override the router's Zipf bias s")
     ap.add_argument("--balanced", type=int, choices=[0, 1], default=None, help="override the balanced plan")
     ap.add_argument("--capacity", type=int, default=0, help="override the LL per-expert capacity (smaller buffers)")
