@@ -152,3 +152,35 @@ def test_binding_rejects_a_tensor_on_another_device():
     assert ep._ptr(_FakeCudaTensor(1), torch.float32, 4, "x").value == 4096  # no handle: no device to match
     with pytest.raises(ValueError, match="must have 8 elements"):
         ep._ptr(_FakeCudaTensor(0), torch.float32, 8, "x", device=0)
+
+
+def test_shape_queries_agree_with_the_oracle_layout(L):
+    """ep_recv_rows / ep_recv_counts_len (host-only) against the receive
+    buffer the oracle lays out, over random HT, LL and planned configs."""
+    import numpy as np
+
+    import oracle
+    from combine_ep_dispatch_03_b200 import ep, synth
+
+    oracle.build()
+    rng = np.random.default_rng(5)
+    for i in range(40):
+        R = int(rng.choice([1, 2, 4, 8]))
+        E = R * int(rng.choice([1, 2, 4, 8]))
+        K = int(rng.integers(1, min(E, 8) + 1))
+        T = int(rng.integers(1, 200))
+        mode = "ll" if i % 3 == 0 else "ht"
+        cap = int(rng.integers(1, T + 1)) if mode == "ll" else 0
+        balanced = mode == "ht" and i % 3 == 1
+        direct = balanced and i % 2 == 0
+        idx, _ = synth.routing(T, E, K, zipf_s=1.0, seed=i)
+        ref = oracle.route(idx, E=E, R=R, mode=mode, cap=cap, balanced=balanced, direct=direct)
+        cfg = ep.make_config(T, 128, E, K, R, mode=mode, ll_capacity=cap, balanced=balanced,
+                             direct_overflow=direct)
+        rows, n = ctypes.c_int64(), ctypes.c_int64()
+        assert L.ep_recv_rows(ctypes.byref(cfg), ctypes.byref(rows)) == 0
+        assert L.ep_recv_counts_len(ctypes.byref(cfg), ctypes.byref(n)) == 0
+        assert rows.value == ref.recv_rows
+        assert n.value == ref.recv_counts.size
+        shape = ep.output_shape(cfg)
+        assert int(np.prod(shape)) == ref.recv_rows * 128
