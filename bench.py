@@ -737,7 +737,7 @@ def cpu_baseline(sample_tokens: int):
     """The oracle as it stands, single-threaded on a host core, on a bounded
     sample of the HT prefill workload: full routing of all 32768 tokens, then
     FP8 dispatch and combine of `sample_tokens` tokens in chunks of 2048. The
-    default is the whole step once, about 10 s on one core of the GPU host."""
+    default is the whole step once: about 10 s on one core of a B200 server."""
     import numpy as np
 
     import oracle
