@@ -67,6 +67,13 @@ MUTANTS = [
      "                q[b * 128 + i] = orc_e4m3_from_f32(orc_bf16_to_f32(x[b * 128 + i]) / s);",
      "            q[b * 128 + i] = orc_e4m3_from_f32(orc_bf16_to_f32(x[b * 128 + i]) / s);",
      [lambda: pins.test_fp8_dequant_error_bound(oracle), lambda: pins.test_fp8_block_golden(oracle)]),
+    ("FP8 cast multiplies by the reciprocal of the scale",
+     "q[b * 128 + i] = orc_e4m3_from_f32(orc_bf16_to_f32(x[b * 128 + i]) / s);",
+     "q[b * 128 + i] = orc_e4m3_from_f32(orc_bf16_to_f32(x[b * 128 + i]) * (1.0f / s));",
+     [lambda: pins.test_fp8_cast_is_the_exactly_rounded_quotient(oracle)]),
+    ("FP8 scale multiplies by a rounded 1/448",
+     "float s = amax / 448.0f;", "float s = amax * (1.0f / 448.0f);",
+     [lambda: pins.test_fp8_cast_is_the_exactly_rounded_quotient(oracle), lambda: pins.test_fp8_block_golden(oracle)]),
     ("replica slot offset counts its own slot",
      "for (int s2 = 0; s2 < s; s2++) off += slot_len[r * S + s2];",
      "for (int s2 = 0; s2 <= s; s2++) off += slot_len[r * S + s2];",

@@ -15,6 +15,7 @@
   dispatch-backward, exact on small-integer data.
 """
 import math
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -360,6 +361,84 @@ def test_fp8_block_golden(orc):
         i, c = tok.split(":")
         expect[int(i)] = int(c, 16)
     np.testing.assert_array_equal(recv[0], expect)
+
+
+# Exact rational arithmetic for the FP8 cast: IEEE binary32 round-to-nearest-
+# even of a real number, and OCP E4M3 round-to-nearest-even with saturation,
+# both from their definitions (normal fp32 range only, which these inputs keep).
+def _exp2_floor(a: Fraction) -> int:
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    return e
+
+
+def _round_half_even(n: Fraction) -> int:
+    fl = n.numerator // n.denominator
+    rest = n - fl
+    if rest > Fraction(1, 2) or (rest == Fraction(1, 2) and fl % 2):
+        fl += 1
+    return fl
+
+
+def _round_f32(q: Fraction) -> Fraction:
+    if q == 0:
+        return q
+    a = abs(q)
+    e = _exp2_floor(a)
+    assert -126 <= e <= 127
+    ulp = Fraction(2) ** (e - 23)
+    return (1 if q > 0 else -1) * _round_half_even(a / ulp) * ulp
+
+
+def _e4m3_code(q: Fraction) -> int:
+    sign = 0x80 if q < 0 else 0
+    a = abs(q)
+    if a == 0:
+        return sign
+    step = Fraction(2) ** (max(_exp2_floor(a), -6) - 3)  # subnormal step 2^-9 below 2^-6
+    v = min(_round_half_even(a / step) * step, Fraction(448))
+    if v == 0:
+        return sign
+    if v < Fraction(1, 64):
+        return sign | int(v * 512)  # subnormal: v = m * 2^-9
+    ev = _exp2_floor(v)
+    return sign | ((ev + 7) << 3) | int((v / Fraction(2) ** ev - 1) * 8)
+
+
+# bf16 bit patterns (amax, x) where RN(x * RN(1/s)) falls on the other side of
+# an e4m3 rounding boundary from RN(x / s), s = RN(amax / 448): a cast that
+# multiplied by the reciprocal would give another code for x.
+_FP8_NEAR_BOUNDARY = [(0x3C27, 0x3427), (0x3CD0, 0x359C), (0x3D52, 0x3516), (0x3EB1, 0x36B1),
+                      (0x3F4D, 0x374D), (0x406B, 0x386B), (0x40FA, 0x38FA), (0x41A3, 0x39A3),
+                      (0x423F, 0x3A3F), (0x4336, 0x3BA9), (0x4384, 0x3B84), (0x447B, 0x3C7B)]
+
+
+def test_fp8_cast_is_the_exactly_rounded_quotient(orc):
+    """Every code of the FP8 cast equals e4m3(RN_f32(x / RN_f32(amax / 448)))
+    worked out in exact rational arithmetic: on inputs next to e4m3 rounding
+    boundaries (where dividing and multiplying by the reciprocal disagree)
+    and on random values in each block."""
+    rng = np.random.default_rng(8)
+    H = 128
+    bits = np.zeros((len(_FP8_NEAR_BOUNDARY), H), np.uint16)
+    for r, (a, x) in enumerate(_FP8_NEAR_BOUNDARY):
+        amax = float(np.array([a << 16], np.uint32).view(np.float32)[0])
+        rand = (rng.uniform(-1.0, 1.0, H) * amax).astype(np.float32)
+        bits[r] = (rand.view(np.uint32) >> 16).astype(np.uint16)  # truncation keeps |v| <= amax
+        bits[r, 0], bits[r, 1], bits[r, 2] = a, x, x | 0x8000
+    xb = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    T = bits.shape[0]
+    recv, scales, _, _ = orc.dispatch(xb, np.zeros((T, 1), np.int32), np.ones((T, 1), np.float32),
+                                      np.arange(T, dtype=np.int32), T, fp8=True)
+    vals = xb.float().numpy()
+    for r in range(T):
+        s = _round_f32(Fraction(float(vals[r, 0])) / 448)
+        assert Fraction(float(scales[r, 0])) == s
+        want = [_e4m3_code(_round_f32(Fraction(float(v)) / s)) for v in vals[r]]
+        assert recv[r].tolist() == want, r
 
 
 def test_fp8_dequant_error_bound(orc):
