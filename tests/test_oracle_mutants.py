@@ -74,6 +74,10 @@ MUTANTS = [
     ("FP8 scale multiplies by a rounded 1/448",
      "float s = amax / 448.0f;", "float s = amax * (1.0f / 448.0f);",
      [lambda: pins.test_fp8_cast_is_the_exactly_rounded_quotient(oracle), lambda: pins.test_fp8_block_golden(oracle)]),
+    ("combine rounds each product before adding it",
+     "acc = fmaf(w[(int64_t)t * K + k], v, acc);", "acc = w[(int64_t)t * K + k] * v + acc;",
+     [lambda: pins.test_combine_is_the_exact_fma_chain(oracle), lambda: pins.test_combine_golden(oracle),
+      lambda: pins.test_affine_expert_and_fp64_error_bound(oracle)]),
     ("replica slot offset counts its own slot",
      "for (int s2 = 0; s2 < s; s2++) off += slot_len[r * S + s2];",
      "for (int s2 = 0; s2 <= s; s2++) off += slot_len[r * S + s2];",

@@ -491,6 +491,45 @@ def test_combine_golden(orc):
     assert (orc.bf16_bits_to_f32(out2) == 1.0).all()
 
 
+def _round_bf16(q: Fraction) -> Fraction:
+    """bfloat16 (8 significant bits) round-to-nearest-even, normal range."""
+    if q == 0:
+        return q
+    a = abs(q)
+    ulp = Fraction(2) ** (_exp2_floor(a) - 7)
+    return (1 if q > 0 else -1) * _round_half_even(a / ulp) * ulp
+
+
+def test_combine_is_the_exact_fma_chain(orc):
+    """out[t] = bf16(acc_K), acc_k = RN_f32(w_k * y_k + acc_{k-1}), acc_0 = +0,
+    worked out in exact rational arithmetic (one rounding per step: a fused
+    multiply-add chain in k order). Checked on every element where such a
+    chain and one that rounds the product first end up on different sides of
+    a bf16 rounding boundary, and on 256 random elements."""
+    rng = np.random.default_rng(3)
+    T, K, H = 64, 8, 4096
+    w = rng.dirichlet(np.ones(K), size=T).astype(np.float32)
+    y = torch.randn(T * K, H, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    out = orc.combine(y, w, np.arange(T * K, dtype=np.int32), T, K)  # choice k of token t reads row t*K+k
+    yv = y.float().numpy().reshape(T, K, H)
+    # where the two chains part ways (fp64 holds each product exactly)
+    fused = np.zeros((T, H), np.float32)
+    split = np.zeros((T, H), np.float32)
+    for k in range(K):
+        fused = (w[:, k:k + 1].astype(np.float64) * yv[:, k] + fused).astype(np.float32)
+        split = (w[:, k:k + 1] * yv[:, k]).astype(np.float32) + split
+    to_bf16 = lambda a: torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy()
+    parted = np.argwhere(to_bf16(fused) != to_bf16(split))
+    assert len(parted) > 0  # the inputs reach the cases this pin exists for
+    picks = [tuple(p) for p in parted] + [(int(rng.integers(T)), int(rng.integers(H))) for _ in range(256)]
+    for t, i in picks:
+        acc = Fraction(0)
+        for k in range(K):
+            acc = _round_f32(Fraction(float(w[t, k])) * Fraction(float(yv[t, k, i])) + acc)
+        got = np.array([np.uint32(out[t, i]) << 16], np.uint32).view(np.float32)[0]
+        assert Fraction(float(got)) == _round_bf16(acc), (t, i)
+
+
 @pytest.mark.parametrize("mode", ["ht", "ll", "balanced"])
 def test_identity_expert_returns_x(orc, mode):
     T, H, E, K, R = 128, 1024, 16, 2, 4
