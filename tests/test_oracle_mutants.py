@@ -78,6 +78,14 @@ MUTANTS = [
      "acc = fmaf(w[(int64_t)t * K + k], v, acc);", "acc = w[(int64_t)t * K + k] * v + acc;",
      [lambda: pins.test_combine_is_the_exact_fma_chain(oracle), lambda: pins.test_combine_golden(oracle),
       lambda: pins.test_affine_expert_and_fp64_error_bound(oracle)]),
+    ("plan spills the coldest expert first",
+     "(cnt[order[b]] < cnt[v] || (cnt[order[b]] == cnt[v] && order[b] > v))",
+     "(cnt[order[b]] > cnt[v] || (cnt[order[b]] == cnt[v] && order[b] > v))",
+     [lambda: pins.test_plan_golden(oracle)]),
+    ("plan visits receivers by ascending deficit",
+     "(D[recv[b]] < D[v] || (D[recv[b]] == D[v] && recv[b] > v))",
+     "(D[recv[b]] > D[v] || (D[recv[b]] == D[v] && recv[b] > v))",
+     [lambda: pins.test_plan_golden(oracle)]),
     ("replica slot offset counts its own slot",
      "for (int s2 = 0; s2 < s; s2++) off += slot_len[r * S + s2];",
      "for (int s2 = 0; s2 <= s; s2++) off += slot_len[r * S + s2];",
