@@ -86,6 +86,10 @@ MUTANTS = [
      "(D[recv[b]] < D[v] || (D[recv[b]] == D[v] && recv[b] > v))",
      "(D[recv[b]] > D[v] || (D[recv[b]] == D[v] && recv[b] > v))",
      [lambda: pins.test_plan_golden(oracle)]),
+    ("router rounds each exponential to float before summing",
+     "ex[k] = exp((double)l[idx[(int64_t)t * K + k]] - lmax);",
+     "ex[k] = (float)exp((double)l[idx[(int64_t)t * K + k]] - lmax);",
+     [lambda: pins.test_router_topk_matches_library_routines(oracle)]),
     ("replica slot offset counts its own slot",
      "for (int s2 = 0; s2 < s; s2++) off += slot_len[r * S + s2];",
      "for (int s2 = 0; s2 <= s; s2++) off += slot_len[r * S + s2];",
