@@ -90,6 +90,22 @@ MUTANTS = [
      "ex[k] = exp((double)l[idx[(int64_t)t * K + k]] - lmax);",
      "ex[k] = (float)exp((double)l[idx[(int64_t)t * K + k]] - lmax);",
      [lambda: pins.test_router_topk_matches_library_routines(oracle)]),
+    ("combine backward uses the next choice's weight",
+     "float wk = w[(int64_t)t * K + k];", "float wk = w[(int64_t)t * K + (k + 1) % K];",
+     [lambda: pins.test_adjoint_identities_exact(oracle, False)]),
+    ("replica reduce adds only the first replica",
+     "for (int a = 0; a < n; a++) acc = acc + rep[(int64_t)list[a] * G + i];",
+     "for (int a = 0; a < (n > 0 ? 1 : 0); a++) acc = acc + rep[(int64_t)list[a] * G + i];",
+     [lambda: pins.test_replica_reduce_sums_exactly(oracle)]),
+    ("replica reduce drops the owner's value",
+     "float acc = owner[(int64_t)e * G + i];", "float acc = 0.0f;",
+     [lambda: pins.test_replica_reduce_sums_exactly(oracle)]),
+    ("dispatch records the token id as the expert",
+     "if (recv_expert) recv_expert[row] = idx[p];", "if (recv_expert) recv_expert[row] = t;",
+     [lambda: pins.test_dispatch_bf16_rows_follow_sorted_pairs(oracle)]),
+    ("dispatch records the first choice's weight for every row",
+     "if (recv_w) recv_w[row] = w[p];", "if (recv_w) recv_w[row] = w[(int64_t)t * K];",
+     [lambda: pins.test_dispatch_bf16_rows_follow_sorted_pairs(oracle)]),
     ("replica slot offset counts its own slot",
      "for (int s2 = 0; s2 < s; s2++) off += slot_len[r * S + s2];",
      "for (int s2 = 0; s2 <= s; s2++) off += slot_len[r * S + s2];",
