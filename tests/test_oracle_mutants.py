@@ -106,6 +106,14 @@ MUTANTS = [
     ("dispatch records the first choice's weight for every row",
      "if (recv_w) recv_w[row] = w[p];", "if (recv_w) recv_w[row] = w[(int64_t)t * K];",
      [lambda: pins.test_dispatch_bf16_rows_follow_sorted_pairs(oracle)]),
+    ("e4m3 saturates to NaN instead of 448",
+     "if (a > 448.0) return (uint8_t)(sign | 0x7e);", "if (a > 448.0) return (uint8_t)(sign | 0x7f);",
+     [lambda: pins.test_e4m3_golden_table(oracle),
+      lambda: pins.test_e4m3_matches_torch_in_range_all_bf16_times_scales(oracle)]),
+    ("e4m3 loses the sign of a negative zero",
+     "uint8_t sign = signbit(v) ? 0x80 : 0x00;", "uint8_t sign = (v < 0.0f) ? 0x80 : 0x00;",
+     [lambda: pins.test_e4m3_golden_table(oracle),
+      lambda: pins.test_e4m3_matches_torch_in_range_all_bf16_times_scales(oracle)]),
     ("replica slot offset counts its own slot",
      "for (int s2 = 0; s2 < s; s2++) off += slot_len[r * S + s2];",
      "for (int s2 = 0; s2 <= s; s2++) off += slot_len[r * S + s2];",
