@@ -114,6 +114,18 @@ MUTANTS = [
      "uint8_t sign = signbit(v) ? 0x80 : 0x00;", "uint8_t sign = (v < 0.0f) ? 0x80 : 0x00;",
      [lambda: pins.test_e4m3_golden_table(oracle),
       lambda: pins.test_e4m3_matches_torch_in_range_all_bf16_times_scales(oracle)]),
+    ("owner's tail placed before its kept rows",
+     "dest_row[p] = (int32_t)(rank_off[owner] + own_off + keep[e] + (j[p] - tail_start[e]));",
+     "dest_row[p] = (int32_t)(rank_off[owner] + own_off + (j[p] - tail_start[e]));",
+     [lambda: pins.test_plan_golden(oracle)]),
+    ("later own experts ignore an earlier expert's tail",
+     "for (int e2 = owner * g; e2 < e; e2++) own_off += keep[e2] + tail_len[e2];",
+     "for (int e2 = owner * g; e2 < e; e2++) own_off += keep[e2];",
+     [lambda: pins.test_plan_golden(oracle)]),
+    ("direct pieces ignore earlier direct pieces",
+     "for (int i2 = 0; i2 < i; i2++) off += direct_len[r * E + i2];",
+     "for (int i2 = 0; i2 < 0; i2++) off += direct_len[r * E + i2];",
+     [lambda: pins.test_direct_plan_invariants(oracle, 16, 4, 1)]),
     ("replica slot offset counts its own slot",
      "for (int s2 = 0; s2 < s; s2++) off += slot_len[r * S + s2];",
      "for (int s2 = 0; s2 <= s; s2++) off += slot_len[r * S + s2];",

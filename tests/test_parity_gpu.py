@@ -234,6 +234,26 @@ def test_ll_capacity_overflow_drops_and_flags():
     g.run_backward(r, seed=4)
 
 
+def test_hand_worked_plans():
+    """The hand-worked balanced plans of tests/golden/plan_worked.txt (a normal
+    case, slot overflow with and without a tail between kept rows, the
+    inference plan, and a case decided by the spill and receiver orders) run
+    on the GPU: loads and replica table equal to the worked values, routing,
+    rows and combine equal to the oracle."""
+    from test_oracle_pins import _golden_plans, _idx_from_counts
+
+    g = _gc()
+    for n, c in enumerate(_golden_plans()):
+        E, R, S = c["E"][0], c["R"][0], c["S"][0]
+        idx = torch.from_numpy(_idx_from_counts(c["cnt"]))
+        T = idx.shape[0]
+        r = g.run_forward(T, 128, E, 1, R, balanced=True, slots=S, direct=bool(c.get("direct", [0])[0]),
+                          idx=idx, w=torch.ones((T, 1), dtype=torch.float32), seed=40 + n)
+        rep, load = r["h"].get_plan()
+        assert rep == c["replica_expert"] and load == c["rank_load"]
+        assert r["flags"] == c["flags"][0]
+
+
 def test_balanced_plan_slot_overflow_keeps_rows_on_owner():
     """Replica slots limited to 1 per rank under heavy skew: the plan runs out
     of slots, raises PLAN_SLOTS and keeps the leftover rows on the owner; the
