@@ -18,7 +18,9 @@ import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ep_oracle.c")
 
-# name, text to replace (must occur once), replacement, pins that must catch it
+# name, text to replace (must occur once), replacement, pins that must catch it;
+# a mistake that needs several edits gives a list of (text, replacement) pairs
+# and None for the replacement
 MUTANTS = [
     ("combine drops the first choice",
      "            for (int k = 0; k < K; k++) {\n                int32_t row = dest_row[(int64_t)t * K + k];\n"
@@ -134,6 +136,36 @@ MUTANTS = [
      "                for (int s2 = 0; s2 < S; s2++) off += slot_len[r * S + s2];\n                for (int i2 = 0;",
      "                for (int s2 = 0; s2 < 0; s2++) off += slot_len[r * S + s2];\n                for (int i2 = 0;",
      [lambda: pins.test_plan_golden(oracle), lambda: pins.test_direct_plan_invariants(oracle, 16, 4, 1)]),
+    ("dispatch-backward sum taken in reverse order",
+     "            for (int k = 0; k < K; k++) {\n                int32_t row = dest_row[(int64_t)t * K + k];\n"
+     "                if (row < 0) continue;\n                float v",
+     "            for (int k0 = 0; k0 < K; k0++) {\n                int k = w ? k0 : K - 1 - k0;\n"
+     "                int32_t row = dest_row[(int64_t)t * K + k];\n                if (row < 0) continue;\n"
+     "                float v",
+     [lambda: pins.test_dispatch_backward_is_the_exact_sum_chain(oracle)]),
+    ("dispatch-backward sum taken as a pairwise tree",
+     [("            float acc = 0.0f;", "            float acc = 0.0f, buf[32] = {0};"),
+      ("                else\n                    acc = acc + v;", "                else\n                    buf[k] = v;"),
+      ("            out[(int64_t)t * H + i] = orc_bf16_from_f32(acc);",
+       "            for (int n = K, m; !w && n > 1; n = m) {\n                m = (n + 1) / 2;\n"
+       "                for (int a = 0; a < n / 2; a++) buf[a] = buf[2 * a] + buf[2 * a + 1];\n"
+       "                if (n & 1) buf[m - 1] = buf[n - 1];\n            }\n"
+       "            if (!w) acc = acc + buf[0];\n"
+       "            out[(int64_t)t * H + i] = orc_bf16_from_f32(acc);")],
+     None,
+     [lambda: pins.test_dispatch_backward_is_the_exact_sum_chain(oracle)]),
+    ("dispatch-backward sum kept in bf16 between adds",
+     "acc = acc + v;", "acc = orc_bf16_to_f32(orc_bf16_from_f32(acc + v));",
+     [lambda: pins.test_dispatch_backward_is_the_exact_sum_chain(oracle)]),
+    ("combine backward rounds the exact product straight to bf16",
+     "                float prod = wk * orc_bf16_to_f32(g[(int64_t)t * H + i]);",
+     "                int ex2;\n"
+     "                double m2 = frexp((double)wk * (double)orc_bf16_to_f32(g[(int64_t)t * H + i]), &ex2);\n"
+     "                float prod = (float)ldexp(nearbyint(m2 * 256.0) / 256.0, ex2);",
+     [lambda: pins.test_combine_backward_is_one_fp32_product_then_bf16(oracle)]),
+    ("combine backward multiplies in bf16",
+     "float prod = wk * orc_bf16_to_f32(", "float prod = orc_bf16_to_f32(orc_bf16_from_f32(wk)) * orc_bf16_to_f32(",
+     [lambda: pins.test_combine_backward_is_one_fp32_product_then_bf16(oracle)]),
 ]
 
 
@@ -143,9 +175,14 @@ def mutant_lib(tmp_path):
     src = open(SRC).read()
 
     def load(find, repl):
-        assert src.count(find) == 1, f"mutation anchor not unique: {find!r}"
+        # one (anchor, replacement) pair, or a list of pairs applied in turn
+        edits = find if isinstance(find, list) else [(find, repl)]
+        text = src
+        for a, b in edits:
+            assert text.count(a) == 1, f"mutation anchor not unique: {a!r}"
+            text = text.replace(a, b)
         path = tmp_path / "mutant.c"
-        path.write_text(src.replace(find, repl))
+        path.write_text(text)
         so = oracle.compile_to(str(path), str(tmp_path / "libmutant.so"))
         oracle._lib = oracle.configure(ctypes.CDLL(so))
 

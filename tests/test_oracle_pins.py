@@ -592,6 +592,139 @@ def test_adjoint_identities_exact(orc, balanced):
     assert lhs2 == rhs2
 
 
+def _bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float32 array -> bf16 bit patterns, by torch's round-to-nearest-even."""
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).view(torch.int16).numpy()
+
+
+def _wide_range_sums(rng, T: int, K: int, H: int) -> np.ndarray:
+    """Expert-output rows [T*K, H] (float32 values of bf16 numbers) whose K
+    terms per element are far apart in magnitude, so that the fp32 sum rounds
+    and its order shows. First half of the tokens: per element one term
+    b in [1, 2)*2^e, one term of half a bf16 step of b (the sum of the two
+    sits on a bf16 rounding tie), and K-2 terms below half an fp32 step of b,
+    in a random order; second half: random bf16 values with exponents in
+    [-12, 12]."""
+    y = np.zeros((T, K, H), np.float32)
+    h = T // 2
+    e = rng.integers(-4, 5, size=(h, 1, H)).astype(np.float64)
+    big = (1.0 + rng.integers(0, 128, size=(h, 1, H)) / 128.0) * 2.0 ** e
+    half = rng.choice([-1.0, 1.0], size=(h, 1, H)) * 2.0 ** (e - 8)
+    tiny = (rng.choice([-1.0, 1.0], size=(h, K - 2, H)) * (1.0 + rng.integers(0, 128, size=(h, K - 2, H)) / 128.0)
+            * 2.0 ** (e - rng.integers(21, 28, size=(h, K - 2, H))))
+    terms = np.concatenate([big, half, tiny], axis=1)
+    perm = np.argsort(rng.random((h, K, H)), axis=1)
+    y[:h] = np.take_along_axis(terms, perm, axis=1)
+    y[h:] = (rng.choice([-1.0, 1.0], size=(T - h, K, H)) * (1.0 + rng.integers(0, 128, size=(T - h, K, H)) / 128.0)
+             * 2.0 ** rng.integers(-12, 13, size=(T - h, K, H)))
+    return y.reshape(T * K, H)
+
+
+def test_dispatch_backward_is_the_exact_sum_chain(orc):
+    """grad_x[t] = bf16(acc_K), acc_k = RN_f32(acc_{k-1} + y_k) in k order
+    from acc_0 = +0, unrouted pairs skipped (the dispatch-gradient combine of
+    the NCCL EP page's Fig. 5: one fp32 add per routed row, one rounding to
+    bf16), worked out in exact rational arithmetic. Checked on every element
+    (up to 1500 of each kind) where that chain and a reverse-order sum, a
+    pairwise sum or a bf16 running sum land on different bf16 values, and on
+    256 random elements."""
+    rng = np.random.default_rng(21)
+    T, K, H = 64, 8, 1024
+    yv = _wide_range_sums(rng, T, K, H)
+    dest = np.arange(T * K, dtype=np.int32)
+    dest[rng.random(T * K) < 0.05] = -1  # a few unrouted pairs
+    y = torch.from_numpy(yv).to(torch.bfloat16)
+    assert (y.float().numpy() == yv).all()  # the terms are bf16 numbers
+    out = orc.combine(y, None, dest, T, K)
+    terms = np.where((dest >= 0)[:, None], yv, 0.0).astype(np.float32).reshape(T, K, H)
+    fwd = np.zeros((T, H), np.float32)
+    rev = np.zeros((T, H), np.float32)
+    run16 = np.zeros((T, H), np.float32)
+    for k in range(K):
+        fwd = fwd + terms[:, k]
+        rev = rev + terms[:, K - 1 - k]
+        run16 = torch.from_numpy(run16 + terms[:, k]).to(torch.bfloat16).float().numpy()
+    level = [terms[:, k] for k in range(K)]
+    while len(level) > 1:
+        level = [level[i] + level[i + 1] if i + 1 < len(level) else level[i] for i in range(0, len(level), 2)]
+    want = _bf16_bits(fwd)
+    picks = set()
+    for alt in (rev, level[0], run16):
+        parted = np.argwhere(_bf16_bits(alt) != want)
+        assert len(parted) > 0  # each alternative is reached by these inputs
+        for p in rng.permutation(len(parted))[:1500]:
+            picks.add(tuple(parted[p]))
+    picks |= {(int(rng.integers(T)), int(rng.integers(H))) for _ in range(256)}
+    for t, i in sorted(picks):
+        acc = Fraction(0)
+        for k in range(K):
+            if dest[t * K + k] >= 0:
+                acc = _round_f32(acc + Fraction(float(yv[t * K + k, i])))
+        got = np.array([np.uint32(out[t, i]) << 16], np.uint32).view(np.float32)[0]
+        assert Fraction(float(got)) == _round_bf16(acc), (t, i)
+
+
+def _rn_bf16_of_f64(a: np.ndarray) -> np.ndarray:
+    """Normal float64 values -> nearest bf16 value (ties to even), in one
+    rounding from the float64 value, as float64."""
+    u = np.ascontiguousarray(a, np.float64).view(np.uint64)
+    low = u & np.uint64((1 << 45) - 1)
+    up = u >> np.uint64(45)
+    half = np.uint64(1 << 44)
+    up = up + ((low > half) | ((low == half) & ((up & np.uint64(1)) == 1))).astype(np.uint64)
+    return (up << np.uint64(45)).view(np.float64)
+
+
+def test_combine_backward_is_one_fp32_product_then_bf16(orc):
+    """grad_y[dest_row[t,k]] = bf16(RN_f32(w[t,k] * g[t])): the product is
+    rounded to fp32 once, then to bf16 once (the combine gradient of the NCCL
+    EP page's Fig. 5), worked out in exact rational arithmetic. The inputs
+    include products whose fp32 rounding lands exactly on a bf16 tie while the
+    exact product does not (found by search), so rounding the exact product
+    straight to bf16 gives another value there; a bf16 multiply (w rounded to
+    bf16 first) parts elsewhere. Checked on every element where either
+    alternative differs, and on 256 random ones."""
+    rng = np.random.default_rng(22)
+    K, H = 8, 1024
+    # products w * g whose fp32 rounding is a bf16 tie but which are not exact
+    gv = (1.0 + np.arange(128) / 128.0)[None, :] * 2.0 ** np.arange(-30, 31)[:, None]
+    gv = gv.reshape(-1)
+    hits = []
+    for _ in range(1200):
+        wv = np.float32(rng.uniform(0.001, 1.0))
+        p = np.float64(wv) * gv  # exact: 24 x 8 significant bits
+        f = p.astype(np.float32)
+        tie = ((f.view(np.uint32) & 0xFFFF) == 0x8000) & (f.astype(np.float64) != p)
+        hits += [(wv, gv[j]) for j in np.nonzero(tie)[0]]
+    assert len(hits) >= 40
+    T0 = 64
+    T = T0 + len(hits)
+    w = rng.dirichlet(np.ones(K), size=T).astype(np.float32)
+    g = torch.randn(T, H, generator=torch.Generator().manual_seed(23)).to(torch.bfloat16).float().numpy()
+    for n, (wv, gval) in enumerate(hits):
+        w[T0 + n, n % K] = wv
+        g[T0 + n, (7 * n) % H] = gval * rng.choice([-1.0, 1.0])
+    gb = torch.from_numpy(g).to(torch.bfloat16)
+    assert (gb.float().numpy() == g).all()
+    gy = orc.combine_backward(gb, w, np.arange(T * K, dtype=np.int32), T * K).reshape(T, K, H)
+    prod = w.astype(np.float64)[:, :, None] * g.astype(np.float64)[:, None, :]  # exact
+    want = _bf16_bits(prod.astype(np.float32))
+    direct = _bf16_bits(_rn_bf16_of_f64(prod).astype(np.float32))  # exact in fp32: 8 bits
+    w16 = torch.from_numpy(w).to(torch.bfloat16).float().numpy().astype(np.float64)
+    mul16 = _bf16_bits((w16[:, :, None] * g[:, None, :]).astype(np.float32))  # 8 x 8 bits: exact in fp32
+    picks = set()
+    for alt in (direct, mul16):
+        parted = np.argwhere(alt != want)
+        assert len(parted) > 0
+        for p in rng.permutation(len(parted))[:1500]:
+            picks.add(tuple(parted[p]))
+    picks |= {(int(rng.integers(T)), int(rng.integers(K)), int(rng.integers(H))) for _ in range(256)}
+    for t, k, i in sorted(picks):
+        exact = _round_bf16(_round_f32(Fraction(float(w[t, k])) * Fraction(float(g[t, i]))))
+        got = np.array([np.uint32(gy[t, k, i]) << 16], np.uint32).view(np.float32)[0]
+        assert Fraction(float(got)) == exact, (t, k, i)
+
+
 # ------------------------------------------------------------------ replica reduce
 
 def test_replica_reduce_sums_exactly(orc):
