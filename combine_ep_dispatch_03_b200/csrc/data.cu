@@ -142,7 +142,12 @@ __global__ void __launch_bounds__(32) k_dispatch_bulk(const uint8_t *__restrict_
         if (off > 0) bulk_load(s_row, src + off, (uint32_t)len, &s_bar);
         if (!mbar_wait(&s_bar, parity)) {
             atomicOr(status, EP_FLAG_WAIT_TIMEOUT);
-            mbar_wait(&s_bar, parity); // the load in flight still writes s_row
+            // The load in flight still writes s_row: stay resident (bounded,
+            // up to 8 more waits of 2 s) so that its bytes cannot land in the
+            // shared memory of a CTA that takes this one's place. Past that
+            // the flag stands for the whole launch.
+            for (int r = 0; r < 8 && !mbar_wait(&s_bar, parity); ++r) {
+            }
             return;
         }
         const uint64_t pol = policy_evict_first();

@@ -26,6 +26,10 @@ std::atomic<void *> g_scratch_ptr[64];
 
 size_t al256(size_t n) { return (n + 255) & ~(size_t)255; }
 
+// every int32 argument must be 4-byte aligned; a misaligned one is refused
+// before anything is launched
+bool aligned4(const void *p) { return ((uintptr_t)p & 3u) == 0; }
+
 // Bytes of scratch the routing kernels need for these sizes (plain HT layout,
 // one logical rank).
 size_t scratch_need(const Dims &d) {
@@ -57,8 +61,8 @@ extern "C" ep_status_t ep_route_noalloc(const int32_t *topk_idx, int32_t num_tok
     Dims d;
     ep_status_t s = derive_dims(&cfg, &d);
     if (s != EP_OK) return s;
-    if (!expert_counts || !flags) return EP_ERR_INVALID_ARG;
-    if (d.L > 0 && (!topk_idx || !dest_row)) return EP_ERR_INVALID_ARG;
+    if (!expert_counts || !flags || !aligned4(expert_counts) || !aligned4(flags)) return EP_ERR_INVALID_ARG;
+    if (d.L > 0 && (!topk_idx || !dest_row || !aligned4(topk_idx) || !aligned4(dest_row))) return EP_ERR_INVALID_ARG;
     if (scratch_need(d) > (size_t)EP_NOALLOC_SCRATCH_BYTES) return EP_ERR_TOO_LARGE;
 
     int dev = 0;

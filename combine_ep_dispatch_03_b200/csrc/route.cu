@@ -664,6 +664,9 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const int32_t *__r
     // each tile's base among this CTA's tiles, and the CTA's totals
     const int tile0 = blockIdx.x * kRouteWarps;
     const int ntile = min(kRouteWarps, d.ntiles - tile0);
+    // the scan kernel's ticket starts every plan at 0, whatever an earlier
+    // launch left there (the scan waits for this grid to complete)
+    if (d.balanced && blockIdx.x == 0 && threadIdx.x == 0) *ws.ticket = 0ull;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
         for (int ww = 0; ww < ntile; ++ww) {
@@ -728,7 +731,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_route_scan(Dims d, Workspace w
     if (tid == 0) {
         __threadfence();
         const unsigned long long t = atomicAdd(ws.ticket, 1ull);
-        s_last = ((t + 1) % gridDim.x) == 0; // every launch draws exactly gridDim.x tickets
+        s_last = t + 1 == gridDim.x; // the histogram kernel reset the counter to 0
         s_fl = 0;
     }
     __syncthreads();

@@ -120,6 +120,23 @@ def test_null_arguments_rejected_without_gpu(L):
     assert L.ep_get_status(None, None, None) == 1
 
 
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="host-only check: needs no GPU")
+def test_noalloc_refuses_misaligned_pointers_before_any_launch(L):
+    """ep_route_noalloc checks every int32 pointer for 4-byte alignment and
+    returns EP_ERR_INVALID_ARG (1) before it touches the device: here there is
+    no GPU, so a call that got past the checks would report EP_ERR_CUDA (2)
+    instead. The addresses are never dereferenced."""
+    ok, odd = ctypes.c_void_p(4096), ctypes.c_void_p(4098)
+    T, K, E = 64, 2, 16
+    for i in range(4):
+        args = [ok, ok, ok, ok]
+        args[i] = odd
+        idx, dest, cnt, fl = args
+        assert L.ep_route_noalloc(idx, T, K, E, dest, cnt, fl, None) == 1, i
+    # the same call with aligned pointers gets as far as the device lookup
+    assert L.ep_route_noalloc(ok, T, K, E, ok, ok, ok, None) == 2
+
+
 class _FakeCudaTensor:
     """Stands in for a CUDA tensor (no GPU here): only what the binding's
     pointer marshalling reads."""
