@@ -49,6 +49,33 @@ def algorithmic_bytes(T, H, K, rows_placed, fp8):
     return {"plan": plan, "dispatch": dispatch, "combine": combine}
 
 
+def compute_dtype(wl: dict) -> str:
+    """What the path computes in: bf16 rows (e4m3 codes with fp32 scales when
+    the dispatch casts), fp32 accumulation in combine and the backward."""
+    return "bf16+e4m3 (fp32 accumulate)" if wl["fp8"] else "bf16 (fp32 accumulate)"
+
+
+def workload_config(name: str, wl: dict, world: int, l2_note: str) -> dict:
+    """The `config` object of the JSON line; both arms print the same one."""
+    return {"workload": name, "T": wl["T"], "H": wl["H"], "E": wl["E"], "topk": wl["K"],
+            "logical_ranks": wl["R"], "layout": wl["mode"], "ll_capacity": wl["cap"],
+            "balanced_plan": wl["balanced"], "zipf_s": wl["s"], "backward": wl["backward"],
+            "payload": ("bf16 x -> fp8 e4m3 dispatch (per-128 fp32 scales)" if wl["fp8"]
+                        else "bf16 dispatch") + " -> bf16 combine (fp32 accumulation)",
+            "l2": l2_note,
+            "parallelism": f"{world} independent EP worlds (one per GPU), R logical ranks each"}
+
+
+def l2_note_for(step_bytes: int, l2: int, flushed: bool) -> str:
+    if flushed:
+        return (f"flushed: each step moves {step_bytes / 1e6:.1f} MB, at most 4x L2 ({l2 / 2**20:.0f} MiB), so "
+                f"a {2 * l2 / 2**20:.0f} MiB buffer is written before every timed step and the steps are "
+                "timed one by one")
+    if needs_l2_flush(step_bytes, l2):
+        return "not flushed (--no-flush): the working set is partly L2-resident"
+    return f"no flush: each step moves {step_bytes / 1e9:.2f} GB, more than 4x L2 ({l2 / 2**20:.0f} MiB)"
+
+
 def hbm_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -90,13 +117,19 @@ def committed_traffic(kernel: str, workload: str):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling SM clocks and throttle reasons every 20 ms, with a
+    timestamp on each sample. stop() summarises every sample; window() those
+    taken within a host-time interval (a timed region shorter than the sampling
+    period is given the samples of the surrounding interval it names)."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.samples = []  # (host epoch seconds, sm MHz, max MHz, set of reasons)
 
     def start(self):
         try:
@@ -105,6 +138,29 @@ class ClockSampler:
                  "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+
+    def _parse(self, out: str):
+        import datetime
+
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, smax = float(parts[2]), float(parts[3])
+            except ValueError:
+                continue
+            reasons = {n for n, v in zip(self.REASONS, parts[6:10]) if v.lower() == "active"}
+            self.samples.append((ts, sm, smax, reasons))
+
+    @staticmethod
+    def _summary(samples):
+        if not samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = set().union(*(r for _, _, _, r in samples))
+        return {"sm_mhz": statistics.median(s for _, s, _, _ in samples), "sm_max_mhz": samples[-1][2],
+                "reasons": sorted(reasons), "samples": len(samples)}
 
     def stop(self):
         if self.proc is None:
@@ -115,22 +171,22 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        self._parse(out)
+        self.proc = None
+        return self._summary(self.samples)
+
+    def window(self, t0: float, t1: float, margin: float = 0.1):
+        """Samples taken from t0 - margin to t1 + margin (host epoch seconds),
+        widened step by step to at least 5 samples where the region is short."""
+        sel = []
+        while margin <= 1.6:
+            sel = [x for x in self.samples if t0 - margin <= x[0] <= t1 + margin]
+            if len(sel) >= 5:
+                break
+            margin *= 2
+        rec = self._summary(sel)
+        rec["window_s"] = round(t1 - t0 + 2 * min(margin, 1.6), 3)
+        return rec
 
 
 # ------------------------------------------------------------------ distributed
@@ -202,7 +258,16 @@ WORKLOADS = {
                    backward=False, G=0, kind="router"),
     "prefetch": dict(T=131072, H=7168, E=384, K=8, R=16, mode="ht", cap=0, fp8=False, balanced=True, s=1.0,
                      backward=False, G=0, kind="prefetch", wbytes=7168 * 2048 * 2),
+    # the inference plan at decode size (a few prefetch slots, overflow rows
+    # read the owner's weights in place) on skewed routing, and the same batch
+    # without a plan
+    "inference_decode": dict(T=1024, H=7168, E=256, K=8, R=8, mode="ht", cap=0, fp8=False, balanced=True, s=1.0,
+                             backward=False, G=0, slots=2, direct=True),
+    "ht_decode": dict(T=1024, H=7168, E=256, K=8, R=8, mode="ht", cap=0, fp8=False, balanced=False, s=1.0,
+                      backward=False, G=0),
 }
+# the workloads timed beside the headline in the default run (sub-records)
+SIDE_WORKLOADS = ("ll_decode", "large_train", "tiny", "router", "prefetch", "inference_decode", "ht_decode")
 HT = WORKLOADS["ht_prefill"]
 SWEEP = WORKLOADS["imbalance"]
 
@@ -237,7 +302,8 @@ class Step:
         self.w_host = w.pin_memory() if host_inputs else w
         self.xd, self.idxd, self.wd = self.x_host.to(dev), self.idx_host.to(dev), self.w_host.to(dev)
         h = ep.Ep(T, H, E, K, R, mode=wl["mode"], ll_capacity=wl["cap"], fp8=wl["fp8"], balanced=wl["balanced"],
-                  grad_elems_per_expert=wl["G"])
+                  replica_slots=wl.get("slots", 0), grad_elems_per_expert=wl["G"],
+                  direct_overflow=wl.get("direct", False))
         self.h = h
         self.bufs = h.empty_recv(dev)
         g = torch.Generator(device=dev).manual_seed(1000 + seed)
@@ -543,6 +609,10 @@ def run_native(args):
         wl["balanced"] = bool(args.balanced)
     if args.capacity:
         wl["cap"] = args.capacity
+    if args.grad_elems:
+        wl["G"] = args.grad_elems
+    if args.weight_bytes:
+        wl["wbytes"] = args.weight_bytes
     name = args.workload if wl == WORKLOADS[args.workload] else args.workload + "_custom"
     seed = rank  # each rank: its own EP world (weak scaling)
     step = Step(wl, dev, seed)
@@ -555,12 +625,16 @@ def run_native(args):
     if not args.no_flush and needs_l2_flush(step_bytes, l2):
         flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    sampler.start()
+    time.sleep(0.3)  # nvidia-smi's first samples arrive after its start-up
     barrier(world)
     torch.cuda.synchronize()
-    sampler.start()
+    t0 = time.time()
     total_ms, per = timed(step, args.steps, args.warmup, stream, min(args.steps, 50), graph=not args.no_graph,
                           flush=flush)
-    clocks = sampler.stop()
+    t1 = time.time()
+    sampler.stop()
+    clocks = sampler.window(t0, t1)
     barrier(world)
     value, ms_step = weak_scaling_value(step_bytes, total_ms / args.steps, world)
     flags = step.h.status(stream) if step.h is not None else 0
@@ -576,30 +650,16 @@ def run_native(args):
 
     e2e = None if (args.no_e2e or step.kind == "prefetch") else run_e2e(step, dev, stream, max(3, min(args.steps, 20)),
                                                                         world, step_bytes)
-    if flush is not None:
-        l2_note = (f"flushed: each step moves {step_bytes / 1e6:.1f} MB, at most 4x L2 ({l2 / 2**20:.0f} MiB), so "
-                   f"a {2 * l2 / 2**20:.0f} MiB buffer is written before every timed step and the steps are "
-                   "timed one by one")
-    elif needs_l2_flush(step_bytes, l2):
-        l2_note = "not flushed (--no-flush): the working set is partly L2-resident"
-    else:
-        l2_note = (f"no flush: each step moves {step_bytes / 1e9:.2f} GB, more than 4x L2 "
-                   f"({l2 / 2**20:.0f} MiB)")
+    l2_note = l2_note_for(step_bytes, l2, flush is not None)
     del flush
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": compute_dtype(wl),
         "data": "synthetic",
-        "config": {"workload": name, "T": wl["T"], "H": wl["H"], "E": wl["E"], "topk": wl["K"],
-                   "logical_ranks": wl["R"], "layout": wl["mode"], "ll_capacity": wl["cap"],
-                   "balanced_plan": wl["balanced"], "zipf_s": wl["s"], "backward": wl["backward"],
-                   "payload": ("bf16 x -> fp8 e4m3 dispatch (per-128 fp32 scales)" if wl["fp8"]
-                               else "bf16 dispatch") + " -> bf16 combine (fp32 accumulation)",
-                   "l2": l2_note,
-                   "parallelism": f"{world} independent EP worlds (one per GPU), R logical ranks each",
-                   "launch": ("stream" if args.no_graph else "CUDA graph replay of the captured step calls")
-                             + (", one step per timed interval" if l2_note.startswith("flushed") else "")},
+        "config": workload_config(name, wl, world, l2_note),
+        "launch": ("stream" if args.no_graph else "CUDA graph replay of the captured step calls")
+                  + (", one step per timed interval" if l2_note.startswith("flushed") else ""),
         "tokens_per_s": round(world * wl["T"] / (ms_step * 1e-3), 1),
         "rows_per_s": round(world * step.placed / (ms_step * 1e-3), 1),
         "frac_of_hbm": round(step_bytes / (ms_step * 1e-3) / 1e9 / peak, 4),
@@ -623,6 +683,8 @@ def run_native(args):
     torch.cuda.empty_cache()
     if not args.no_sweep and args.workload == "ht_prefill":
         result["skew_sweep"] = run_sweep(dev, stream, seed, peak)
+    if not args.no_side and args.workload == "ht_prefill" and name == "ht_prefill":
+        result["workloads"] = run_side_workloads(dev, stream, seed, peak, world, args.no_graph)
     if world == 1 and rank == 0 and not args.no_cpu_baseline and args.workload == "ht_prefill":
         result["cpu_baseline"] = cpu_baseline(args.cpu_sample_tokens)
     if rank == 0:
@@ -733,6 +795,80 @@ def run_sweep(dev, stream, seed, peak, steps=10, warmup=3):
     return rows
 
 
+def side_record(name: str, dev, stream, seed, peak, world, no_graph, steps, warmup, flushed: bool):
+    """One workload timed as the headline is (CUDA-graph replays, CUDA events
+    on the launching stream, max over ranks), with or without an L2 flush
+    before every step: step time, GB/s of algorithmic bytes, fraction of the
+    measured copy bandwidth, per-call split and the clocks seen."""
+    import torch
+
+    from combine_ep_dispatch_03_b200 import ep
+
+    wl = WORKLOADS[name]
+    step = Step(wl, dev, seed, host_inputs=False)
+    nb = step.measure_bytes(stream)
+    step_bytes = sum(nb.values())
+    l2 = l2_bytes(dev)
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev) if flushed else None
+    torch.cuda.synchronize()
+    t0 = time.time()
+    total, per = timed(step, steps, warmup, stream, min(steps, 20), graph=not no_graph, flush=flush)
+    t1 = time.time()
+    gbs, ms = weak_scaling_value(step_bytes, total / steps, world)
+    avg = {k: sum(v) / len(v) for k, v in per.items()}
+    rec = {"ms": round(ms, 4), "gbs": round(gbs, 1), "frac": round(gbs / world / peak, 4),
+           "frac_of_8tbs_nominal": round(gbs / world / 8000.0, 4), "bytes_per_step": step_bytes,
+           "l2": l2_note_for(step_bytes, l2, flushed), "steps": steps,
+           "per_call_us": {k: round(v * 1e3, 2) for k, v in avg.items()},
+           "per_call_gbs": {k: round(nb[k] / (avg[k] * 1e-3) / 1e9, 1) for k in avg},
+           "per_call_frac": {k: round(nb[k] / (avg[k] * 1e-3) / 1e9 / peak, 4) for k in avg},
+           "timed_host_interval": (t0, t1)}  # replaced by the clocks seen in it
+    if step.kind == "path":
+        rec["tokens_per_s"] = round(world * wl["T"] / (ms * 1e-3), 1)
+        rec["flags"] = step.h.status(stream)
+        load = step.h.tensor(ep.T_RANK_LOAD).cpu().tolist()
+        if sum(load):
+            rec["load_max_over_mean"] = round(max(load) / (sum(load) / len(load)), 4)
+    if step.h is not None:
+        step.h.close()
+    del step, flush
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_side_workloads(dev, stream, seed, peak, world, no_graph):
+    """The other workloads of the path, each its own sub-record of the line.
+    Workloads whose step moves at most 4x L2 are timed after an L2 flush
+    before every step (and, for LL decode and the two decode-size plan cases,
+    also back to back without one)."""
+    out = {}
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    for name in SIDE_WORKLOADS:
+        big = name in ("large_train", "prefetch")
+        steps, warmup = (10, 3) if big else (50, 5)
+        small = name in ("ll_decode", "tiny", "router", "inference_decode", "ht_decode")
+        cfg = WORKLOADS[name]
+        rec = {"config": {k: v for k, v in cfg.items() if k not in ("kind",)}}
+        if small:
+            rec["flushed"] = side_record(name, dev, stream, seed, peak, world, no_graph, steps, warmup, True)
+            if name in ("ll_decode", "inference_decode", "ht_decode"):
+                rec["back_to_back"] = side_record(name, dev, stream, seed, peak, world, no_graph, steps, warmup,
+                                                  False)
+        else:
+            rec["back_to_back"] = side_record(name, dev, stream, seed, peak, world, no_graph, steps, warmup, False)
+        out[name] = rec
+    out["clocks"] = sampler.stop()  # every sample of the side workloads together
+    for rec in out.values():
+        for mode in ("flushed", "back_to_back"):
+            if isinstance(rec, dict) and mode in rec:
+                rec[mode]["clocks"] = sampler.window(*rec[mode].pop("timed_host_interval"))
+    if "inference_decode" in out and "ht_decode" in out:
+        a, b = out["inference_decode"]["flushed"]["ms"], out["ht_decode"]["flushed"]["ms"]
+        out["inference_decode"]["over_unplanned_flushed"] = round(a / b, 4)
+    return out
+
+
 def cpu_baseline(sample_tokens: int):
     """The oracle as it stands, single-threaded on a host core, on a bounded
     sample of the HT prefill workload: full routing of all 32768 tokens, then
@@ -803,11 +939,23 @@ def run_reference(args):
     b = algorithmic_bytes(n, H, K, n * K, True)
     gbs = sum(b.values()) / dt / 1e9
     sample = f"ht_prefill: route + FP8 dispatch + combine of {n} of {T} tokens per step"
+    # the GPU arm's config for the same workload (every pair of HT prefill is
+    # placed, so its step bytes follow from the shape)
+    full = algorithmic_bytes(T, H, K, T * K, True)
+    l2 = L2_FALLBACK_BYTES
+    try:
+        import torch
+
+        if torch.cuda.is_available():
+            l2 = l2_bytes(torch.device("cuda", 0))
+    except Exception:
+        pass
+    config = workload_config("ht_prefill", HT, world, l2_note_for(sum(full.values()), l2, False))
     print(json.dumps({
         "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
-        "config": {"workload": "ht_prefill", "T": T, "H": H, "E": E, "topk": K, "logical_ranks": R},
+        "vs_baseline": None, "dtype": compute_dtype(HT), "data": "synthetic", "impl": "reference",
+        "config": config,
         "tokens_per_s": round(n / dt, 1),
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -826,12 +974,17 @@ def main():
     ap.add_argument("--zipf", type=float, default=None, help="override the router's Zipf bias s")
     ap.add_argument("--balanced", type=int, choices=[0, 1], default=None, help="override the balanced plan")
     ap.add_argument("--capacity", type=int, default=0, help="override the LL per-expert capacity (smaller buffers)")
+    ap.add_argument("--grad-elems", type=int, default=0,
+                    help="override the replica-gradient elements per expert (a multiple of 4)")
+    ap.add_argument("--weight-bytes", type=int, default=0,
+                    help="override the prefetch stand-in's bytes per expert (a multiple of 16)")
     ap.add_argument("--no-graph", action="store_true", help="time stream launches instead of CUDA-graph replays")
     ap.add_argument("--no-flush", action="store_true",
                     help="never flush L2 between timed steps (by default steps moving at most 4x L2 are flushed)")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-side", action="store_true", help="skip the other workloads' sub-records")
     ap.add_argument("--cpu-sample-tokens", type=int, default=32768)
     args = ap.parse_args()
     if args.warmup < 3:
