@@ -127,7 +127,8 @@ static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
     X(red_experts, d.E)                                                                                               \
     X(red_count, 1)                                                                                                   \
     X(flags, 1)                                                                                                       \
-    X(ticket, 2)
+    X(ticket, 2)                                                                                                      \
+    X(jbase, d.E)
 
 size_t workspace_bytes(const Dims &d) {
     size_t n = 0;
@@ -277,6 +278,7 @@ ep_status_t ep_destroy(ep_handle_t *h) {
 ep_status_t ep_plan(ep_handle_t *h, const int32_t *topk_idx, void *stream) {
     if (!h) return EP_ERR_INVALID_ARG;
     if (h->d.T > 0 && (!topk_idx || !aligned(topk_idx, 4))) return EP_ERR_INVALID_ARG;
+    h->counts_ready = 0;
     if (launch_plan(h->d, h->ws, topk_idx, as_stream(stream)) != cudaSuccess) return EP_ERR_CUDA;
     h->planned = 1;
     return EP_OK;
@@ -287,6 +289,7 @@ ep_status_t ep_dispatch(ep_handle_t *h, const void *x, const int32_t *topk_idx, 
                         void *stream) {
     if (!h) return EP_ERR_INVALID_ARG;
     if (!h->planned) return EP_ERR_NOT_PLANNED;
+    if (h->planned == 2) return EP_ERR_UNSUPPORTED; // rows are global: the peer calls
     const Dims &d = h->d;
     if (d.T > 0) {
         if (!x || !recv_x || !aligned(x, 16) || !aligned(recv_x, 16)) return EP_ERR_INVALID_ARG;
@@ -306,6 +309,7 @@ ep_status_t ep_dispatch(ep_handle_t *h, const void *x, const int32_t *topk_idx, 
 ep_status_t ep_combine(ep_handle_t *h, const void *expert_out, const float *topk_w, void *out, void *stream) {
     if (!h) return EP_ERR_INVALID_ARG;
     if (!h->planned) return EP_ERR_NOT_PLANNED;
+    if (h->planned == 2) return EP_ERR_UNSUPPORTED; // rows are global: the peer calls
     if (h->d.T > 0 && (!expert_out || !topk_w || !out || !aligned(expert_out, 16) || !aligned(out, 16) ||
                        !aligned(topk_w, 4)))
         return EP_ERR_INVALID_ARG;
@@ -317,6 +321,7 @@ ep_status_t ep_combine_backward(ep_handle_t *h, const void *grad_out, const floa
                                 void *stream) {
     if (!h) return EP_ERR_INVALID_ARG;
     if (!h->planned) return EP_ERR_NOT_PLANNED;
+    if (h->planned == 2) return EP_ERR_UNSUPPORTED; // rows are global: the peer calls
     if (h->d.T > 0 && (!grad_out || !topk_w || !grad_expert_out || !aligned(grad_out, 16) ||
                        !aligned(grad_expert_out, 16) || !aligned(topk_w, 4)))
         return EP_ERR_INVALID_ARG;
@@ -328,6 +333,7 @@ ep_status_t ep_combine_backward(ep_handle_t *h, const void *grad_out, const floa
 ep_status_t ep_dispatch_backward(ep_handle_t *h, const void *grad_recv, void *grad_x, void *stream) {
     if (!h) return EP_ERR_INVALID_ARG;
     if (!h->planned) return EP_ERR_NOT_PLANNED;
+    if (h->planned == 2) return EP_ERR_UNSUPPORTED; // rows are global: the peer calls
     if (h->d.T > 0 && (!grad_recv || !grad_x || !aligned(grad_recv, 16) || !aligned(grad_x, 16)))
         return EP_ERR_INVALID_ARG;
     if (launch_combine(h->d, h->ws, grad_recv, nullptr, grad_x, as_stream(stream)) != cudaSuccess)
@@ -339,6 +345,7 @@ ep_status_t ep_reduce_replica_grads(ep_handle_t *h, const float *replica_grad, f
     if (!h) return EP_ERR_INVALID_ARG;
     if (!h->d.balanced) return EP_ERR_UNSUPPORTED;
     if (!h->planned) return EP_ERR_NOT_PLANNED;
+    if (h->planned == 2) return EP_ERR_UNSUPPORTED; // rows are global: the peer calls
     if (h->d.G > 0 && (!replica_grad || !owner_grad || !aligned(replica_grad, 16) || !aligned(owner_grad, 16)))
         return EP_ERR_INVALID_ARG;
     if (launch_replica_reduce(h->d, h->ws, replica_grad, owner_grad, as_stream(stream)) != cudaSuccess)
@@ -351,6 +358,7 @@ ep_status_t ep_prefetch_replica_weights(ep_handle_t *h, const void *expert_weigh
     if (!h) return EP_ERR_INVALID_ARG;
     if (!h->d.balanced) return EP_ERR_UNSUPPORTED;
     if (!h->planned) return EP_ERR_NOT_PLANNED;
+    if (h->planned == 2) return EP_ERR_UNSUPPORTED; // rows are global: the peer calls
     if (bytes_per_expert <= 0 || bytes_per_expert % 16 != 0 || !expert_weights || !prefetch_slots ||
         !aligned(expert_weights, 16) || !aligned(prefetch_slots, 16))
         return EP_ERR_INVALID_ARG;

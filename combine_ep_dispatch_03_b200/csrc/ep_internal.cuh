@@ -24,7 +24,9 @@ constexpr int kMaxTopk = 32;
 constexpr int kRouterMaxExperts = 1024;   // ep_router_topk keeps a token's logits in one warp's registers
 constexpr int kMaxRouteSmem = 200 * 1024; // dynamic shared memory cap of the routing kernels
 constexpr int kSmallMaxPairs = 1024;      // single-CTA routing up to this many pairs ...
-constexpr int kSmallMaxExperts = 512;     // ... and experts (plain layouts only)
+constexpr int kSmallMaxExperts = 512;     // ... and experts (plain layouts)
+constexpr int kSmallMaxPlanPairs = 1024;  // single-CTA routing with a balanced plan up to this many pairs
+                                          // (beyond it the three kernels measured faster: 8192 pairs, 43 vs 54 us)
 constexpr int kClusterThreads = 1024;     // one-launch cluster routing: threads per CTA, at most
 constexpr int kClusterWarps = kClusterThreads / 32;
 constexpr int kClusterMaxPairs = 32768;  // ... up to this many (token, k) pairs
@@ -61,6 +63,7 @@ struct Workspace {
     int32_t *red_count;      // [1]
     uint32_t *flags;         // [1]: EP_FLAG_* bits of the last plan
     unsigned long long *ticket; // [1]: CTAs of the scan kernel that have finished
+    int32_t *jbase;          // [E]: world plan: this rank's first stable index within each expert
 };
 
 struct Dims {
@@ -76,6 +79,7 @@ struct Dims {
     int cl_warps;            // cluster routing: warps per CTA (16 or 32)
     int nx_max;              // bound on extra pieces (R*S + E with a plan, else 0)
     int counts_len;          // recv_counts entries
+    int world;               // 1: the routing completes a world plan (global rows, see ep_plan_world)
 };
 
 // Sizes derived from a validated configuration; also used by the host-only
@@ -96,6 +100,11 @@ int plan_launches(const Dims &d);
 
 // ---- launchers (each returns the launch's cudaError_t) ----
 cudaError_t launch_plan(const Dims &d, const Workspace &ws, const int32_t *topk_idx, cudaStream_t st);
+// world mode (ep_plan_local_counts / ep_plan_world)
+cudaError_t launch_plan_local_counts(const Dims &d, const Workspace &ws, const int32_t *topk_idx, cudaStream_t st);
+cudaError_t launch_plan_world(const Dims &d, const Workspace &ws, const int32_t *world_counts, int rank,
+                              cudaStream_t st);
+size_t route_smem_world(const Dims &d);
 cudaError_t launch_dispatch(const Dims &d, const Workspace &ws, const void *x, const int32_t *topk_idx,
                             const float *topk_w, void *recv_x, float *recv_scales, float *recv_w,
                             int32_t *recv_expert, int32_t *recv_counts, cudaStream_t st);
@@ -109,6 +118,10 @@ cudaError_t launch_replica_reduce(const Dims &d, const Workspace &ws, const floa
                                   cudaStream_t st);
 
 int num_sms();
+// row movers' launch shape: vectors per thread and threads per CTA for a row
+// part of n 16-byte vectors; vectors per row part for T rows of nvec vectors
+void pick_shape(int n, int *per_thread, int *threads);
+int row_part(int T, int nvec);
 
 // Programmatic dependent launch: every kernel of the library waits for the
 // grid before it in the stream to complete (and its writes to be visible)
@@ -143,5 +156,7 @@ struct ep_handle {
     epb::Workspace ws;
     void *base;
     int device;
-    int planned;
+    int planned;       // 0 none, 1 ep_plan (single-GPU layout), 2 ep_plan_world (global rows)
+    int counts_ready;  // ep_plan_local_counts ran since the last plan
+    int world_rank;    // this handle's rank in its world plan
 };

@@ -760,15 +760,17 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspac
     int32_t *s_len = sm;         // [E] length of piece 0
     int32_t *s_base = s_len + E; // [E] first row of piece 0
     int32_t *s_cnt = s_base + E; // [E] (plain layouts)
-    int32_t *s_xoff = s_cnt + E; // [E+1] extra pieces (plan only)
+    int32_t *s_xoff = s_cnt + E; // [E+1] extra pieces (plan or world)
     int32_t *s_xs = s_xoff + E + 1;
     int32_t *s_xl = s_xs + d.nx_max;
     int32_t *s_xd = s_xl + d.nx_max;
+    int32_t *s_jb = s_xd + d.nx_max; // [E] world: this rank's first stable index per expert
     if (tid == 0) s_fl = 0;
-    if (d.balanced) {
+    if (d.balanced || d.world) {
         for (int i = tid; i < E; i += nth) {
             s_base[i] = ws.base0[i];
             s_len[i] = ws.len0[i];
+            if (d.world) s_jb[i] = ws.jbase[i];
         }
         for (int i = tid; i <= E; i += nth) s_xoff[i] = ws.xoff[i];
         const int nx = ws.xoff[E];
@@ -813,10 +815,10 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspac
         const int e = pk[u] & 0xffff;
         int dest = -1;
         if (e != 0xffff) {
-            const int j = jb[u] + (pk[u] >> 16);
+            const int j = jb[u] + (pk[u] >> 16) + (d.world ? s_jb[e] : 0);
             if (j < s_len[e]) {
                 dest = s_base[e] + j;
-            } else if (d.balanced) {
+            } else if (d.balanced || d.world) {
                 for (int x = s_xoff[e]; x < s_xoff[e + 1]; ++x)
                     if (j >= s_xs[x] && j < s_xs[x] + s_xl[x]) {
                         dest = s_xd[x] + (j - s_xs[x]);
@@ -825,8 +827,55 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspac
             }
         }
         ws.dest_row[p] = dest;
-        if (dest >= 0 && ws.src_row) ws.src_row[dest] = (int32_t)p;
+        if (dest >= 0 && ws.src_row && !d.world) ws.src_row[dest] = (int32_t)p; // world rows are global
     }
+}
+
+// ---------------------------------------------------------------------------
+// world plan: the global layout from every rank's counts (one CTA). Every
+// rank runs it on the same counts and computes the same tables; jbase holds
+// the pairs of expert e on lower ranks, which come first in the expert's
+// stable order (source rank, t, k).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kPlanThreads) k_route_world(Dims d, Workspace ws,
+                                                               const int32_t *__restrict__ wc, int rank) {
+    pdl_wait();
+    pdl_launch_dependents();
+    extern __shared__ int32_t sm[];
+    __shared__ int32_t s_warp[33];
+    __shared__ uint32_t s_fl;
+    const int E = d.E, R = d.R, tid = threadIdx.x, nth = blockDim.x;
+    int32_t *s_cnt = sm;          // [E] the world's counts
+    int32_t *s_len = s_cnt + E;   // [E] plain layouts
+    int32_t *s_base = s_len + E;  // [E]
+    int32_t *s_plan = s_base + E; // the planner's scratch (balanced)
+    if (tid == 0) s_fl = 0;
+    __syncthreads();
+    uint32_t fl = 0; // this rank's id checks, from its histogram CTAs
+    for (int b = tid; b < d.nhist; b += nth) fl |= ws.tile_flags[b];
+    block_or(fl, &s_fl);
+    for (int e = tid; e < E; e += nth) {
+        int all = 0, before = 0;
+        for (int r = 0; r < R; ++r) {
+            const int v = wc[(int64_t)r * E + e];
+            all += v;
+            if (r < rank) before += v;
+        }
+        s_cnt[e] = all;
+        ws.cnt[e] = all;
+        ws.jbase[e] = before;
+        ws.xoff[e] = 0; // plain layouts have no extra pieces; the planner rewrites them
+    }
+    if (tid == 0) ws.xoff[E] = 0;
+    __syncthreads();
+    if (d.balanced) {
+        layout_balanced(d, ws, s_cnt, s_plan, s_warp, &s_fl);
+    } else {
+        const int total = plain_tables(d, s_cnt, s_len, s_base, s_warp, &s_fl);
+        plain_outputs(d, ws, s_len, s_base, total);
+    }
+    __syncthreads();
+    if (tid == 0) *ws.flags = s_fl;
 }
 
 // ---------------------------------------------------------------------------
@@ -966,7 +1015,8 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
 }
 
 // ---------------------------------------------------------------------------
-// small batches, plain layouts: everything in one CTA
+// small batches: everything in one CTA (counts, layout or balanced plan,
+// assignment), one launch
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__restrict__ idx, Dims d,
                                                                 Workspace ws) {
@@ -978,9 +1028,10 @@ __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__
     const int E = d.E, K = d.K, w = threadIdx.x >> 5, np = (int)d.L;
     int32_t *s_wc = sm;                   // [warps][E]
     int32_t *s_cnt = s_wc + kSmallWarps * E;
-    int32_t *s_len = s_cnt + E;
-    int32_t *s_base = s_len + E;
+    int32_t *s_len = s_cnt + E;           // [E] kept rows (plain) / rows of piece 0 (plan)
+    int32_t *s_base = s_len + E;          // [E] first row of the expert / of piece 0
     int32_t *s_ids = s_base + E;          // [L]
+    int32_t *s_plan = s_ids + np;         // the planner's scratch (balanced only)
     if (threadIdx.x == 0) s_fl = 0;
     for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) s_wc[i] = 0;
     load_ids(idx, 0, np, s_ids);
@@ -1005,10 +1056,29 @@ __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__
         ws.cnt[e] = run;
     }
     __syncthreads();
-    const int total = plain_tables(d, s_cnt, s_len, s_base, s_warp, &s_fl);
-    plain_outputs(d, ws, s_len, s_base, total);
-    warp_assign(s_ids, lo, hi, K, E, my, ws.dest_row, ws.src_row,
-                [&](int e, int j) { return j < s_len[e] ? s_base[e] + j : -1; });
+    if (!d.balanced) {
+        const int total = plain_tables(d, s_cnt, s_len, s_base, s_warp, &s_fl);
+        plain_outputs(d, ws, s_len, s_base, total);
+        warp_assign(s_ids, lo, hi, K, E, my, ws.dest_row, ws.src_row,
+                    [&](int e, int j) { return j < s_len[e] ? s_base[e] + j : -1; });
+    } else {
+        // The plan's tables go to the workspace; this CTA's own writes are
+        // visible to it after the barrier. Piece 0 of each expert is kept in
+        // shared memory, the few extra pieces are read from the workspace.
+        layout_balanced(d, ws, s_cnt, s_plan, s_warp, &s_fl);
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            s_len[e] = ws.len0[e];
+            s_base[e] = ws.base0[e];
+        }
+        __syncthreads();
+        const int32_t *xoff = ws.xoff, *xs = ws.xstart, *xl = ws.xlen, *xd = ws.xdst;
+        warp_assign(s_ids, lo, hi, K, E, my, ws.dest_row, ws.src_row, [&](int e, int j) {
+            if (j < s_len[e]) return s_base[e] + j;
+            for (int x = xoff[e]; x < xoff[e + 1]; ++x)
+                if (j >= xs[x] && j < xs[x] + xl[x]) return xd[x] + (j - xs[x]);
+            return -1;
+        });
+    }
     __syncthreads();
     if (threadIdx.x == 0) *ws.flags = s_fl;
 }
@@ -1024,13 +1094,18 @@ size_t route_smem_layout(const Dims &d) {
 size_t route_smem_assign(const Dims &d) {
     const size_t E = d.E;
     size_t n = 3 * E;
-    if (d.balanced) n += E + 1 + 3 * (size_t)d.nx_max;
+    if (d.balanced || d.world) n += E + 1 + 3 * (size_t)d.nx_max;
+    if (d.world) n += E;
     return sizeof(int32_t) * n;
 }
 
+size_t route_smem_world(const Dims &d) { return sizeof(int32_t) * 3 * (size_t)d.E + route_smem_layout(d); }
+
 size_t route_smem_hist(const Dims &d) { return sizeof(int32_t) * (size_t)kRouteWarps * (d.E + d.wt); }
 
-size_t route_smem_small(const Dims &d) { return sizeof(int32_t) * ((size_t)(kSmallWarps + 3) * d.E + d.L); }
+size_t route_smem_small(const Dims &d) {
+    return sizeof(int32_t) * ((size_t)(kSmallWarps + 3) * d.E + d.L) + route_smem_layout(d);
+}
 
 size_t route_smem_cluster(const Dims &d) {
     return sizeof(int32_t) * ((size_t)(d.cl_warps + 4 + d.cl_size) * d.E + 2 * (size_t)d.cl_ppw * d.cl_warps);
@@ -1076,22 +1151,14 @@ bool route_use_cluster(const Dims &d) {
 }
 
 bool route_use_small(const Dims &d) {
-    return !d.balanced && d.L <= kSmallMaxPairs && d.E <= kSmallMaxExperts;
+    if (d.balanced) return d.L <= kSmallMaxPlanPairs && route_smem_small(d) <= (size_t)kMaxRouteSmem;
+    return d.L <= kSmallMaxPairs && d.E <= kSmallMaxExperts;
 }
 
+static void set_route_attrs();
+
 cudaError_t launch_plan(const Dims &d, const Workspace &ws, const int32_t *topk_idx, cudaStream_t st) {
-    // per-device function attributes, set once; the flag is published after them
-    static std::atomic<bool> attrs_set[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attrs_set[dev].load(std::memory_order_acquire)) {
-        const int max_dyn = kMaxRouteSmem;
-        cudaFuncSetAttribute(k_route_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
-        cudaFuncSetAttribute(k_route_assign, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
-        cudaFuncSetAttribute(k_route_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
-        cudaFuncSetAttribute(k_route_small, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
-        attrs_set[dev].store(true, std::memory_order_release);
-    }
+    set_route_attrs();
     cudaError_t err;
     if (route_use_cluster(d)) {
         cudaLaunchConfig_t cfg = {};
@@ -1119,6 +1186,50 @@ cudaError_t launch_plan(const Dims &d, const Workspace &ws, const int32_t *topk_
     err = launch_pdl(k_route_scan, dim3((d.E + 31) / 32), dim3(kPlanThreads), route_smem_layout(d), st, d, ws);
     if (err != cudaSuccess) return err;
     return launch_pdl(k_route_assign, dim3(d.nassign), dim3(kRouteThreads), route_smem_assign(d), st, d, ws);
+}
+
+static void set_route_attrs() {
+    // per-device function attributes, set once; the flag is published after them
+    static std::atomic<bool> attrs_set[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attrs_set[dev].load(std::memory_order_acquire)) {
+        const int max_dyn = kMaxRouteSmem;
+        cudaFuncSetAttribute(k_route_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+        cudaFuncSetAttribute(k_route_assign, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+        cudaFuncSetAttribute(k_route_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+        cudaFuncSetAttribute(k_route_small, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+        cudaFuncSetAttribute(k_route_world, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn);
+        attrs_set[dev].store(true, std::memory_order_release);
+    }
+}
+
+// World mode, step 1: the histogram and the per-tile scan of this rank's
+// pairs (the three-kernel path's first two kernels, without a plan); the
+// per-expert counts are left in ws.cnt.
+cudaError_t launch_plan_local_counts(const Dims &d, const Workspace &ws, const int32_t *topk_idx, cudaStream_t st) {
+    set_route_attrs();
+    Dims dl = d;
+    dl.balanced = 0;
+    dl.world = 0;
+    cudaError_t err;
+    if (dl.L > 0) {
+        err = launch_pdl(k_route_hist, dim3(dl.nhist), dim3(kRouteThreads), route_smem_hist(dl), st, topk_idx, dl, ws);
+        if (err != cudaSuccess) return err;
+    }
+    return launch_pdl(k_route_scan, dim3((dl.E + 31) / 32), dim3(kPlanThreads), (size_t)0, st, dl, ws);
+}
+
+// World mode, step 2: the global layout (one CTA), then each pair's global row.
+cudaError_t launch_plan_world(const Dims &d, const Workspace &ws, const int32_t *world_counts, int rank,
+                              cudaStream_t st) {
+    set_route_attrs();
+    Dims dw = d;
+    dw.world = 1;
+    cudaError_t err =
+        launch_pdl(k_route_world, dim3(1), dim3(kPlanThreads), route_smem_world(dw), st, dw, ws, world_counts, rank);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(k_route_assign, dim3(dw.nassign), dim3(kRouteThreads), route_smem_assign(dw), st, dw, ws);
 }
 
 int plan_launches(const Dims &d) {

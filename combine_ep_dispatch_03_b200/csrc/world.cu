@@ -1,0 +1,497 @@
+// world.cu -- expert parallelism across GPUs, one rank per GPU: the send and
+// receive halves of dispatch over peer memory, completion flags, combine that
+// reads the peers' expert outputs, and CUDA IPC for building the peer table.
+//
+// NCCL EP paper (arXiv 2603.13606): the staged mode splits dispatch and
+// combine into send and receive phases (Table II, Fig. 2); LL mode runs as an
+// all-to-all mesh and combine reduces per token at the receiver (Table III).
+// MoonEP article, para. 4: rows go straight into expert-grouped positions on
+// the remote rank, with no staging copy through a communication buffer.
+//
+// The routing of a world plan (global rows) is in route.cu. Here a global row
+// g is mapped to its rank r (the last r with rank_off[r] <= g) and local row
+// g - rank_off[r], and every row moves with plain 16-byte stores (dispatch)
+// or loads (combine) through the peer table: over NVLink when the table holds
+// other GPUs' mapped buffers, within one HBM when it holds local ones. No bulk
+// or multicast copy touches a peer's memory.
+#include <string.h>
+
+#include "bulk.cuh"
+#include "ep_internal.cuh"
+#include "rows.cuh"
+
+namespace epb {
+namespace {
+
+// the peers' receive arrays, passed by value as a kernel parameter
+struct PeerRows {
+    uint8_t *x[EP_MAX_PEERS];
+    float *scales[EP_MAX_PEERS];
+    float *w[EP_MAX_PEERS];
+    int32_t *expert[EP_MAX_PEERS];
+    int64_t cap; // rows of every rank's receive buffer
+};
+
+struct PeerFlags {
+    uint32_t *f[EP_MAX_PEERS];
+};
+
+// The rank holding global row g: the last r with roff[r] <= g (roff ascending
+// from roff[0] = 0; empty ranks share their offset with the next rank).
+__device__ __forceinline__ int row_rank(const int32_t *roff, int R, int g) {
+    int lo = 0, hi = R - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (roff[mid] <= g)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+// Threads k < K of the CTA: rank and local row of pair (t, k), or rank -1 for
+// a pair without a row or with a row beyond the capacity (flagged).
+__device__ __forceinline__ void stage_peer_rows(const int32_t *__restrict__ dest_row,
+                                                const int32_t *__restrict__ rank_off, int R, int K, int64_t pb,
+                                                int64_t cap, int32_t *s_roff, int *s_rank, int64_t *s_lrow,
+                                                uint32_t *status) {
+    for (int i = threadIdx.x; i <= R; i += blockDim.x) s_roff[i] = rank_off[i];
+    __syncthreads();
+    if (threadIdx.x < K) {
+        const int g = dest_row[pb + threadIdx.x];
+        int r = -1;
+        int64_t lr = -1;
+        if (g >= 0) {
+            r = row_rank(s_roff, R, g);
+            lr = g - s_roff[r];
+            if (lr >= cap) {
+                if (status) atomicOr(status, EP_FLAG_CAPACITY);
+                r = -1;
+            }
+        }
+        s_rank[threadIdx.x] = r;
+        s_lrow[threadIdx.x] = lr;
+    }
+}
+
+// dispatch send, bf16 rows: one CTA per (token, row part), VPT 16-byte vectors
+// a thread; the token's vectors are read once and stored K times.
+template <int VPT>
+__global__ void __launch_bounds__(256) k_dispatch_peers(const uint4 *__restrict__ x, const int32_t *__restrict__ idx,
+                                                        const float *__restrict__ w,
+                                                        const int32_t *__restrict__ dest_row,
+                                                        const int32_t *__restrict__ rank_off, int R, int K, int nvec,
+                                                        int part, PeerRows pr, uint32_t *__restrict__ status) {
+    __shared__ int32_t s_roff[EP_MAX_PEERS + 1];
+    __shared__ int s_rank[kMaxTopk];
+    __shared__ int64_t s_lrow[kMaxTopk];
+    __shared__ uint4 *s_dst[kMaxTopk];
+    const int t = blockIdx.x;
+    const int64_t pb = (int64_t)t * K;
+    const int cb = blockIdx.y * part, n = min(part, nvec - cb);
+    const uint4 *src = x + (int64_t)t * nvec + cb;
+    const int step = VPT * blockDim.x;
+    uint4 v[VPT];
+    load_slab<VPT>(src, 0, n, v); // before the wait: the routing never writes x
+    pdl_wait();
+    stage_peer_rows(dest_row, rank_off, R, K, pb, pr.cap, s_roff, s_rank, s_lrow,
+                    blockIdx.y == 0 ? status : nullptr);
+    if (threadIdx.x < K) {
+        const int r = s_rank[threadIdx.x];
+        const int64_t lr = s_lrow[threadIdx.x];
+        s_dst[threadIdx.x] = r >= 0 ? reinterpret_cast<uint4 *>(pr.x[r]) + lr * nvec + cb : nullptr;
+        if (r >= 0 && blockIdx.y == 0) {
+            if (pr.w[r]) pr.w[r][lr] = w[pb + threadIdx.x];
+            if (pr.expert[r]) pr.expert[r][lr] = idx[pb + threadIdx.x];
+        }
+    }
+    __syncthreads();
+    for (int c0 = 0; c0 < n; c0 += step) {
+        if (c0 > 0) load_slab<VPT>(src, c0, n, v);
+        for (int k = 0; k < K; ++k) {
+            uint4 *dst = s_dst[k];
+            if (!dst) continue;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int c = c0 + threadIdx.x + i * blockDim.x;
+                if (c < n) dst[c] = v[i];
+            }
+        }
+    }
+}
+
+// dispatch send, FP8 rows: the same cast as the single-GPU FP8 dispatch (one
+// thread per 16-element chunk, the 8 lanes of a 128-element block reduce its
+// amax), then the codes and scales stored to each pair's rank.
+template <int CPT>
+__global__ void __launch_bounds__(256) k_dispatch_peers_fp8(const uint4 *__restrict__ x,
+                                                            const int32_t *__restrict__ idx,
+                                                            const float *__restrict__ w,
+                                                            const int32_t *__restrict__ dest_row,
+                                                            const int32_t *__restrict__ rank_off, int R, int K,
+                                                            int nchunk, int part, PeerRows pr,
+                                                            uint32_t *__restrict__ status) {
+    __shared__ int32_t s_roff[EP_MAX_PEERS + 1];
+    __shared__ int s_rank[kMaxTopk];
+    __shared__ int64_t s_lrow[kMaxTopk];
+    __shared__ uint4 *s_dst[kMaxTopk];
+    __shared__ float *s_sc[kMaxTopk];
+    const int t = blockIdx.x;
+    const int64_t pb = (int64_t)t * K;
+    const int nb = nchunk >> 3; // 128-element blocks per row
+    const int cb = blockIdx.y * part, n = min(part, nchunk - cb); // part: whole blocks
+    const uint4 *src = x + (int64_t)t * 2 * nchunk + 2 * cb;
+    const int step = CPT * blockDim.x;
+    uint4 a[CPT], b[CPT];
+    load_pairs<CPT>(src, 0, n, a, b); // before the wait: the routing never writes x
+    pdl_wait();
+    stage_peer_rows(dest_row, rank_off, R, K, pb, pr.cap, s_roff, s_rank, s_lrow,
+                    blockIdx.y == 0 ? status : nullptr);
+    if (threadIdx.x < K) {
+        const int r = s_rank[threadIdx.x];
+        const int64_t lr = s_lrow[threadIdx.x];
+        s_dst[threadIdx.x] = r >= 0 ? reinterpret_cast<uint4 *>(pr.x[r]) + lr * nchunk + cb : nullptr;
+        s_sc[threadIdx.x] = r >= 0 ? pr.scales[r] + lr * nb + (cb >> 3) : nullptr;
+        if (r >= 0 && blockIdx.y == 0) {
+            if (pr.w[r]) pr.w[r][lr] = w[pb + threadIdx.x];
+            if (pr.expert[r]) pr.expert[r][lr] = idx[pb + threadIdx.x];
+        }
+    }
+    __syncthreads();
+    for (int c0 = 0; c0 < n; c0 += step) {
+        if (c0 > 0) load_pairs<CPT>(src, c0, n, a, b);
+        uint4 q[CPT];
+        float sc[CPT];
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) quant_chunk(a[i], b[i], q[i], sc[i]);
+        for (int k = 0; k < K; ++k) {
+            uint4 *dst = s_dst[k];
+            if (!dst) continue;
+            float *scr = s_sc[k];
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) {
+                const int c = c0 + threadIdx.x + i * blockDim.x;
+                if (c < n) {
+                    dst[c] = q[i];
+                    if ((c & 7) == 0) scr[c >> 3] = sc[i];
+                }
+            }
+        }
+    }
+}
+
+// combine across ranks: out[t] = bf16(fold_k fmaf(w[t,k], y_k, acc)) with y_k
+// the pair's row in its rank's expert outputs, k in order, acc from +0.
+template <int CPT>
+__global__ void __launch_bounds__(256) k_combine_peers(PeerRows pr, const float *__restrict__ w,
+                                                       const int32_t *__restrict__ dest_row,
+                                                       const int32_t *__restrict__ rank_off, int R, int K, int nvec,
+                                                       int part, uint4 *__restrict__ out) {
+    __shared__ int32_t s_roff[EP_MAX_PEERS + 1];
+    __shared__ int s_rank[kMaxTopk];
+    __shared__ int64_t s_lrow[kMaxTopk];
+    __shared__ const uint4 *s_src[kMaxTopk];
+    __shared__ float s_w[kMaxTopk];
+    pdl_wait();
+    const int t = blockIdx.x;
+    const int64_t pb = (int64_t)t * K;
+    const int cb = blockIdx.y * part, n = min(part, nvec - cb);
+    stage_peer_rows(dest_row, rank_off, R, K, pb, pr.cap, s_roff, s_rank, s_lrow, nullptr);
+    if (threadIdx.x < K) {
+        const int r = s_rank[threadIdx.x];
+        s_src[threadIdx.x] =
+            r >= 0 ? reinterpret_cast<const uint4 *>(pr.x[r]) + s_lrow[threadIdx.x] * nvec + cb : nullptr;
+        s_w[threadIdx.x] = w[pb + threadIdx.x];
+    }
+    __syncthreads();
+    const int step = CPT * blockDim.x;
+    for (int c0 = 0; c0 < n; c0 += step) {
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = c0 + threadIdx.x + i * blockDim.x;
+            if (c >= n) continue;
+            float acc[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
+            for (int k0 = 0; k0 < K; k0 += 8) {
+                uint4 v[8];
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const int k = k0 + kk;
+                    const uint4 *p = k < K ? s_src[k] : nullptr;
+                    v[kk] = p ? p[c] : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const int k = k0 + kk;
+                    if (k >= K || !s_src[k]) continue;
+                    float f[8];
+                    unpack8(v[kk], f);
+                    const float wk = s_w[k];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) acc[u] = __fmaf_rn(wk, f[u], acc[u]);
+                }
+            }
+            out[(int64_t)t * nvec + cb + c] = pack8(acc);
+        }
+    }
+}
+
+__device__ __forceinline__ void st_release_sys(uint32_t *p, uint32_t v) {
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// signal: after the kernels before it (griddepcontrol.wait), a system-scope
+// fence, then flags[r][rank] = epoch on every rank r (release).
+__global__ void __launch_bounds__(64) k_signal(PeerFlags pf, int R, int rank, uint32_t epoch) {
+    pdl_wait();
+    __threadfence_system();
+    for (int r = threadIdx.x; r < R; r += blockDim.x) st_release_sys(pf.f[r] + rank, epoch);
+}
+
+// wait: thread s polls flags[s] (acquire) until it reaches epoch (wrapping
+// 32-bit comparison), for at most limit_ns; a thread that gives up sets
+// EP_FLAG_WAIT_TIMEOUT. Nothing else runs in this kernel, and the kernels
+// after it start only when it has completed.
+__global__ void __launch_bounds__(64) k_wait(const uint32_t *flags, int R, uint32_t epoch, uint64_t limit_ns,
+                                             uint32_t *status) {
+    pdl_wait();
+    for (int s = threadIdx.x; s < R; s += blockDim.x) {
+        const uint64_t t0 = global_ns();
+        while ((int32_t)(ld_acquire_sys(flags + s) - epoch) < 0) {
+            if (global_ns() - t0 > limit_ns) {
+                atomicOr(status, EP_FLAG_WAIT_TIMEOUT);
+                break;
+            }
+            __nanosleep(256);
+        }
+    }
+}
+
+} // namespace
+} // namespace epb
+
+using namespace epb;
+
+static inline bool aligned_to(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// common checks of a peer table against a handle
+static ep_status_t check_table(const ep_handle_t *h, const ep_peer_table_t *pt, bool need_x) {
+    if (!pt || pt->num_ranks != h->d.R || h->d.R > EP_MAX_PEERS || pt->capacity_rows < 0) return EP_ERR_INVALID_ARG;
+    if (pt->capacity_rows > INT32_MAX) return EP_ERR_INVALID_ARG;
+    if (need_x)
+        for (int r = 0; r < h->d.R; ++r)
+            if (!pt->recv_x[r] || !aligned_to(pt->recv_x[r], 16)) return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+static void fill_rows(const ep_peer_table_t *pt, int R, PeerRows *pr) {
+    memset(pr, 0, sizeof *pr);
+    for (int r = 0; r < R; ++r) {
+        pr->x[r] = (uint8_t *)pt->recv_x[r];
+        pr->scales[r] = pt->recv_scales[r];
+        pr->w[r] = pt->recv_w[r];
+        pr->expert[r] = pt->recv_expert[r];
+    }
+    pr->cap = pt->capacity_rows;
+}
+
+extern "C" {
+
+ep_status_t ep_world_recv_rows(const ep_config_t *cfg, int64_t *rows) {
+    Dims d;
+    if (!rows) return EP_ERR_INVALID_ARG;
+    const ep_status_t s = derive_dims(cfg, &d);
+    if (s != EP_OK) return s;
+    if (d.mode == EP_MODE_LL)
+        *rows = (int64_t)d.g * d.cap;
+    else
+        *rows = d.balanced ? d.L : (int64_t)d.R * d.L; // ceil(R*L / R) = L with a plan
+    return EP_OK;
+}
+
+ep_status_t ep_plan_local_counts(ep_handle_t *h, const int32_t *topk_idx, int32_t *counts, void *stream) {
+    if (!h || !counts || !aligned_to(counts, 4)) return EP_ERR_INVALID_ARG;
+    if (h->d.T > 0 && (!topk_idx || !aligned_to(topk_idx, 4))) return EP_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    h->planned = 0;
+    h->counts_ready = 0;
+    if (launch_plan_local_counts(h->d, h->ws, topk_idx, st) != cudaSuccess) return EP_ERR_CUDA;
+    if (cudaMemcpyAsync(counts, h->ws.cnt, sizeof(int32_t) * h->d.E, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return EP_ERR_CUDA;
+    h->counts_ready = 1;
+    return EP_OK;
+}
+
+ep_status_t ep_plan_world(ep_handle_t *h, const int32_t *world_counts, int32_t rank, void *stream) {
+    if (!h || !world_counts || !aligned_to(world_counts, 4) || rank < 0 || rank >= h->d.R) return EP_ERR_INVALID_ARG;
+    if (!h->counts_ready) return EP_ERR_NOT_PLANNED;
+    if (h->d.R > EP_MAX_PEERS) return EP_ERR_UNSUPPORTED;
+    if ((int64_t)h->d.R * h->d.L > INT32_MAX / 2) return EP_ERR_INVALID_ARG; // global rows fit 31 bits
+    Dims dw = h->d;
+    dw.world = 1;
+    if (route_smem_world(dw) > (size_t)kMaxRouteSmem || route_smem_assign(dw) > (size_t)kMaxRouteSmem)
+        return EP_ERR_UNSUPPORTED;
+    if (launch_plan_world(h->d, h->ws, world_counts, rank, (cudaStream_t)stream) != cudaSuccess) return EP_ERR_CUDA;
+    h->planned = 2;
+    h->world_rank = rank;
+    return EP_OK;
+}
+
+ep_status_t ep_dispatch_peers(ep_handle_t *h, const void *x, const int32_t *topk_idx, const float *topk_w,
+                              const ep_peer_table_t *peers, void *stream) {
+    if (!h) return EP_ERR_INVALID_ARG;
+    if (h->planned != 2) return h->planned == 1 ? EP_ERR_UNSUPPORTED : EP_ERR_NOT_PLANNED;
+    const Dims &d = h->d;
+    ep_status_t s = check_table(h, peers, true);
+    if (s != EP_OK) return s;
+    bool any_w = false, any_e = false;
+    for (int r = 0; r < d.R; ++r) {
+        if (peers->recv_w[r] && !aligned_to(peers->recv_w[r], 4)) return EP_ERR_INVALID_ARG;
+        if (peers->recv_expert[r] && !aligned_to(peers->recv_expert[r], 4)) return EP_ERR_INVALID_ARG;
+        if (d.fp8 && (!peers->recv_scales[r] || !aligned_to(peers->recv_scales[r], 4))) return EP_ERR_INVALID_ARG;
+        if (!d.fp8 && peers->recv_scales[r]) return EP_ERR_INVALID_ARG;
+        any_w |= peers->recv_w[r] != nullptr;
+        any_e |= peers->recv_expert[r] != nullptr;
+    }
+    if (d.T == 0) return EP_OK;
+    if (!x || !aligned_to(x, 16)) return EP_ERR_INVALID_ARG;
+    if (any_w && (!topk_w || !aligned_to(topk_w, 4))) return EP_ERR_INVALID_ARG;
+    if (any_e && (!topk_idx || !aligned_to(topk_idx, 4))) return EP_ERR_INVALID_ARG;
+    PeerRows pr;
+    fill_rows(peers, d.R, &pr);
+    cudaStream_t st = (cudaStream_t)stream;
+    int per, threads;
+    cudaError_t err;
+    if (d.fp8) {
+        const int nchunk = d.H / 16;
+        const int part = row_part(d.T, nchunk);
+        const dim3 grid(d.T, (nchunk + part - 1) / part);
+        pick_shape(part, &per, &threads);
+#define EPB_PEER_FP8(C)                                                                                              \
+    launch_pdl(k_dispatch_peers_fp8<C>, grid, dim3(threads), 0, st, (const uint4 *)x, topk_idx, topk_w, h->ws.dest_row, \
+               h->ws.rank_off, d.R, d.K, nchunk, part, pr, h->ws.flags)
+        err = per == 1 ? EPB_PEER_FP8(1) : per == 2 ? EPB_PEER_FP8(2) : per == 4 ? EPB_PEER_FP8(4) : EPB_PEER_FP8(8);
+#undef EPB_PEER_FP8
+    } else {
+        const int nvec = d.H / 8;
+        const int part = row_part(d.T, nvec);
+        const dim3 grid(d.T, (nvec + part - 1) / part);
+        pick_shape(part, &per, &threads);
+#define EPB_PEER_BF16(V)                                                                                             \
+    launch_pdl(k_dispatch_peers<V>, grid, dim3(threads), 0, st, (const uint4 *)x, topk_idx, topk_w, h->ws.dest_row,   \
+               h->ws.rank_off, d.R, d.K, nvec, part, pr, h->ws.flags)
+        err = per == 1 ? EPB_PEER_BF16(1) : per == 2 ? EPB_PEER_BF16(2) : per == 4 ? EPB_PEER_BF16(4) : EPB_PEER_BF16(8);
+#undef EPB_PEER_BF16
+    }
+    return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+ep_status_t ep_signal_peers(ep_handle_t *h, const ep_peer_table_t *peers, uint32_t epoch, void *stream) {
+    if (!h) return EP_ERR_INVALID_ARG;
+    ep_status_t s = check_table(h, peers, false);
+    if (s != EP_OK) return s;
+    PeerFlags pf;
+    memset(&pf, 0, sizeof pf);
+    for (int r = 0; r < h->d.R; ++r) {
+        if (!peers->flags[r] || !aligned_to(peers->flags[r], 4)) return EP_ERR_INVALID_ARG;
+        pf.f[r] = peers->flags[r];
+    }
+    // the rank index of this handle: the one ep_plan_world was given
+    if (h->planned != 2) return EP_ERR_NOT_PLANNED;
+    const cudaError_t err =
+        launch_pdl(k_signal, dim3(1), dim3(64), 0, (cudaStream_t)stream, pf, h->d.R, h->world_rank, epoch);
+    return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+ep_status_t ep_wait_peers(ep_handle_t *h, const uint32_t *flags, uint32_t epoch, int64_t timeout_us, void *stream) {
+    if (!h || !flags || !aligned_to(flags, 4) || timeout_us < 0 || timeout_us > 600000000) return EP_ERR_INVALID_ARG;
+    const uint64_t limit_ns = timeout_us == 0 ? kWaitLimitNs : (uint64_t)timeout_us * 1000ull;
+    const cudaError_t err =
+        launch_pdl(k_wait, dim3(1), dim3(64), 0, (cudaStream_t)stream, flags, h->d.R, epoch, limit_ns, h->ws.flags);
+    return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+ep_status_t ep_combine_peers(ep_handle_t *h, const ep_peer_table_t *peers, const float *topk_w, void *out,
+                             void *stream) {
+    if (!h) return EP_ERR_INVALID_ARG;
+    if (h->planned != 2) return h->planned == 1 ? EP_ERR_UNSUPPORTED : EP_ERR_NOT_PLANNED;
+    const Dims &d = h->d;
+    ep_status_t s = check_table(h, peers, true);
+    if (s != EP_OK) return s;
+    if (d.T == 0) return EP_OK;
+    if (!topk_w || !out || !aligned_to(topk_w, 4) || !aligned_to(out, 16)) return EP_ERR_INVALID_ARG;
+    PeerRows pr;
+    fill_rows(peers, d.R, &pr);
+    const int nvec = d.H / 8;
+    const int part = row_part(d.T, nvec);
+    const dim3 grid(d.T, (nvec + part - 1) / part);
+    int per, threads;
+    pick_shape(part, &per, &threads);
+    cudaStream_t st = (cudaStream_t)stream;
+#define EPB_PEER_COMB(C)                                                                                             \
+    launch_pdl(k_combine_peers<C>, grid, dim3(threads), 0, st, pr, topk_w, h->ws.dest_row, h->ws.rank_off, d.R, d.K,   \
+               nvec, part, (uint4 *)out)
+    const cudaError_t err =
+        per == 1 ? EPB_PEER_COMB(1) : per == 2 ? EPB_PEER_COMB(2) : per == 4 ? EPB_PEER_COMB(4) : EPB_PEER_COMB(8);
+#undef EPB_PEER_COMB
+    return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+// ---- CUDA IPC ---------------------------------------------------------------
+
+typedef int (*mem_range_fn)(uintptr_t *base, size_t *size, uintptr_t ptr);
+
+ep_status_t ep_ipc_export(const void *dev_ptr, uint8_t handle[64], int64_t *offset) {
+    if (!dev_ptr || !handle || !offset) return EP_ERR_INVALID_ARG;
+    // the allocation's base, from the driver (cuMemGetAddressRange)
+    static mem_range_fn range = nullptr;
+    if (!range) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return EP_ERR_CUDA;
+        range = (mem_range_fn)fn;
+    }
+    uintptr_t base = 0;
+    size_t size = 0;
+    if (range(&base, &size, (uintptr_t)dev_ptr) != 0) return EP_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t hd;
+    if (cudaIpcGetMemHandle(&hd, (void *)base) != cudaSuccess) {
+        cudaGetLastError();
+        return EP_ERR_CUDA;
+    }
+    static_assert(sizeof(cudaIpcMemHandle_t) == 64, "a CUDA IPC handle is 64 bytes");
+    memcpy(handle, &hd, 64);
+    *offset = (int64_t)((uintptr_t)dev_ptr - base);
+    return EP_OK;
+}
+
+ep_status_t ep_ipc_import(const uint8_t handle[64], int64_t offset, void **dev_ptr, void **base) {
+    if (!handle || !dev_ptr || !base || offset < 0) return EP_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t hd;
+    memcpy(&hd, handle, 64);
+    void *b = nullptr;
+    if (cudaIpcOpenMemHandle(&b, hd, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+        cudaGetLastError();
+        return EP_ERR_CUDA;
+    }
+    *base = b;
+    *dev_ptr = (char *)b + offset;
+    return EP_OK;
+}
+
+ep_status_t ep_ipc_close(void *base) {
+    if (!base) return EP_ERR_INVALID_ARG;
+    return cudaIpcCloseMemHandle(base) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+} // extern "C"

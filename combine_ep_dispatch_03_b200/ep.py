@@ -40,6 +40,22 @@ class EpConfig(ctypes.Structure):
     ]
 
 
+MAX_PEERS = 64  # EP_MAX_PEERS
+
+
+class EpPeerTable(ctypes.Structure):
+    """ep_peer_table_t: every rank's receive arrays as device addresses."""
+    _fields_ = [
+        ("num_ranks", ctypes.c_int32),
+        ("capacity_rows", ctypes.c_int64),
+        ("recv_x", ctypes.c_void_p * MAX_PEERS),
+        ("recv_scales", ctypes.c_void_p * MAX_PEERS),
+        ("recv_w", ctypes.c_void_p * MAX_PEERS),
+        ("recv_expert", ctypes.c_void_p * MAX_PEERS),
+        ("flags", ctypes.c_void_p * MAX_PEERS),
+    ]
+
+
 class EpError(RuntimeError):
     def __init__(self, call: str, status: int):
         self.status = status
@@ -71,6 +87,17 @@ SIGNATURES = {
     "ep_get_status": (ctypes.c_int, [_P, ctypes.POINTER(_I32), _P]),
     "ep_get_tensor": (ctypes.c_int, [_P, ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(_I64)]),
     "ep_route_noalloc": (ctypes.c_int, [_P, _I32, _I32, _I32, _P, _P, _P, _P]),
+    "ep_world_recv_rows": (ctypes.c_int, [_CFG, ctypes.POINTER(_I64)]),
+    "ep_plan_local_counts": (ctypes.c_int, [_P, _P, _P, _P]),
+    "ep_plan_world": (ctypes.c_int, [_P, _P, _I32, _P]),
+    "ep_dispatch_peers": (ctypes.c_int, [_P, _P, _P, _P, ctypes.POINTER(EpPeerTable), _P]),
+    "ep_signal_peers": (ctypes.c_int, [_P, ctypes.POINTER(EpPeerTable), ctypes.c_uint32, _P]),
+    "ep_wait_peers": (ctypes.c_int, [_P, _P, ctypes.c_uint32, _I64, _P]),
+    "ep_combine_peers": (ctypes.c_int, [_P, ctypes.POINTER(EpPeerTable), _P, _P, _P]),
+    "ep_ipc_export": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint8 * 64), ctypes.POINTER(_I64)]),
+    "ep_ipc_import": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint8 * 64), _I64, ctypes.POINTER(_P),
+                                     ctypes.POINTER(_P)]),
+    "ep_ipc_close": (ctypes.c_int, [_P]),
     "ep_router_topk": (ctypes.c_int, [_P, _I32, _I32, _I32, _P, _P, _P]),
 }
 
@@ -175,6 +202,64 @@ def route_noalloc(topk_idx: torch.Tensor, num_experts: int, dest_row: torch.Tens
         _ptr(dest_row, torch.int32, T * K, "dest_row"), _ptr(expert_counts, torch.int32, num_experts,
                                                              "expert_counts"),
         _ptr(flags, torch.int32, 1, "flags"), _stream(stream)))
+
+
+def world_recv_rows(cfg: EpConfig) -> int:
+    """Rows one rank's receive buffer needs in a world of cfg.num_ranks GPUs."""
+    rows = ctypes.c_int64()
+    _check("ep_world_recv_rows", lib().ep_world_recv_rows(ctypes.byref(cfg), ctypes.byref(rows)))
+    return rows.value
+
+
+def _addr(t) -> int | None:
+    """Device address of a CUDA tensor, or an int address as it is (peer
+    buffers mapped through IPC have no tensor), or None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("peer buffers must be contiguous CUDA tensors or device addresses")
+    return t.data_ptr()
+
+
+def peer_table(capacity_rows: int, recv_x, flags, recv_scales=None, recv_w=None, recv_expert=None) -> EpPeerTable:
+    """An ep_peer_table_t from per-rank lists (entry r: rank r's buffer, a CUDA
+    tensor or a device address; the optional lists may be None)."""
+    R = len(recv_x)
+    if R > MAX_PEERS:
+        raise ValueError(f"at most {MAX_PEERS} ranks")
+    tab = EpPeerTable()
+    tab.num_ranks = R
+    tab.capacity_rows = capacity_rows
+    for r in range(R):
+        tab.recv_x[r] = _addr(recv_x[r])
+        tab.flags[r] = _addr(flags[r]) if flags is not None else None
+        tab.recv_scales[r] = _addr(recv_scales[r]) if recv_scales is not None else None
+        tab.recv_w[r] = _addr(recv_w[r]) if recv_w is not None else None
+        tab.recv_expert[r] = _addr(recv_expert[r]) if recv_expert is not None else None
+    return tab
+
+
+def ipc_export(t: torch.Tensor) -> tuple[bytes, int]:
+    """(64-byte CUDA IPC handle of the allocation holding t, t's offset in it)."""
+    h = (ctypes.c_uint8 * 64)()
+    off = ctypes.c_int64()
+    _check("ep_ipc_export", lib().ep_ipc_export(ctypes.c_void_p(t.data_ptr()), ctypes.byref(h), ctypes.byref(off)))
+    return bytes(h), off.value
+
+
+def ipc_import(handle: bytes, offset: int) -> tuple[int, int]:
+    """Map a peer's exported buffer: (device address of the buffer, mapping
+    base to pass to ipc_close)."""
+    h = (ctypes.c_uint8 * 64).from_buffer_copy(handle)
+    p, base = ctypes.c_void_p(), ctypes.c_void_p()
+    _check("ep_ipc_import", lib().ep_ipc_import(ctypes.byref(h), offset, ctypes.byref(p), ctypes.byref(base)))
+    return p.value, base.value
+
+
+def ipc_close(base: int) -> None:
+    _check("ep_ipc_close", lib().ep_ipc_close(ctypes.c_void_p(base)))
 
 
 class _DeviceArray:
@@ -297,6 +382,38 @@ class Ep:
             raise ValueError("prefetch_slots must hold R*S rows of one expert's weights")
         _check("ep_prefetch_replica_weights", lib().ep_prefetch_replica_weights(
             self._h, self._p(expert_weights), nbytes, self._p(prefetch_slots), _stream(stream)))
+
+    # -- expert parallelism across GPUs (one rank per GPU; see include/ep.h)
+    def plan_local_counts(self, topk_idx, counts, stream=None) -> None:
+        """This rank's routed pairs per expert into counts (int32 [E])."""
+        _check("ep_plan_local_counts", lib().ep_plan_local_counts(
+            self._h, self._p(topk_idx, torch.int32, self.T * self.K, "topk_idx"),
+            self._p(counts, torch.int32, self.E, "counts"), _stream(stream)))
+
+    def plan_world(self, world_counts, rank: int, stream=None) -> None:
+        """The world's plan from every rank's counts (int32 [R, E], rank order)."""
+        _check("ep_plan_world", lib().ep_plan_world(
+            self._h, self._p(world_counts, torch.int32, self.R * self.E, "world_counts"), rank, _stream(stream)))
+
+    def dispatch_peers(self, x, topk_idx, topk_w, table: EpPeerTable, stream=None) -> None:
+        _check("ep_dispatch_peers", lib().ep_dispatch_peers(
+            self._h, self._p(x, torch.bfloat16, self.T * self.H, "x"),
+            self._p(topk_idx, torch.int32, self.T * self.K, "topk_idx"),
+            self._p(topk_w, torch.float32, self.T * self.K, "topk_w"), ctypes.byref(table), _stream(stream)))
+
+    def signal_peers(self, table: EpPeerTable, epoch: int, stream=None) -> None:
+        _check("ep_signal_peers", lib().ep_signal_peers(self._h, ctypes.byref(table), epoch, _stream(stream)))
+
+    def wait_peers(self, flags, epoch: int, timeout_us: int = 0, stream=None) -> None:
+        """Wait (bounded) until every source has signalled `epoch` into flags
+        (this rank's uint32 [R], given as an int32 CUDA tensor)."""
+        _check("ep_wait_peers", lib().ep_wait_peers(
+            self._h, self._p(flags, torch.int32, self.R, "flags"), epoch, timeout_us, _stream(stream)))
+
+    def combine_peers(self, table: EpPeerTable, topk_w, out, stream=None) -> None:
+        _check("ep_combine_peers", lib().ep_combine_peers(
+            self._h, ctypes.byref(table), self._p(topk_w, torch.float32, self.T * self.K, "topk_w"),
+            self._p(out, torch.bfloat16, self.T * self.H, "out"), _stream(stream)))
 
     # -- inspection
     def get_plan(self, stream=None) -> tuple[list[int], list[int]]:

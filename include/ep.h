@@ -140,8 +140,9 @@ ep_status_t ep_output_shape(const ep_config_t *cfg, int64_t dims[4], int32_t *nd
 ep_status_t ep_workspace_bytes(const ep_config_t *cfg, size_t *bytes);
 
 /* Number of kernels one ep_plan launches for this configuration: one for
- * batches of up to 1024 (token, k) pairs without a balanced plan, and for
- * up to 32768 pairs when the current device can hold the routing cluster
+ * batches of up to 1024 (token, k) pairs (with a balanced plan, when its
+ * tables and the batch fit one CTA's shared memory), and for up to 32768
+ * pairs without a plan when the current device can hold the routing cluster
  * (asked of the device; reported as not holdable where there is no GPU),
  * else three. Every other data call launches one kernel. */
 ep_status_t ep_plan_kernel_count(const ep_config_t *cfg, int32_t *count);
@@ -280,6 +281,116 @@ ep_status_t ep_get_status(ep_handle_t *h, int32_t *flags, void *stream);
 /* Read-only device pointer and element count of one piece of the handle's
  * routing state (valid until the next ep_plan or ep_destroy). */
 ep_status_t ep_get_tensor(const ep_handle_t *h, ep_tensor_t which, const void **dptr, int64_t *numel);
+
+/* ---- expert parallelism across GPUs: one rank per GPU ------------------
+ *
+ * The same path with the R ranks of the EP world on R GPUs (NVLink 5 through
+ * NVSwitch), or, for testing, on one GPU with R separate receive buffers. The
+ * steps follow the pages' statement of the exchange:
+ *   - counts:  every rank counts its own routed pairs per expert
+ *              (ep_plan_local_counts); the caller all-gathers the R count rows
+ *              (R*E int32, e.g. one NCCL all-gather) into world_counts;
+ *   - plan:    every rank derives the same global layout from world_counts,
+ *              and the global row of each of its own pairs (ep_plan_world);
+ *              the stable order of an expert's rows is (source rank, t, k),
+ *              so rank r's pairs of expert e follow the pairs of ranks < r;
+ *   - send:    rows go straight into the owning rank's receive buffer
+ *              (ep_dispatch_peers: NCCL EP Table II / Fig. 2, the send half of
+ *              the staged mode; MoonEP article para. 4, placement straight into
+ *              expert-grouped remote positions with no staging copy);
+ *   - signal / wait: per-source completion flags (ep_signal_peers,
+ *              ep_wait_peers: the receive half of the staged mode);
+ *   - combine: each rank reads its tokens' K rows from the ranks holding them
+ *              and reduces them locally (ep_combine_peers: NCCL EP Table III,
+ *              per-token reduction at the receiver).
+ * Remote rows move with plain 16-byte stores and loads in the library's own
+ * kernels (no bulk or multicast copies touch another GPU's memory).
+ *
+ * A handle for this mode is created with cfg.num_tokens = this rank's tokens
+ * (the same on every rank) and cfg.num_ranks = R, the number of GPUs; global
+ * row g of the world's receive buffer (the layout ep_plan gives for the
+ * concatenation of all ranks' tokens, rank order) belongs to the rank r with
+ * rank_offset[r] <= g < rank_offset[r+1], at local row g - rank_offset[r].
+ * After ep_plan_world the single-GPU data calls (ep_dispatch, ep_combine, the
+ * backward calls) refuse the handle with EP_ERR_UNSUPPORTED, and the peer
+ * calls refuse a handle planned by ep_plan.
+ */
+
+#define EP_MAX_PEERS 64
+
+/* Per-rank buffers of an EP world, as device addresses this GPU can reach
+ * (CUDA IPC or symmetric-memory mappings of the peers' buffers, or plain
+ * allocations on one GPU). Entry r belongs to rank r; unused arrays are NULL. */
+typedef struct ep_peer_table {
+    int32_t num_ranks;                   /* R, as in the handle's configuration */
+    int64_t capacity_rows;               /* rows of every rank's receive buffer */
+    void *recv_x[EP_MAX_PEERS];          /* [capacity_rows, H] bf16, or e4m3 bytes with fp8;
+                                            ep_combine_peers reads the expert outputs here */
+    float *recv_scales[EP_MAX_PEERS];    /* [capacity_rows, H/128] fp32 with fp8, else NULL */
+    float *recv_w[EP_MAX_PEERS];         /* [capacity_rows] fp32, or NULL */
+    int32_t *recv_expert[EP_MAX_PEERS];  /* [capacity_rows] int32, or NULL */
+    uint32_t *flags[EP_MAX_PEERS];       /* [R] uint32: rank r's completion flags, one per source rank */
+} ep_peer_table_t;
+
+/* Rows one rank's receive buffer must hold for any routing (host-only):
+ * LL (E/R)*ll_capacity; HT with a balanced plan ceil(L/R) for L = R*T*K pairs
+ * of the world (more only when the plan flags EP_FLAG_PLAN_SLOTS); HT without
+ * a plan L, since all pairs may route to one rank. */
+ep_status_t ep_world_recv_rows(const ep_config_t *cfg, int64_t *rows);
+
+/* Count this rank's routed pairs per expert: counts (device int32 [E]) as in
+ * EP_T_EXPERT_COUNTS, the same rules for masked, bad and repeated ids (the
+ * status word is cleared first). Keeps the per-tile ranks that ep_plan_world
+ * completes. Always the three-kernel routing path's first two kernels. */
+ep_status_t ep_plan_local_counts(ep_handle_t *h, const int32_t *topk_idx, int32_t *counts, void *stream);
+
+/* Complete the plan of this rank (`rank`, in [0, R)) from world_counts
+ * (device int32 [R, E], row r = rank r's ep_plan_local_counts output), after
+ * ep_plan_local_counts on the same handle and batch. Every rank computes the
+ * same layout (with cfg.balanced, the same balanced plan of the world's
+ * counts); EP_T_DEST_ROW then holds global rows, EP_T_RANK_OFFSET,
+ * EP_T_RANK_LOAD, EP_T_RECV_COUNTS, EP_T_REPLICA_EXPERT and
+ * EP_T_EXPERT_COUNTS describe the whole world, and EP_T_SRC_ROW is not kept.
+ * Counts inconsistent with the batch give unspecified rows (never an access
+ * outside the buffers: ep_dispatch_peers checks every row against
+ * capacity_rows). */
+ep_status_t ep_plan_world(ep_handle_t *h, const int32_t *world_counts, int32_t rank, void *stream);
+
+/* The send phase: for every routed pair (t,k) of this rank with global row g
+ * on rank r at local row l, the same values as ep_dispatch (bf16 copy, or the
+ * FP8 cast with its scales, recv_w, recv_expert) written to
+ * peers->recv_x[r] row l (and the other arrays likewise). A row at or beyond
+ * peers->capacity_rows is skipped and EP_FLAG_CAPACITY raised. */
+ep_status_t ep_dispatch_peers(ep_handle_t *h, const void *x, const int32_t *topk_idx, const float *topk_w,
+                              const ep_peer_table_t *peers, void *stream);
+
+/* After the kernels before it on `stream` (stream order), make their writes
+ * visible to the whole system and set peers->flags[r][rank] = epoch on every
+ * rank r, with release semantics. */
+ep_status_t ep_signal_peers(ep_handle_t *h, const ep_peer_table_t *peers, uint32_t epoch, void *stream);
+
+/* The receive phase: a kernel on `stream` waits until flags[s] (device
+ * uint32 [R], this rank's flags) has reached `epoch` for every source s
+ * (acquire semantics), so the kernels after it see every row the sources
+ * wrote before signalling. The wait is bounded: after timeout_us (0 = 2 s)
+ * it gives up, sets EP_FLAG_WAIT_TIMEOUT in the status word and returns. */
+ep_status_t ep_wait_peers(ep_handle_t *h, const uint32_t *flags, uint32_t epoch, int64_t timeout_us,
+                          void *stream);
+
+/* Combine across ranks: out[t] as ep_combine computes it, each pair's row
+ * read from peers->recv_x[r] at local row l (the expert outputs of rank r,
+ * bf16). out: device bf16 [T, H] of this rank's tokens. */
+ep_status_t ep_combine_peers(ep_handle_t *h, const ep_peer_table_t *peers, const float *topk_w, void *out,
+                             void *stream);
+
+/* CUDA IPC of one device buffer, for building a peer table across processes:
+ * export gives a 64-byte handle of the allocation holding dev_ptr and the
+ * pointer's offset inside it; import maps a peer's allocation into this
+ * process (with peer access enabled) and returns the address at that offset
+ * and the mapping's base (to release with ep_ipc_close). */
+ep_status_t ep_ipc_export(const void *dev_ptr, uint8_t handle[64], int64_t *offset);
+ep_status_t ep_ipc_import(const uint8_t handle[64], int64_t offset, void **dev_ptr, void **base);
+ep_status_t ep_ipc_close(void *base);
 
 /* ---- routing without allocation ---------------------------------------- */
 

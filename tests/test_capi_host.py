@@ -102,8 +102,10 @@ def test_output_shape(L):
 @pytest.mark.parametrize("kw,count", [
     (dict(T=100, E=256, K=8, R=8), 1),            # 800 pairs: one CTA
     (dict(T=32768, E=256, K=8, R=8), 3),          # 262144 pairs: three kernels
+    (dict(T=100, E=256, K=8, R=8, balanced=True), 1),    # 800 pairs with a plan: one CTA
+    (dict(T=128, E=256, K=8, R=8, balanced=True), 1),    # 1024 pairs: the largest one-CTA plan
+    (dict(T=129, E=256, K=8, R=8, balanced=True), 3),
     (dict(T=1024, E=256, K=8, R=8, balanced=True), 3),
-    (dict(T=100, E=256, K=8, R=8, balanced=True), 3),
 ])
 def test_plan_kernel_count(L, kw, count):
     """Counts that do not depend on the device (the cluster path, 1025 to

@@ -160,6 +160,25 @@ def test_routing_shape_boundaries(T, K):
     assert r["flags"] == 0
 
 
+@pytest.mark.parametrize("T,K,E,R,direct", [(128, 8, 256, 8, False), (129, 8, 256, 8, False),
+                                             (128, 8, 256, 8, True), (1024, 1, 64, 4, False),
+                                             (1025, 1, 64, 4, True), (300, 3, 384, 16, False)])
+def test_balanced_plan_shape_boundaries(T, K, E, R, direct):
+    """The balanced plan is built inside the one-CTA routing kernel up to
+    1024 pairs and by the three-kernel path beyond: both sides of the switch,
+    with skewed routing, training and inference plans (two slots a rank for
+    the inference plan), forward and backward with the replica reduce."""
+    g = _gc()
+    h = ep.Ep(T, 128, E, K, R, balanced=True, replica_slots=2 if direct else 0, direct_overflow=direct)
+    assert ep.plan_launches(h) == (1 if T * K <= 1024 else 3)
+    h.close()
+    r = g.run_forward(T, 128, E, K, R, balanced=True, slots=2 if direct else 0, direct=direct, zipf_s=1.0,
+                      seed=T + K, G=0 if direct else 256)
+    assert r["flags"] == 0
+    if not direct:
+        g.run_backward(r, seed=T)
+
+
 @pytest.mark.parametrize("T,H,fp8", [(1000, 7176, False), (1000, 7296, True), (300, 2056, False),
                                       (64, 20480, False), (64, 40960, True)])
 def test_rows_split_across_ctas(T, H, fp8):
