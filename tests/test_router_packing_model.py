@@ -13,8 +13,10 @@ unchosen lane head agrees there with the last chosen word.
 This is a numpy model of that selection and of its two votes. On inputs
 built to trip the packing (exact ties, logits that differ only in their low
 mantissa bits, signed zeros), every token where the packed choice differs
-from the oracle's top-K must be one the votes flag. It is a check of the
-argument, not of the CUDA code; the GPU parity tests check the kernel."""
+from the oracle's top-K must be one the votes flag. The same holds for the
+four-lanes-per-token form (K <= 8), whose second check compares the last
+choice with the largest unchosen word. These check the argument, not the CUDA
+code; the GPU parity tests check the kernel."""
 import numpy as np
 import pytest
 
@@ -102,6 +104,61 @@ def test_unflagged_choices_on_plain_logits_match_and_flags_are_rare(E, K, most):
     flags = 0
     for t in range(T):
         got, flagged = _packed_selection(logits[t], K)
+        flags += flagged
+        if not flagged:
+            assert got == want[t].tolist()
+    assert flags <= most * T
+
+
+def _lanes_selection(v, K):
+    """(chosen ids, flagged) as the four-lanes-per-token kernel sees a token
+    (K <= 8, E a multiple of 16): the K largest packed words are chosen (its
+    sorts and merges select them exactly), and a token is flagged when two
+    chosen words, or the last chosen word and the largest unchosen one (the
+    (K+1)-th largest word, which the merges carry along), agree above the low
+    bits."""
+    E = len(v)
+    epl = 1
+    while 32 * epl < E:
+        epl *= 2
+    M = (1 << _ID_BITS[epl]) - 1
+    keys = _order_keys(v)
+    words = sorted(((int(keys[e]) & ~M) | (M - e) for e in range(E)), reverse=True)
+    chosen = words[:K]
+    unchosen = words[K] if K < E else 0
+    high = ~M
+    flagged = any((chosen[j] ^ chosen[j + 1]) & high == 0 for j in range(K - 1))
+    flagged |= (chosen[-1] ^ unchosen) & high == 0
+    return [M - (m & M) for m in chosen], flagged
+
+
+def test_every_wrong_lanes_choice_is_flagged():
+    oracle.build()
+    rng = np.random.default_rng(13)
+    flagged_needed = 0
+    for v, K in _cases(rng, 900):
+        E = len(v) - len(v) % 16
+        if E < 16:
+            continue
+        v, K = v[:E], min(K, 8)
+        want = oracle.router_topk(v[None, :], K)[0][0].tolist()
+        got, flagged = _lanes_selection(v, K)
+        if got != want:
+            assert flagged, (v.tolist(), K, got, want)
+            flagged_needed += 1
+    assert flagged_needed > 0
+
+
+@pytest.mark.parametrize("E,K,most", [(256, 8, 0.02), (128, 8, 0.02), (384, 8, 0.02), (1024, 8, 0.05)])
+def test_lanes_flags_are_rare_on_plain_logits(E, K, most):
+    oracle.build()
+    rng = np.random.default_rng(E + 7 * K)
+    T = 200
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    want = oracle.router_topk(logits, K)[0]
+    flags = 0
+    for t in range(T):
+        got, flagged = _lanes_selection(logits[t], K)
         flags += flagged
         if not flagged:
             assert got == want[t].tolist()

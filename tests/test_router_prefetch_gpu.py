@@ -61,6 +61,12 @@ def _check_router(logits, K):
     (50, 1024, 32, 0.5),    # the largest E and K
     (64, 8, 8, 0.0),        # K = E
     (37, 33, 1, 0.0),       # K = 1, one lane holds two experts
+    # four lanes a token (K <= 8, E a multiple of 16): a last warp with fewer
+    # than 8 tokens, an odd count of 16-byte vectors a lane, K < 8, E = 1024
+    (1001, 48, 3, 0.0),
+    (777, 1024, 8, 0.0),
+    (513, 64, 1, 0.5),
+    (9, 16, 8, 0.0),
 ])
 def test_router_topk_parity(T, E, K, s):
     _check_router(synth.router_logits(T, E, zipf_s=s, seed=T + E + K), K)
@@ -72,7 +78,7 @@ def test_router_topk_ties():
     _check_router(logits.contiguous(), 8)
 
 
-@pytest.mark.parametrize("T,E,K", [(3000, 256, 8), (200, 1024, 32), (500, 40, 5)])
+@pytest.mark.parametrize("T,E,K", [(3000, 256, 8), (200, 1024, 32), (500, 40, 5), (300, 1024, 8), (257, 48, 6)])
 def test_router_topk_near_ties(T, E, K):
     """Each token's logits agree in all but their lowest 11 mantissa bits: the
     choices and their order must follow the full fp32 values."""
