@@ -101,12 +101,13 @@ def code_sha(paths) -> str:
 
 
 def committed_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current code of the kernel's sources (else None)."""
+    """DRAM bytes per launch from the committed ncu summary of this kernel on
+    this workload ("kernel@workload"), if it was taken on the current code of
+    the kernel's sources (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
-            rec = json.load(f)[kernel]
+            rec = json.load(f)[f"{kernel}@{workload}"]
         if code_sha(rec["sources"]) != rec["code_sha"] or rec["workload"] != workload:
             return None
         return int(rec["dram_bytes_per_launch"])

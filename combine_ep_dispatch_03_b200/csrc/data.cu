@@ -106,10 +106,15 @@ __global__ void __launch_bounds__(32) k_dispatch_bulk(const uint8_t *__restrict_
 // One thread owns 16 consecutive elements (two 16-byte loads, one 16-byte
 // store); the 8 threads of a 128-block are 8 consecutive lanes.
 // ---------------------------------------------------------------------------
-// At least 5 CTAs per SM (48 registers): measured faster than the unbounded
-// 64-register build (HT prefill step 1016 -> 1011 us).
+// At least 5 CTAs per SM (48 registers) for up to two chunks a thread:
+// measured faster than the unbounded 64-register build (HT prefill step
+// 1016 -> 1011 us). Four and eight chunks a thread (rows of more than 8192
+// elements) hold 2-4x the data in registers and would spill under that bound;
+// they take 3 and 2 CTAs per SM.
+constexpr int fp8_min_ctas(int cpt) { return cpt <= 2 ? 5 : cpt == 4 ? 3 : 2; }
+
 template <int CPT>
-__global__ void __launch_bounds__(256, 5) k_dispatch_fp8(const uint4 *__restrict__ x, const int32_t *__restrict__ idx,
+__global__ void __launch_bounds__(256, fp8_min_ctas(CPT)) k_dispatch_fp8(const uint4 *__restrict__ x, const int32_t *__restrict__ idx,
                                                       const float *__restrict__ w,
                                                       const int32_t *__restrict__ dest_row, int K, int nchunk,
                                                       int part, uint4 *__restrict__ recv, float *__restrict__ scales,
