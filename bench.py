@@ -455,6 +455,147 @@ class Step:
         return plan_launches(self.h) + len(self.calls) - 1
 
 
+class WorldStep:
+    """One pass of the path across ranks through the peer table (ep_plan_local_counts,
+    the gathered counts, ep_plan_world, ep_dispatch_peers, signal and wait,
+    ep_combine_peers). With one process the workload's R ranks are R handles
+    with R separate buffers on this GPU, run in stream order (every wait finds
+    flags that earlier kernels set); with N processes (N = R GPUs) each process
+    is one rank, the counts are all-gathered with NCCL and the peers' buffers
+    are mapped through CUDA IPC."""
+
+    def __init__(self, wl: dict, dev, seed: int, world: int, rank: int):
+        import torch
+
+        from combine_ep_dispatch_03_b200 import ep, synth
+        from combine_ep_dispatch_03_b200 import world as wmod
+
+        self.wl, self.kind, self.h = wl, "world", None
+        T, H, E, K, R = wl["T"], wl["H"], wl["E"], wl["K"], wl["R"]
+        self.T, self.H, self.E, self.K, self.R = T, H, E, K, R
+        self.multi = world > 1
+        if self.multi and world != R:
+            raise ValueError(f"--exchange across GPUs needs --gpus equal to the workload's R ({R})")
+        Tl = T // R
+        x = synth.tokens_bf16(T, H, seed=seed)
+        idx, w = synth.routing(T, E, K, zipf_s=wl["s"], seed=seed)
+        mine = [rank] if self.multi else list(range(R))
+        self.hs = {q: ep.Ep(Tl, H, E, K, R, mode=wl["mode"], ll_capacity=wl["cap"], fp8=wl["fp8"],
+                            balanced=wl["balanced"], replica_slots=wl.get("slots", 0),
+                            direct_overflow=wl.get("direct", False)) for q in mine}
+        cap = ep.world_recv_rows(next(iter(self.hs.values())).cfg)
+        self.cap = cap
+        self.xs = {q: x[q * Tl:(q + 1) * Tl].to(dev) for q in mine}
+        self.ids = {q: idx[q * Tl:(q + 1) * Tl].contiguous().to(dev) for q in mine}
+        self.ws = {q: w[q * Tl:(q + 1) * Tl].contiguous().to(dev) for q in mine}
+        dt = torch.float8_e4m3fn if wl["fp8"] else torch.bfloat16
+        g = torch.Generator(device=dev).manual_seed(2000 + seed)
+        own = {}
+        for q in mine:
+            own[q] = {"recv_x": torch.empty((cap, H), dtype=dt, device=dev),
+                      "recv_scales": torch.empty((cap, H // 128), dtype=torch.float32, device=dev) if wl["fp8"] else None,
+                      "recv_w": torch.empty(cap, dtype=torch.float32, device=dev),
+                      "recv_expert": torch.empty(cap, dtype=torch.int32, device=dev),
+                      "flags": torch.zeros(R, dtype=torch.int32, device=dev)}
+            # the expert-FFN output stand-in of rank q, resident (not timed)
+            own[q]["y"] = torch.randn((cap, H), generator=g, device=dev).to(torch.bfloat16)
+        self.own = own
+        self.bases = []
+        if self.multi:
+            handles = wmod.exchange_handles(wmod.export_buffers({k: v for k, v in own[rank].items()}))
+            self.table, b1 = wmod.peer_table_from_handles(rank, own[rank], handles, cap)
+            ytab_own = {"recv_x": own[rank]["y"], "flags": own[rank]["flags"]}
+            yh = [{"recv_x": h["y"], "flags": h["flags"]} for h in handles]
+            self.ytable, b2 = wmod.peer_table_from_handles(rank, ytab_own, yh, cap)
+            self.bases = b1 + b2
+        else:
+            col = lambda k: [own[q][k] for q in range(R)]
+            self.table = ep.peer_table(cap, col("recv_x"), col("flags"), col("recv_scales") if wl["fp8"] else None,
+                                       col("recv_w"), col("recv_expert"))
+            self.ytable = ep.peer_table(cap, col("y"), col("flags"))
+        self.counts = torch.zeros((R, E), dtype=torch.int32, device=dev)
+        self.local = torch.zeros(E, dtype=torch.int32, device=dev)
+        self.outs = {q: torch.empty((Tl, H), dtype=torch.bfloat16, device=dev) for q in mine}
+        self.epoch = 0
+        self.mine = mine
+        self.rank = rank
+        self.calls = [("plan", self._plan), ("dispatch", self._dispatch), ("combine", self._combine)]
+        self.outputs = list(self.outs.values())
+
+    def _plan(self, st):
+        from combine_ep_dispatch_03_b200 import world as wmod
+
+        if self.multi:
+            h = self.hs[self.rank]
+            h.plan_local_counts(self.ids[self.rank], self.local, st)
+            import torch
+
+            with torch.cuda.stream(st):
+                self.counts.copy_(wmod.gather_counts(self.local))
+            h.plan_world(self.counts, self.rank, st)
+        else:
+            for q in self.mine:
+                self.hs[q].plan_local_counts(self.ids[q], self.counts[q], st)
+            for q in self.mine:
+                self.hs[q].plan_world(self.counts, q, st)
+
+    def _exchange(self, table, st):
+        self.epoch += 1
+        for q in self.mine:
+            self.hs[q].signal_peers(table, self.epoch, st)
+        for q in self.mine:
+            self.hs[q].wait_peers(self.own[q]["flags"], self.epoch, 0, st)
+
+    def _dispatch(self, st):
+        for q in self.mine:
+            self.hs[q].dispatch_peers(self.xs[q], self.ids[q], self.ws[q], self.table, st)
+        self._exchange(self.table, st)
+
+    def _combine(self, st):
+        self._exchange(self.table, st)  # every rank's expert outputs are ready
+        for q in self.mine:
+            self.hs[q].combine_peers(self.ytable, self.ws[q], self.outs[q], st)
+
+    def run(self, st):
+        for _, f in self.calls:
+            f(st)
+
+    def measure_bytes(self, st):
+        """The same algorithmic bytes as the single-GPU step of this workload
+        (this process's share with one rank per GPU)."""
+        self.run(st)
+        st.synchronize()
+        from combine_ep_dispatch_03_b200 import ep
+
+        T, H, K = self.T, self.H, self.K
+        placed = 0
+        for q in self.mine:
+            dest = self.hs[q].tensor(ep.T_DEST_ROW)
+            placed += int((dest >= 0).sum().item())
+        share = len(self.mine) / self.R
+        b = algorithmic_bytes(int(T * share), H, K, placed, self.wl["fp8"])
+        self.bytes, self.placed = b, placed
+        return b
+
+    def launches(self):
+        per_rank = 2 + 2 + 1 + 2 + 2 + 1  # counts (2), world plan (2), dispatch, signal+wait, signal+wait, combine
+        return per_rank * len(self.mine)
+
+    def status(self, st):
+        f = 0
+        for h in self.hs.values():
+            f |= h.status(st)
+        return f
+
+    def close(self):
+        from combine_ep_dispatch_03_b200 import ep
+
+        for b in self.bases:
+            ep.ipc_close(b)
+        for h in self.hs.values():
+            h.close()
+
+
 L2_FALLBACK_BYTES = 126 * 2**20
 
 
@@ -615,6 +756,8 @@ def run_native(args):
     if args.weight_bytes:
         wl["wbytes"] = args.weight_bytes
     name = args.workload if wl == WORKLOADS[args.workload] else args.workload + "_custom"
+    if args.exchange:
+        return run_exchange(args, wl, name, rank, world, dev, stream)
     seed = rank  # each rank: its own EP world (weak scaling)
     step = Step(wl, dev, seed)
     nbytes = step.measure_bytes(stream)
@@ -688,6 +831,59 @@ def run_native(args):
         result["workloads"] = run_side_workloads(dev, stream, seed, peak, world, args.no_graph)
     if world == 1 and rank == 0 and not args.no_cpu_baseline and args.workload == "ht_prefill":
         result["cpu_baseline"] = cpu_baseline(args.cpu_sample_tokens)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def run_exchange(args, wl, name, rank, world, dev, stream):
+    """--exchange: the path across ranks through the peer table (WorldStep).
+    Stream launches (the flags' epochs change every step), no L2 flush (the
+    workloads it serves move far more than L2). With N GPUs the whole job is
+    one EP world of N ranks, so the total work is fixed ("strong")."""
+    import torch
+
+    step = WorldStep(wl, dev, 0, world, rank)
+    nbytes = step.measure_bytes(stream)
+    step_bytes = sum(nbytes.values())
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    t0 = time.time()
+    total_ms, per = timed(step, args.steps, args.warmup, stream, min(args.steps, 20), graph=False)
+    t1 = time.time()
+    sampler.stop()
+    barrier(world)
+    ms_local = total_ms / args.steps
+    ms = max_over_ranks(ms_local, world)
+    total_bytes = step_bytes * (world if step.multi else 1)
+    value = total_bytes / (ms * 1e-3) / 1e9
+    peak, _ = hbm_peak()
+    avg = {k: sum(v) / len(v) for k, v in per.items()}
+    flags = step.status(stream)
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "strong" if step.multi else "weak", "vs_baseline": None, "dtype": compute_dtype(wl),
+        "data": "synthetic", "impl": "native-exchange",
+        "config": dict(workload_config(name, wl, world, l2_note_for(step_bytes, l2_bytes(dev), False)),
+                       parallelism=(f"one EP world of {world} GPUs (one rank each), peer stores and loads"
+                                    if step.multi else
+                                    f"{wl['R']} ranks as separate buffers on one GPU, peer-table path")),
+        "launch": "stream",
+        "tokens_per_s": round(wl["T"] / (ms * 1e-3), 1),
+        "frac_of_hbm": round(value / max(world, 1) / peak, 4),
+        "per_call_us": {k: round(v * 1e3, 2) for k, v in avg.items()},
+        "per_call_note": "per call over all of this process's ranks, including the signal and wait kernels",
+        "bytes_per_step": total_bytes, "capacity_rows_per_rank": step.cap,
+        "gpu_launches": step.launches() * args.steps, "clocks": sampler.window(t0, t1), "device_flags": flags,
+    }
+    step.close()
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -986,6 +1182,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side", action="store_true", help="skip the other workloads' sub-records")
+    ap.add_argument("--exchange", action="store_true",
+                    help="the path across ranks through the peer table: the workload's R ranks as separate buffers "
+                         "on one GPU, or one rank per GPU with --gpus R")
     ap.add_argument("--cpu-sample-tokens", type=int, default=32768)
     args = ap.parse_args()
     if args.warmup < 3:
