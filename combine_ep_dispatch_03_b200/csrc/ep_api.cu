@@ -73,14 +73,15 @@ ep_status_t derive_dims(const ep_config_t *c, Dims *d) {
     d->nhist = (d->ntiles + kRouteWarps - 1) / kRouteWarps;
     const int64_t per_cta = (int64_t)kRouteThreads * kAssignPer; // pairs per assignment CTA
     d->nassign = (int)(L > 0 ? (L + per_cta - 1) / per_cta : 1);
-    // cluster routing: plain layouts and at most kClusterMaxPairs pairs
-    // (measured faster than the three-kernel path there, slower beyond). The
+    // cluster routing: at most kClusterMaxPairs pairs (measured faster than
+    // the three-kernel path there, slower beyond); with a balanced plan, CTA 0
+    // of the cluster runs the planner between two cluster barriers. The
     // cluster shape keeps each warp near 64 pairs with as few warps per SM as
     // that allows, since the warp votes of the first pass issue slowly when
     // every warp of an SM votes. Step times measured per shape: 8192 pairs,
     // 8 CTAs x 16 warps 48.5 us (x 32 warps 49.0); 16384 pairs, 16 x 16
     // 53.5 us (8 x 32 54.9); 32768 pairs, 16 x 32 105.6 us (16 x 16 106.5).
-    if (!c->balanced && L <= kClusterMaxPairs) {
+    if (L <= kClusterMaxPairs) {
         const int cs = L > 8192 ? 16 : 8, cw = L > 16384 ? 32 : 16;
         const int64_t ppw = ((L + (int64_t)cs * cw - 1) / ((int64_t)cs * cw) + 31) / 32 * 32;
         d->cl_size = cs;

@@ -124,9 +124,11 @@ __device__ __forceinline__ uint32_t block_or(uint32_t v, uint32_t *s_acc) {
 }
 
 // Exclusive scan of a[0..n) in shared memory by the whole block; returns the
-// total. s_warp needs 33 ints. Every thread of the block must call it.
+// total. s_warp needs 32 ints. Every thread of the block must call it. Two
+// barriers: after the warps' totals are stored, every warp scans the 32
+// totals itself (instead of one warp scanning them behind a third barrier).
 __device__ int block_exscan(int32_t *a, int n, int32_t *s_warp) {
-    const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, w = tid >> 5;
+    const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, w = tid >> 5, nw = nth >> 5;
     const int per = (n + nth - 1) / nth;
     const int lo = min(n, tid * per), hi = min(n, lo + per);
     int sum = 0;
@@ -139,27 +141,22 @@ __device__ int block_exscan(int32_t *a, int n, int32_t *s_warp) {
     }
     if (lane == 31) s_warp[w] = incl;
     __syncthreads();
-    if (w == 0) {
-        const int nw = nth >> 5;
-        const int v = lane < nw ? s_warp[lane] : 0;
-        int inc = v;
+    const int v = lane < nw ? s_warp[lane] : 0;
+    int inc = v;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int u = __shfl_up_sync(kFull, inc, o);
-            if (lane >= o) inc += u;
-        }
-        if (lane < nw) s_warp[lane] = inc - v;
-        if (lane == 31) s_warp[32] = inc;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc += u;
     }
-    __syncthreads();
-    int run = s_warp[w] + incl - sum;
+    const int wbase = __shfl_sync(kFull, inc - v, w); // totals of the warps before this one
+    const int total = __shfl_sync(kFull, inc, 31);
+    int run = wbase + incl - sum;
     for (int i = lo; i < hi; ++i) {
-        const int v = a[i];
+        const int x = a[i];
         a[i] = run;
-        run += v;
+        run += x;
     }
-    const int total = s_warp[32];
-    __syncthreads();
+    __syncthreads(); // a[] is complete, and s_warp may be reused
     return total;
 }
 
@@ -277,8 +274,7 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     int32_t *s_D = s_pn + E;                  // [R] deficits, then loads
     int32_t *s_nrep = s_D + R;                // [R]
     int32_t *s_recv = s_nrep + R;             // [R] receivers in visiting order
-    int32_t *s_roff = s_recv + R;             // [R+1]
-    int32_t *s_dn = s_roff + R + 1;           // [R] direct pieces per rank
+    int32_t *s_dn = s_recv + R;               // [R] direct pieces per rank
     int32_t *s_dsum = s_dn + R;               // [R] rows in direct pieces per rank
     int32_t *s_dbase = s_dsum + R;            // [R] own + slot rows per rank
     int32_t *s_slot_e = s_dbase + R;          // [R*S]
@@ -293,12 +289,11 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     int32_t *s_x_aux = s_x_slot + NX;         // [NX] direct: rows before it among the rank's direct rows
     int32_t *s_A = s_x_aux + NX;              // [E+1] first spilled row of each spilled expert (fill order)
     int32_t *s_B = s_A + E + 1;               // [R+1] first deficit row of each receiver (visiting order)
-    __shared__ int s_L, s_nrecv, s_seq;
+    int32_t *s_seg = s_B + R + 1;             // [R + 2E + R*S]: the scans of the fill and of the tables
+    __shared__ int s_nrecv, s_seq;
+    __shared__ int s_wsum[32];
 
-    if (tid == 0) {
-        s_L = 0;
-        s_nrecv = 0;
-    }
+    if (tid == 0) s_nrecv = 0;
     for (int i = tid; i < R * S; i += nth) {
         s_slot_e[i] = -1;
         s_slot_len[i] = 0;
@@ -310,7 +305,6 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     }
     if (d.direct)
         for (int i = tid; i < R * E; i += nth) ws.direct_expert[i] = -1;
-    __syncthreads();
     int part = 0;
     for (int e = tid; e < E; e += nth) {
         s_tail[e] = 0;
@@ -319,9 +313,11 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
         part += s_cnt[e];
     }
     part = __reduce_add_sync(kFull, part);
-    if ((tid & 31) == 0) atomicAdd(&s_L, part);
+    if ((tid & 31) == 0) s_wsum[tid >> 5] = part;
     __syncthreads();
-    const int L = s_L, q = L / R, rem = L % R;
+    int L = 0;
+    for (int w = 0; w < (nth >> 5); ++w) L += s_wsum[w];
+    const int q = L / R, rem = L % R;
 
     // keep: rows of the experts visited before e on its rank (sorted order)
     for (int e = tid; e < E; e += nth) {
@@ -375,18 +371,22 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     // piece's slot is its expert's position minus that of the expert holding
     // p's first deficit row. If some receiver would need more than S slots
     // (and overflow is not served directly) the walk below runs instead.
-    for (int i = tid; i < nsp; i += nth) s_A[i] = s_cnt[s_list[i]] - s_keep[s_list[i]];
-    for (int i = tid; i < s_nrecv; i += nth) s_B[i] = s_D[s_recv[i]];
+    // one scan over [spilled rows of each spilled expert | deficits of each
+    // receiver]: the first part's prefixes are the experts' first spilled rows
+    // (and its end the spilled total); the second part, less that total, the
+    // receivers' first deficit rows
+    const int nrecv_all = s_nrecv;
+    for (int i = tid; i < nsp; i += nth) s_seg[i] = s_cnt[s_list[i]] - s_keep[s_list[i]];
+    for (int i = tid; i < nrecv_all; i += nth) s_seg[nsp + i] = s_D[s_recv[i]];
     if (tid == 0) s_seq = 0;
     __syncthreads();
-    const int nrecv_all = s_nrecv;
-    const int spill_total = block_exscan(s_A, nsp, s_warp);
-    block_exscan(s_B, nrecv_all, s_warp);
-    if (tid == 0) {
-        s_A[nsp] = spill_total;
-        s_B[nrecv_all] = spill_total; // the deficits add up to the spilled rows
-    }
-    __syncthreads();
+    block_exscan(s_seg, nsp + nrecv_all, s_warp);
+    const int spill_total = s_seg[nsp];
+    s_A = s_seg; // [nsp + 1]: s_A[nsp] is the spilled total
+    // receiver q's first deficit row, read in place; the deficits add up to
+    // the spilled rows, so the one past the last receiver is the spilled total
+    const int32_t *s_Bs = s_seg + nsp;
+    auto Bv = [&](int q) { return q < nrecv_all ? s_Bs[q] - spill_total : spill_total; };
     // the last index i in [0, n) with a[i] <= v (a ascending, a[0] <= v)
     auto last_le = [](const int32_t *a, int n, int v) {
         int lo = 0, hi = n - 1;
@@ -396,11 +396,20 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
         }
         return lo;
     };
+    // the same over the receivers' first deficit rows
+    auto last_le_B = [&](int v) {
+        int lo = 0, hi = nrecv_all - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (Bv(mid) <= v) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    };
     for (int i = tid; i < nsp; i += nth) { // pass 1: pieces per expert, slot check
         const int a0 = s_A[i], a1 = s_A[i + 1];
         int n = 0;
-        for (int q = last_le(s_B, nrecv_all, a0); q < nrecv_all && s_B[q] < a1; ++q, ++n) {
-            const int slot = i - last_le(s_A, nsp, s_B[q]);
+        for (int q = last_le_B(a0); q < nrecv_all && Bv(q) < a1; ++q, ++n) {
+            const int slot = i - last_le(s_A, nsp, Bv(q));
             if (slot >= S && !d.direct) s_seq = 1;
         }
         s_spill[i] = n; // s_spill is free again: pieces of the i-th expert in fill order
@@ -414,10 +423,10 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
             for (int i2 = 0; i2 < i; ++i2) x += s_spill[i2]; // pieces of earlier experts
             s_pfirst[e] = x;
             s_pn[e] = s_spill[i];
-            for (int q = last_le(s_B, nrecv_all, a0); q < nrecv_all && s_B[q] < a1; ++q, ++x) {
+            for (int q = last_le_B(a0); q < nrecv_all && Bv(q) < a1; ++q, ++x) {
                 const int r = s_recv[q];
-                const int lo = max(a0, s_B[q]), hi = min(a1, s_B[q + 1]);
-                const int fe = last_le(s_A, nsp, s_B[q]);
+                const int lo = max(a0, Bv(q)), hi = min(a1, Bv(q + 1));
+                const int fe = last_le(s_A, nsp, Bv(q));
                 const int slot = i - fe;
                 s_x_start[x] = s_keep[e] + (lo - a0);
                 s_x_len[x] = hi - lo;
@@ -427,7 +436,7 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
                     s_slot_e[r * S + slot] = e;
                     s_slot_len[r * S + slot] = hi - lo;
                 } else { // direct piece slot - S of rank r
-                    const int first_direct_row = min(s_B[q + 1], s_A[fe + S]);
+                    const int first_direct_row = min(Bv(q + 1), s_A[fe + S]);
                     s_x_slot[x] = -3;
                     s_x_aux[x] = lo - first_direct_row;
                     ws.direct_expert[(int64_t)r * E + slot - S] = e;
@@ -438,11 +447,11 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
         }
         for (int q = tid; q < nrecv_all; q += nth) { // per receiver: slots and direct rows used
             const int r = s_recv[q];
-            const int fe = last_le(s_A, nsp, s_B[q]), le = last_le(s_A, nsp, s_B[q + 1] - 1);
+            const int fe = last_le(s_A, nsp, Bv(q)), le = last_le(s_A, nsp, Bv(q + 1) - 1);
             const int npc = le - fe + 1;
             s_nrep[r] = min(S, npc);
             s_dn[r] = max(0, npc - S);
-            s_dsum[r] = npc > S ? s_B[q + 1] - s_A[fe + S] : 0;
+            s_dsum[r] = npc > S ? Bv(q + 1) - s_A[fe + S] : 0;
             s_D[r] = 0;
         }
     }
@@ -453,64 +462,67 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     // suffices; with direct overflow a receiver out of slots still qualifies
     // and takes the rows as a direct piece). Pieces go to shared memory in
     // creation order.
-    if (tid == 0 && s_seq) {
-        const int nrecv = s_nrecv;
-        int p = 0, nx = 0;
-        uint32_t fl = 0;
-        for (int i = 0; i < nsp; ++i) {
-            const int e = s_list[i], owner = e / g;
-            int left = s_cnt[e] - s_keep[e], next = s_keep[e];
-            s_pfirst[e] = nx;
-            while (left > 0) {
-                while (p < nrecv && (s_D[s_recv[p]] == 0 || (!d.direct && s_nrep[s_recv[p]] >= S))) ++p;
-                if (p == nrecv) {
-                    s_tail[e] = left;
+    if (s_seq) { // uniform: set in pass 1, read after its barrier
+        if (tid == 0) {
+            const int nrecv = s_nrecv;
+            int p = 0, nx = 0;
+            uint32_t fl = 0;
+            for (int i = 0; i < nsp; ++i) {
+                const int e = s_list[i], owner = e / g;
+                int left = s_cnt[e] - s_keep[e], next = s_keep[e];
+                s_pfirst[e] = nx;
+                while (left > 0) {
+                    while (p < nrecv && (s_D[s_recv[p]] == 0 || (!d.direct && s_nrep[s_recv[p]] >= S))) ++p;
+                    if (p == nrecv) {
+                        s_tail[e] = left;
+                        s_x_start[nx] = next;
+                        s_x_len[nx] = left;
+                        s_x_rank[nx] = owner;
+                        s_x_slot[nx] = -2;
+                        ++nx;
+                        fl |= EP_FLAG_PLAN_SLOTS;
+                        break;
+                    }
+                    const int r = s_recv[p];
+                    const int give = min(left, s_D[r]);
                     s_x_start[nx] = next;
-                    s_x_len[nx] = left;
-                    s_x_rank[nx] = owner;
-                    s_x_slot[nx] = -2;
+                    s_x_len[nx] = give;
+                    s_x_rank[nx] = r;
+                    if (s_nrep[r] < S) {
+                        const int sl = s_nrep[r]++;
+                        s_slot_e[r * S + sl] = e;
+                        s_slot_len[r * S + sl] = give;
+                        s_x_slot[nx] = sl;
+                    } else { // a direct piece (direct overflow only)
+                        const int di = s_dn[r]++;
+                        ws.direct_expert[(int64_t)r * E + di] = e;
+                        ws.direct_start[(int64_t)r * E + di] = next;
+                        ws.direct_len[(int64_t)r * E + di] = give;
+                        s_x_slot[nx] = -3;
+                        s_x_aux[nx] = s_dsum[r];
+                        s_dsum[r] += give;
+                    }
                     ++nx;
-                    fl |= EP_FLAG_PLAN_SLOTS;
-                    break;
+                    s_D[r] -= give;
+                    left -= give;
+                    next += give;
                 }
-                const int r = s_recv[p];
-                const int give = min(left, s_D[r]);
-                s_x_start[nx] = next;
-                s_x_len[nx] = give;
-                s_x_rank[nx] = r;
-                if (s_nrep[r] < S) {
-                    const int sl = s_nrep[r]++;
-                    s_slot_e[r * S + sl] = e;
-                    s_slot_len[r * S + sl] = give;
-                    s_x_slot[nx] = sl;
-                } else { // a direct piece (direct overflow only)
-                    const int di = s_dn[r]++;
-                    ws.direct_expert[(int64_t)r * E + di] = e;
-                    ws.direct_start[(int64_t)r * E + di] = next;
-                    ws.direct_len[(int64_t)r * E + di] = give;
-                    s_x_slot[nx] = -3;
-                    s_x_aux[nx] = s_dsum[r];
-                    s_dsum[r] += give;
-                }
-                ++nx;
-                s_D[r] -= give;
-                left -= give;
-                next += give;
+                s_pn[e] = nx - s_pfirst[e];
             }
-            s_pn[e] = nx - s_pfirst[e];
+            if (fl) atomicOr(s_fl, fl);
         }
-        if (fl) atomicOr(s_fl, fl);
+        __syncthreads();
     }
-    __syncthreads();
 
-    // layout inside each rank region: own experts, replica slots, direct pieces
-    for (int e = tid; e < E; e += nth) s_own[e] = s_keep[e] + s_tail[e];
-    __syncthreads();
+    // layout inside each rank region (a thread per rank): own experts, replica
+    // slots, direct pieces; and, for the one scan that follows, each expert's
+    // extra pieces, whether it has replicas, and which slots are filled
+    int32_t *q_roff = s_seg, *q_x = s_seg + R, *q_rep = q_x + E, *q_slot = q_rep + E;
     for (int r = tid; r < R; r += nth) {
         int run = 0;
         int32_t *rc = ws.recv_counts + (int64_t)r * (g + S);
         for (int i = 0; i < g; ++i) {
-            const int e = r * g + i, v = s_own[e];
+            const int e = r * g + i, v = s_keep[e] + s_tail[e];
             rc[i] = v;
             s_own[e] = run;
             run += v;
@@ -524,41 +536,57 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
         s_dbase[r] = run;
         run += s_dsum[r];
         if (d.direct) ws.direct_n[r] = s_dn[r];
-        s_roff[r] = run;
+        q_roff[r] = run;
         ws.rank_load[r] = run;
     }
+    for (int e = tid; e < E; e += nth) {
+        const int f = s_pfirst[e], n = s_pn[e];
+        int nrep = 0;
+        for (int i = 0; i < n; ++i) nrep += s_x_slot[f + i] >= 0 ? 1 : 0;
+        q_x[e] = n;
+        q_rep[e] = nrep > 0 ? 1 : 0;
+    }
+    for (int i = tid; i < R * S; i += nth) q_slot[i] = s_slot_e[i] >= 0 ? 1 : 0;
     __syncthreads();
-    const int total = block_exscan(s_roff, R, s_warp);
-    for (int r = tid; r < R; r += nth) ws.rank_off[r] = s_roff[r];
-    if (tid == 0) ws.rank_off[R] = total;
-    for (int i = tid; i < R * S; i += nth) ws.replica_expert[i] = s_slot_e[i];
-    for (int e = tid; e < E; e += nth) s_list[e] = s_pn[e];
-    __syncthreads();
-    const int nxt = block_exscan(s_list, E, s_warp); // s_list[e] = first compact extra piece of e (id order)
-    if (tid == 0) ws.xoff[E] = nxt;
-
+    // one scan over [rank loads | extra pieces | has replicas | filled slots];
+    // each part's prefixes are then relative to its first element's
+    const int grand = block_exscan(s_seg, R + 2 * E + R * S, s_warp);
+    const int rows_total = q_x[0], xb = q_x[0], rb = q_rep[0], sb = q_slot[0];
+    for (int r = tid; r < R; r += nth) ws.rank_off[r] = q_roff[r];
+    if (tid == 0) {
+        ws.rank_off[R] = rows_total;
+        ws.xoff[E] = rb - xb;
+        *ws.red_count = sb - rb;
+        *ws.slot_count = grand - sb;
+    }
+    // the filled replica slots, ascending (the prefetch copies only these)
+    for (int i = tid; i < R * S; i += nth) {
+        ws.replica_expert[i] = s_slot_e[i];
+        if (s_slot_e[i] >= 0) ws.slot_list[q_slot[i] - sb] = i;
+    }
     // piece 0, the compact extra pieces, and the per-expert replica lists
     // (slots r*S+s in ascending order: each entry's place is the number of
     // the expert's slot pieces with a smaller key)
     for (int e = tid; e < E; e += nth) {
         const int owner = e / g;
-        const int own_base = s_roff[owner] + s_own[e];
+        const int own_base = q_roff[owner] + s_own[e];
+        const int xo = q_x[e] - xb;
         ws.base0[e] = own_base;
         ws.len0[e] = s_keep[e];
-        ws.xoff[e] = s_list[e];
+        ws.xoff[e] = xo;
         const int f = s_pfirst[e], n = s_pn[e];
         int nrep = 0;
         for (int i = 0; i < n; ++i) {
             const int x = f + i, r = s_x_rank[x], sl = s_x_slot[x];
-            const int o = s_list[e] + i;
+            const int o = xo + i;
             ws.xstart[o] = s_x_start[x];
             ws.xlen[o] = s_x_len[x];
             if (sl == -2) {
                 ws.xdst[o] = own_base + s_keep[e];
             } else if (sl == -3) { // direct piece: no slot, no gradient to reduce
-                ws.xdst[o] = s_roff[r] + s_dbase[r] + s_x_aux[x];
+                ws.xdst[o] = q_roff[r] + s_dbase[r] + s_x_aux[x];
             } else {
-                ws.xdst[o] = s_roff[r] + s_slot_off[r * S + sl];
+                ws.xdst[o] = q_roff[r] + s_slot_off[r * S + sl];
                 const int key = r * S + sl;
                 int pos = 0;
                 for (int i2 = 0; i2 < n; ++i2) {
@@ -570,24 +598,8 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
             }
         }
         ws.red_n[e] = nrep;
-        s_pn[e] = nrep; // reused below as "has replicas"
+        if (nrep > 0) ws.red_experts[q_rep[e] - rb] = e;
     }
-    __syncthreads();
-    for (int e = tid; e < E; e += nth) s_list[e] = s_pn[e] > 0 ? 1 : 0;
-    __syncthreads();
-    const int nred = block_exscan(s_list, E, s_warp);
-    for (int e = tid; e < E; e += nth)
-        if (s_pn[e] > 0) ws.red_experts[s_list[e]] = e;
-    if (tid == 0) *ws.red_count = nred;
-    __syncthreads();
-    // the filled replica slots, ascending (the prefetch copies only these);
-    // s_slot_len is free again and serves as the flag array
-    for (int i = tid; i < R * S; i += nth) s_slot_len[i] = s_slot_e[i] >= 0 ? 1 : 0;
-    __syncthreads();
-    const int nslot = block_exscan(s_slot_len, R * S, s_warp);
-    for (int i = tid; i < R * S; i += nth)
-        if (s_slot_e[i] >= 0) ws.slot_list[s_slot_len[i]] = i;
-    if (tid == 0) *ws.slot_count = nslot;
     __syncthreads();
 }
 
@@ -993,21 +1005,61 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     }
     __syncthreads();
 
-    // 3. layout (every CTA computes it; CTA 0 publishes it) and assignment
-    const int total = plain_tables(d, s_cnt, s_len, s_off, s_warp, &s_fl);
+    if (!d.balanced) {
+        // 3. layout (every CTA computes it; CTA 0 publishes it) and assignment
+        const int total = plain_tables(d, s_cnt, s_len, s_off, s_warp, &s_fl);
+        if (r == 0) {
+            plain_outputs(d, ws, s_len, s_off, total);
+            for (int e = tid; e < E; e += blockDim.x) ws.cnt[e] = s_cnt[e];
+            __syncthreads();
+            if (tid == 0) *ws.flags = s_fl;
+        }
+        for (int i = lo + lane; i < hi; i += 32) {
+            const int pk = s_pk[i];
+            const int e = pk & 0xffff;
+            int dest = -1;
+            if (e != 0xffff) {
+                const int j = s_cta[e] + my[e] + (pk >> 16);
+                if (j < s_len[e]) dest = s_off[e] + j;
+            }
+            ws.dest_row[c0 + i] = dest;
+            if (dest >= 0 && ws.src_row) ws.src_row[dest] = (int32_t)(c0 + i);
+        }
+        return;
+    }
+    // 3'. balanced plan: CTA 0 builds it from the totals every CTA now holds and
+    // writes its tables to the workspace; the cluster barrier (release /
+    // acquire at cluster scope) makes them visible to every CTA, which then
+    // assigns its own pairs through them
     if (r == 0) {
-        plain_outputs(d, ws, s_len, s_off, total);
+        layout_balanced(d, ws, s_cnt, s_pk + ppc, s_warp, &s_fl); // scratch: after the pair arrays
         for (int e = tid; e < E; e += blockDim.x) ws.cnt[e] = s_cnt[e];
         __syncthreads();
         if (tid == 0) *ws.flags = s_fl;
     }
+    cluster.sync();
+    for (int e = tid; e < E; e += blockDim.x) {
+        s_len[e] = __ldcg(ws.len0 + e);
+        s_off[e] = __ldcg(ws.base0 + e);
+    }
+    __syncthreads();
     for (int i = lo + lane; i < hi; i += 32) {
         const int pk = s_pk[i];
         const int e = pk & 0xffff;
         int dest = -1;
         if (e != 0xffff) {
             const int j = s_cta[e] + my[e] + (pk >> 16);
-            if (j < s_len[e]) dest = s_off[e] + j;
+            if (j < s_len[e]) {
+                dest = s_off[e] + j;
+            } else {
+                for (int x = __ldcg(ws.xoff + e), xe = __ldcg(ws.xoff + e + 1); x < xe; ++x) {
+                    const int xs = __ldcg(ws.xstart + x), xl = __ldcg(ws.xlen + x);
+                    if (j >= xs && j < xs + xl) {
+                        dest = __ldcg(ws.xdst + x) + (j - xs);
+                        break;
+                    }
+                }
+            }
         }
         ws.dest_row[c0 + i] = dest;
         if (dest >= 0 && ws.src_row) ws.src_row[dest] = (int32_t)(c0 + i);
@@ -1088,7 +1140,9 @@ __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__
 size_t route_smem_layout(const Dims &d) {
     if (!d.balanced) return 0;
     const size_t E = d.E, R = d.R, S = d.S, NX = d.nx_max;
-    return sizeof(int32_t) * (E + 7 * E + 7 * R + 1 + 3 * R * S + 5 * NX + E + 1 + R + 1);
+    // s_cnt (callers), 7 E-arrays, 6 R-arrays, 3 slot arrays, 5 piece arrays,
+    // s_A, s_B, and the scans' buffer
+    return sizeof(int32_t) * (E + 7 * E + 6 * R + 3 * R * S + 5 * NX + E + 1 + R + 1 + (R + 2 * E + R * S));
 }
 
 size_t route_smem_assign(const Dims &d) {
@@ -1108,7 +1162,9 @@ size_t route_smem_small(const Dims &d) {
 }
 
 size_t route_smem_cluster(const Dims &d) {
-    return sizeof(int32_t) * ((size_t)(d.cl_warps + 4 + d.cl_size) * d.E + 2 * (size_t)d.cl_ppw * d.cl_warps);
+    // with a plan, the planner's scratch follows the pair arrays (CTA 0 uses it)
+    return sizeof(int32_t) * ((size_t)(d.cl_warps + 4 + d.cl_size) * d.E + 2 * (size_t)d.cl_ppw * d.cl_warps) +
+           route_smem_layout(d);
 }
 
 // Can a cluster of d.cl_size CTAs of this kernel be resident at once on this
@@ -1147,7 +1203,7 @@ static bool cluster_fits(const Dims &d) {
 }
 
 bool route_use_cluster(const Dims &d) {
-    return !d.balanced && d.cl_size > 0 && d.L > kSmallMaxPairs && cluster_fits(d);
+    return d.cl_size > 0 && d.L > (d.balanced ? kSmallMaxPlanPairs : kSmallMaxPairs) && cluster_fits(d);
 }
 
 bool route_use_small(const Dims &d) {

@@ -142,9 +142,9 @@ ep_status_t ep_workspace_bytes(const ep_config_t *cfg, size_t *bytes);
 /* Number of kernels one ep_plan launches for this configuration: one for
  * batches of up to 1024 (token, k) pairs (with a balanced plan, when its
  * tables and the batch fit one CTA's shared memory), and for up to 32768
- * pairs without a plan when the current device can hold the routing cluster
- * (asked of the device; reported as not holdable where there is no GPU),
- * else three. Every other data call launches one kernel. */
+ * pairs, with or without a plan, when the current device can hold the
+ * routing cluster (asked of the device; reported as not holdable where there
+ * is no GPU), else three. Every other data call launches one kernel. */
 ep_status_t ep_plan_kernel_count(const ep_config_t *cfg, int32_t *count);
 
 /* "major.minor.patch" of the library. */

@@ -162,15 +162,20 @@ def test_routing_shape_boundaries(T, K):
 
 @pytest.mark.parametrize("T,K,E,R,direct", [(128, 8, 256, 8, False), (129, 8, 256, 8, False),
                                              (128, 8, 256, 8, True), (1024, 1, 64, 4, False),
-                                             (1025, 1, 64, 4, True), (300, 3, 384, 16, False)])
+                                             (1025, 1, 64, 4, True), (300, 3, 384, 16, False),
+                                             (1024, 8, 256, 8, True), (2048, 8, 384, 16, False),
+                                             (4096, 8, 256, 8, False), (4097, 8, 256, 8, False),
+                                             (4097, 8, 128, 8, True)])
 def test_balanced_plan_shape_boundaries(T, K, E, R, direct):
     """The balanced plan is built inside the one-CTA routing kernel up to
-    1024 pairs and by the three-kernel path beyond: both sides of the switch,
-    with skewed routing, training and inference plans (two slots a rank for
-    the inference plan), forward and backward with the replica reduce."""
+    1024 pairs, by CTA 0 of the one-launch routing cluster up to 32768 pairs
+    (between two cluster barriers), and by the three-kernel path beyond: both
+    sides of each switch, with skewed routing, training and inference plans
+    (two slots a rank for the inference plan), forward and backward with the
+    replica reduce."""
     g = _gc()
     h = ep.Ep(T, 128, E, K, R, balanced=True, replica_slots=2 if direct else 0, direct_overflow=direct)
-    assert ep.plan_launches(h) == (1 if T * K <= 1024 else 3)
+    assert ep.plan_launches(h) == (1 if T * K <= 32768 else 3)
     h.close()
     r = g.run_forward(T, 128, E, K, R, balanced=True, slots=2 if direct else 0, direct=direct, zipf_s=1.0,
                       seed=T + K, G=0 if direct else 256)
