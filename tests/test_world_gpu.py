@@ -232,3 +232,36 @@ def test_wait_gives_up_on_flags_nobody_sets():
     assert h.status() == 0
     assert s.elapsed_time(e) < 40.0
     h.close()
+
+
+def test_world_empty_batches():
+    """Ranks with no tokens: counts of zero, an empty plan, and dispatch and
+    combine calls that launch nothing and succeed."""
+    dev = torch.device("cuda")
+    R, E, K, H = 2, 8, 2, 128
+    hs = [ep.Ep(0, H, E, K, R) for _ in range(R)]
+    cap = ep.world_recv_rows(hs[0].cfg)
+    assert cap == 0
+    counts = torch.full((R, E), 7, dtype=torch.int32, device=dev)
+    ids = torch.empty((0, K), dtype=torch.int32, device=dev)
+    x = torch.empty((0, H), dtype=torch.bfloat16, device=dev)
+    w = torch.empty((0, K), dtype=torch.float32, device=dev)
+    bufs = [torch.zeros((1, H), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    flags = [torch.zeros(R, dtype=torch.int32, device=dev) for _ in range(R)]
+    table = ep.peer_table(cap, bufs, flags)
+    for q in range(R):
+        hs[q].plan_local_counts(ids, counts[q])
+    for q in range(R):
+        hs[q].plan_world(counts, q)
+        hs[q].dispatch_peers(x, ids, w, table)
+        hs[q].signal_peers(table, 3)
+    for q in range(R):
+        hs[q].wait_peers(flags[q], 3, timeout_us=1_000_000)
+        hs[q].combine_peers(table, w, torch.empty((0, H), dtype=torch.bfloat16, device=dev))
+    torch.cuda.synchronize()
+    assert (counts == 0).all()
+    for q in range(R):
+        assert hs[q].status() == 0
+        assert (flags[q] == 3).all()
+        np.testing.assert_array_equal(hs[q].tensor(ep.T_RANK_OFFSET).cpu().numpy(), np.zeros(R + 1))
+        hs[q].close()
