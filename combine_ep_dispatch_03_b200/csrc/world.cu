@@ -76,8 +76,10 @@ __device__ __forceinline__ void stage_peer_rows(const int32_t *__restrict__ dest
 }
 
 // dispatch send, bf16 rows: one CTA per (token, row part), VPT 16-byte vectors
-// a thread; the token's vectors are read once and stored K times.
-template <int VPT>
+// a thread; the token's vectors are read once and stored K times. SCALE (the
+// combine backward across ranks): each row is bf16(w[t,k] * x[t]) instead,
+// one fp32 product and one rounding, and no weights or ids are recorded.
+template <int VPT, bool SCALE>
 __global__ void __launch_bounds__(256) k_dispatch_peers(const uint4 *__restrict__ x, const int32_t *__restrict__ idx,
                                                         const float *__restrict__ w,
                                                         const int32_t *__restrict__ dest_row,
@@ -87,6 +89,7 @@ __global__ void __launch_bounds__(256) k_dispatch_peers(const uint4 *__restrict_
     __shared__ int s_rank[kMaxTopk];
     __shared__ int64_t s_lrow[kMaxTopk];
     __shared__ uint4 *s_dst[kMaxTopk];
+    __shared__ float s_wk[kMaxTopk];
     const int t = blockIdx.x;
     const int64_t pb = (int64_t)t * K;
     const int cb = blockIdx.y * part, n = min(part, nvec - cb);
@@ -101,7 +104,9 @@ __global__ void __launch_bounds__(256) k_dispatch_peers(const uint4 *__restrict_
         const int r = s_rank[threadIdx.x];
         const int64_t lr = s_lrow[threadIdx.x];
         s_dst[threadIdx.x] = r >= 0 ? reinterpret_cast<uint4 *>(pr.x[r]) + lr * nvec + cb : nullptr;
-        if (r >= 0 && blockIdx.y == 0) {
+        if (SCALE) {
+            s_wk[threadIdx.x] = w[pb + threadIdx.x];
+        } else if (r >= 0 && blockIdx.y == 0) {
             if (pr.w[r]) pr.w[r][lr] = w[pb + threadIdx.x];
             if (pr.expert[r]) pr.expert[r][lr] = idx[pb + threadIdx.x];
         }
@@ -112,10 +117,20 @@ __global__ void __launch_bounds__(256) k_dispatch_peers(const uint4 *__restrict_
         for (int k = 0; k < K; ++k) {
             uint4 *dst = s_dst[k];
             if (!dst) continue;
+            const float wk = SCALE ? s_wk[k] : 1.0f;
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 const int c = c0 + threadIdx.x + i * blockDim.x;
-                if (c < n) dst[c] = v[i];
+                if (c >= n) continue;
+                if (SCALE) {
+                    float f[8];
+                    unpack8(v[i], f);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) f[u] = __fmul_rn(wk, f[u]);
+                    dst[c] = pack8(f);
+                } else {
+                    dst[c] = v[i];
+                }
             }
         }
     }
@@ -182,8 +197,9 @@ __global__ void __launch_bounds__(256) k_dispatch_peers_fp8(const uint4 *__restr
 }
 
 // combine across ranks: out[t] = bf16(fold_k fmaf(w[t,k], y_k, acc)) with y_k
-// the pair's row in its rank's expert outputs, k in order, acc from +0.
-template <int CPT>
+// the pair's row in its rank's expert outputs, k in order, acc from +0. UNIT
+// (the dispatch backward across ranks): an unweighted fp32 sum in k order.
+template <int CPT, bool UNIT>
 __global__ void __launch_bounds__(256) k_combine_peers(PeerRows pr, const float *__restrict__ w,
                                                        const int32_t *__restrict__ dest_row,
                                                        const int32_t *__restrict__ rank_off, int R, int K, int nvec,
@@ -202,7 +218,7 @@ __global__ void __launch_bounds__(256) k_combine_peers(PeerRows pr, const float 
         const int r = s_rank[threadIdx.x];
         s_src[threadIdx.x] =
             r >= 0 ? reinterpret_cast<const uint4 *>(pr.x[r]) + s_lrow[threadIdx.x] * nvec + cb : nullptr;
-        s_w[threadIdx.x] = w[pb + threadIdx.x];
+        s_w[threadIdx.x] = UNIT ? 1.0f : w[pb + threadIdx.x];
     }
     __syncthreads();
     const int step = CPT * blockDim.x;
@@ -228,12 +244,75 @@ __global__ void __launch_bounds__(256) k_combine_peers(PeerRows pr, const float 
                     if (k >= K || !s_src[k]) continue;
                     float f[8];
                     unpack8(v[kk], f);
-                    const float wk = s_w[k];
+                    if (UNIT) {
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) acc[u] = __fmaf_rn(wk, f[u], acc[u]);
+                        for (int u = 0; u < 8; ++u) acc[u] = __fadd_rn(acc[u], f[u]);
+                    } else {
+                        const float wk = s_w[k];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) acc[u] = __fmaf_rn(wk, f[u], acc[u]);
+                    }
                 }
             }
             out[(int64_t)t * nvec + cb + c] = pack8(acc);
+        }
+    }
+}
+
+// replica-gradient reduce across ranks: this rank (own experts [e0, e0 + g))
+// adds, for each of its experts with replicas, the replica slots' gradients in
+// ascending slot order (each read from the slot's rank through the table) to
+// its own owner rows (fp32, in place). A persistent grid over (replicated
+// expert, 4096-element chunk) items; experts of other ranks are skipped.
+struct PeerGrads {
+    const float4 *rep[EP_MAX_PEERS]; // rank r's replica gradients [S, G] fp32
+};
+
+constexpr int kRedPeerThreads = 256, kRedPeerUnroll = 4;
+
+__global__ void __launch_bounds__(kRedPeerThreads) k_reduce_peers(PeerGrads pg, float4 *__restrict__ owner,
+                                                                  const int32_t *__restrict__ red_experts,
+                                                                  const int32_t *__restrict__ red_count,
+                                                                  const int32_t *__restrict__ red_list,
+                                                                  const int32_t *__restrict__ red_n, int R, int S,
+                                                                  int e0, int g, int64_t G4) {
+    pdl_wait();
+    const int nred = *red_count;
+    const int64_t chunk = (int64_t)kRedPeerThreads * kRedPeerUnroll;
+    const int per = (int)((G4 + chunk - 1) / chunk); // chunks per expert (host-checked to fit)
+    const int items = nred * per;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+        const int e = red_experts[it / per];
+        if (e < e0 || e >= e0 + g) continue; // another rank's expert
+        const int64_t base = (int64_t)(it % per) * chunk + threadIdx.x;
+        const int n = red_n[e];
+        const int32_t *lst = red_list + (int64_t)e * R;
+        float4 *o = owner + (int64_t)(e - e0) * G4;
+        float4 acc[kRedPeerUnroll];
+#pragma unroll
+        for (int u = 0; u < kRedPeerUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kRedPeerThreads;
+            acc[u] = i < G4 ? o[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int a = 0; a < n; ++a) {
+            const int key = lst[a]; // r * S + s
+            const float4 *src = pg.rep[key / S] + (int64_t)(key % S) * G4;
+#pragma unroll
+            for (int u = 0; u < kRedPeerUnroll; ++u) {
+                const int64_t i = base + (int64_t)u * kRedPeerThreads;
+                if (i < G4) {
+                    const float4 v = src[i];
+                    acc[u].x = __fadd_rn(acc[u].x, v.x);
+                    acc[u].y = __fadd_rn(acc[u].y, v.y);
+                    acc[u].z = __fadd_rn(acc[u].z, v.z);
+                    acc[u].w = __fadd_rn(acc[u].w, v.w);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kRedPeerUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kRedPeerThreads;
+            if (i < G4) o[i] = acc[u];
         }
     }
 }
@@ -386,8 +465,8 @@ ep_status_t ep_dispatch_peers(ep_handle_t *h, const void *x, const int32_t *topk
         const dim3 grid(d.T, (nvec + part - 1) / part);
         pick_shape(part, &per, &threads);
 #define EPB_PEER_BF16(V)                                                                                             \
-    launch_pdl(k_dispatch_peers<V>, grid, dim3(threads), 0, st, (const uint4 *)x, topk_idx, topk_w, h->ws.dest_row,   \
-               h->ws.rank_off, d.R, d.K, nvec, part, pr, h->ws.flags)
+    launch_pdl(k_dispatch_peers<V, false>, grid, dim3(threads), 0, st, (const uint4 *)x, topk_idx, topk_w,             \
+               h->ws.dest_row, h->ws.rank_off, d.R, d.K, nvec, part, pr, h->ws.flags)
         err = per == 1 ? EPB_PEER_BF16(1) : per == 2 ? EPB_PEER_BF16(2) : per == 4 ? EPB_PEER_BF16(4) : EPB_PEER_BF16(8);
 #undef EPB_PEER_BF16
     }
@@ -437,11 +516,93 @@ ep_status_t ep_combine_peers(ep_handle_t *h, const ep_peer_table_t *peers, const
     pick_shape(part, &per, &threads);
     cudaStream_t st = (cudaStream_t)stream;
 #define EPB_PEER_COMB(C)                                                                                             \
-    launch_pdl(k_combine_peers<C>, grid, dim3(threads), 0, st, pr, topk_w, h->ws.dest_row, h->ws.rank_off, d.R, d.K,   \
-               nvec, part, (uint4 *)out)
+    launch_pdl(k_combine_peers<C, false>, grid, dim3(threads), 0, st, pr, topk_w, h->ws.dest_row, h->ws.rank_off, d.R, \
+               d.K, nvec, part, (uint4 *)out)
     const cudaError_t err =
         per == 1 ? EPB_PEER_COMB(1) : per == 2 ? EPB_PEER_COMB(2) : per == 4 ? EPB_PEER_COMB(4) : EPB_PEER_COMB(8);
 #undef EPB_PEER_COMB
+    return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+ep_status_t ep_combine_backward_peers(ep_handle_t *h, const void *grad_out, const float *topk_w,
+                                      const ep_peer_table_t *grad_rows, void *stream) {
+    if (!h) return EP_ERR_INVALID_ARG;
+    if (h->planned != 2) return h->planned == 1 ? EP_ERR_UNSUPPORTED : EP_ERR_NOT_PLANNED;
+    const Dims &d = h->d;
+    ep_status_t s = check_table(h, grad_rows, true);
+    if (s != EP_OK) return s;
+    if (d.T == 0) return EP_OK;
+    if (!grad_out || !topk_w || !aligned_to(grad_out, 16) || !aligned_to(topk_w, 4)) return EP_ERR_INVALID_ARG;
+    PeerRows pr;
+    fill_rows(grad_rows, d.R, &pr);
+    for (int r = 0; r < d.R; ++r) { // gradient rows only: no weights, ids or scales recorded
+        pr.scales[r] = nullptr;
+        pr.w[r] = nullptr;
+        pr.expert[r] = nullptr;
+    }
+    const int nvec = d.H / 8;
+    const int part = row_part(d.T, nvec);
+    const dim3 grid(d.T, (nvec + part - 1) / part);
+    int per, threads;
+    pick_shape(part, &per, &threads);
+    cudaStream_t st = (cudaStream_t)stream;
+#define EPB_PEER_CBWD(V)                                                                                             \
+    launch_pdl(k_dispatch_peers<V, true>, grid, dim3(threads), 0, st, (const uint4 *)grad_out, (const int32_t *)nullptr,\
+               topk_w, h->ws.dest_row, h->ws.rank_off, d.R, d.K, nvec, part, pr, h->ws.flags)
+    const cudaError_t err =
+        per == 1 ? EPB_PEER_CBWD(1) : per == 2 ? EPB_PEER_CBWD(2) : per == 4 ? EPB_PEER_CBWD(4) : EPB_PEER_CBWD(8);
+#undef EPB_PEER_CBWD
+    return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+ep_status_t ep_dispatch_backward_peers(ep_handle_t *h, const ep_peer_table_t *grad_rows, void *grad_x,
+                                       void *stream) {
+    if (!h) return EP_ERR_INVALID_ARG;
+    if (h->planned != 2) return h->planned == 1 ? EP_ERR_UNSUPPORTED : EP_ERR_NOT_PLANNED;
+    const Dims &d = h->d;
+    ep_status_t s = check_table(h, grad_rows, true);
+    if (s != EP_OK) return s;
+    if (d.T == 0) return EP_OK;
+    if (!grad_x || !aligned_to(grad_x, 16)) return EP_ERR_INVALID_ARG;
+    PeerRows pr;
+    fill_rows(grad_rows, d.R, &pr);
+    const int nvec = d.H / 8;
+    const int part = row_part(d.T, nvec);
+    const dim3 grid(d.T, (nvec + part - 1) / part);
+    int per, threads;
+    pick_shape(part, &per, &threads);
+    cudaStream_t st = (cudaStream_t)stream;
+#define EPB_PEER_DBWD(C)                                                                                             \
+    launch_pdl(k_combine_peers<C, true>, grid, dim3(threads), 0, st, pr, (const float *)nullptr, h->ws.dest_row,      \
+               h->ws.rank_off, d.R, d.K, nvec, part, (uint4 *)grad_x)
+    const cudaError_t err =
+        per == 1 ? EPB_PEER_DBWD(1) : per == 2 ? EPB_PEER_DBWD(2) : per == 4 ? EPB_PEER_DBWD(4) : EPB_PEER_DBWD(8);
+#undef EPB_PEER_DBWD
+    return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+ep_status_t ep_reduce_replica_grads_peers(ep_handle_t *h, const ep_peer_table_t *replica_grads, float *owner_grad,
+                                          void *stream) {
+    if (!h) return EP_ERR_INVALID_ARG;
+    if (!h->d.balanced) return EP_ERR_UNSUPPORTED;
+    if (h->planned != 2) return h->planned == 1 ? EP_ERR_UNSUPPORTED : EP_ERR_NOT_PLANNED;
+    const Dims &d = h->d;
+    if (!replica_grads || replica_grads->num_ranks != d.R || d.R > EP_MAX_PEERS) return EP_ERR_INVALID_ARG;
+    const int64_t G4 = d.G / 4;
+    if (G4 == 0) return EP_OK;
+    if (!owner_grad || !aligned_to(owner_grad, 16)) return EP_ERR_INVALID_ARG;
+    PeerGrads pg;
+    memset(&pg, 0, sizeof pg);
+    for (int r = 0; r < d.R; ++r) {
+        if (!replica_grads->recv_x[r] || !aligned_to(replica_grads->recv_x[r], 16)) return EP_ERR_INVALID_ARG;
+        pg.rep[r] = (const float4 *)replica_grads->recv_x[r];
+    }
+    const int grid = num_sms() * 8;
+    const cudaError_t err =
+        launch_pdl(k_reduce_peers, dim3(grid), dim3(kRedPeerThreads), 0, (cudaStream_t)stream, pg, (float4 *)owner_grad,
+                   (const int32_t *)h->ws.red_experts, (const int32_t *)h->ws.red_count,
+                   (const int32_t *)h->ws.red_list, (const int32_t *)h->ws.red_n, d.R, d.S, h->world_rank * d.g, d.g,
+                   G4);
     return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 

@@ -94,6 +94,9 @@ SIGNATURES = {
     "ep_signal_peers": (ctypes.c_int, [_P, ctypes.POINTER(EpPeerTable), ctypes.c_uint32, _P]),
     "ep_wait_peers": (ctypes.c_int, [_P, _P, ctypes.c_uint32, _I64, _P]),
     "ep_combine_peers": (ctypes.c_int, [_P, ctypes.POINTER(EpPeerTable), _P, _P, _P]),
+    "ep_combine_backward_peers": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(EpPeerTable), _P]),
+    "ep_dispatch_backward_peers": (ctypes.c_int, [_P, ctypes.POINTER(EpPeerTable), _P, _P]),
+    "ep_reduce_replica_grads_peers": (ctypes.c_int, [_P, ctypes.POINTER(EpPeerTable), _P, _P]),
     "ep_ipc_export": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint8 * 64), ctypes.POINTER(_I64)]),
     "ep_ipc_import": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint8 * 64), _I64, ctypes.POINTER(_P),
                                      ctypes.POINTER(_P)]),
@@ -414,6 +417,23 @@ class Ep:
         _check("ep_combine_peers", lib().ep_combine_peers(
             self._h, ctypes.byref(table), self._p(topk_w, torch.float32, self.T * self.K, "topk_w"),
             self._p(out, torch.bfloat16, self.T * self.H, "out"), _stream(stream)))
+
+    def combine_backward_peers(self, grad_out, topk_w, grad_rows: EpPeerTable, stream=None) -> None:
+        _check("ep_combine_backward_peers", lib().ep_combine_backward_peers(
+            self._h, self._p(grad_out, torch.bfloat16, self.T * self.H, "grad_out"),
+            self._p(topk_w, torch.float32, self.T * self.K, "topk_w"), ctypes.byref(grad_rows), _stream(stream)))
+
+    def dispatch_backward_peers(self, grad_rows: EpPeerTable, grad_x, stream=None) -> None:
+        _check("ep_dispatch_backward_peers", lib().ep_dispatch_backward_peers(
+            self._h, ctypes.byref(grad_rows), self._p(grad_x, torch.bfloat16, self.T * self.H, "grad_x"),
+            _stream(stream)))
+
+    def reduce_replica_grads_peers(self, replica_grads: EpPeerTable, owner_grad, stream=None) -> None:
+        """This rank's experts' gradients [E/R, G] += their replicas' gradients,
+        read through the table (entry r: rank r's [S, G] fp32)."""
+        _check("ep_reduce_replica_grads_peers", lib().ep_reduce_replica_grads_peers(
+            self._h, ctypes.byref(replica_grads), self._p(owner_grad, torch.float32, (self.E // self.R) * self.G,
+                                                          "owner_grad"), _stream(stream)))
 
     # -- inspection
     def get_plan(self, stream=None) -> tuple[list[int], list[int]]:

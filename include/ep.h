@@ -302,7 +302,9 @@ ep_status_t ep_get_tensor(const ep_handle_t *h, ep_tensor_t which, const void **
  *              ep_wait_peers: the receive half of the staged mode);
  *   - combine: each rank reads its tokens' K rows from the ranks holding them
  *              and reduces them locally (ep_combine_peers: NCCL EP Table III,
- *              per-token reduction at the receiver).
+ *              per-token reduction at the receiver);
+ *   - backward: the same two movements with roles swapped, and the replica
+ *              gradients reduced into their owners across ranks.
  * Remote rows move with plain 16-byte stores and loads in the library's own
  * kernels (no bulk or multicast copies touch another GPU's memory).
  *
@@ -312,8 +314,8 @@ ep_status_t ep_get_tensor(const ep_handle_t *h, ep_tensor_t which, const void **
  * concatenation of all ranks' tokens, rank order) belongs to the rank r with
  * rank_offset[r] <= g < rank_offset[r+1], at local row g - rank_offset[r].
  * After ep_plan_world the single-GPU data calls (ep_dispatch, ep_combine, the
- * backward calls) refuse the handle with EP_ERR_UNSUPPORTED, and the peer
- * calls refuse a handle planned by ep_plan.
+ * backward calls, the replica reduce and prefetch) refuse the handle with
+ * EP_ERR_UNSUPPORTED, and the peer calls refuse a handle planned by ep_plan.
  */
 
 #define EP_MAX_PEERS 64
@@ -382,6 +384,34 @@ ep_status_t ep_wait_peers(ep_handle_t *h, const uint32_t *flags, uint32_t epoch,
  * bf16). out: device bf16 [T, H] of this rank's tokens. */
 ep_status_t ep_combine_peers(ep_handle_t *h, const ep_peer_table_t *peers, const float *topk_w, void *out,
                              void *stream);
+
+/* The backward pass across ranks (NCCL EP Fig. 5: the routing state of the
+ * forward pass serves the backward pass, roles swapped). The rows' tables use
+ * only their recv_x entries: rank r's gradient rows, bf16 [capacity_rows, H].
+ *   ep_combine_backward_peers: for every routed pair (t,k) of this rank with
+ *     global row g on rank r at local row l,
+ *       grad_rows->recv_x[r] row l = bf16(topk_w[t,k] * grad_out[t])
+ *     (one fp32 product, one rounding; as ep_combine_backward). grad_out:
+ *     this rank's bf16 [T, H]. Rows past capacity_rows are skipped and flagged.
+ *   ep_dispatch_backward_peers: grad_x[t] = bf16(sum over k of the pair's row
+ *     in grad_rows->recv_x[r], fp32 adds in k order from +0) (as
+ *     ep_dispatch_backward). grad_x: this rank's bf16 [T, H].
+ * Signal and wait between the ranks' phases as in the forward pass. */
+ep_status_t ep_combine_backward_peers(ep_handle_t *h, const void *grad_out, const float *topk_w,
+                                      const ep_peer_table_t *grad_rows, void *stream);
+ep_status_t ep_dispatch_backward_peers(ep_handle_t *h, const ep_peer_table_t *grad_rows, void *grad_x,
+                                       void *stream);
+
+/* Replica-gradient reduce across ranks (MoonEP article para. 5): this rank
+ * (the `rank` of its ep_plan_world) adds to each of its own experts e that has
+ * replicas under the world's balanced plan the gradients of e's replica slots
+ * (r, s), in ascending (r, s) order, read from replica_grads->recv_x[r] (rank
+ * r's replica gradients, fp32 [S, G]) at slot s:
+ *   owner_grad[e - rank*E/R, :] += replica_grads[r][s, :]   (fp32, in place)
+ * owner_grad: this rank's fp32 [E/R, G], G = cfg.grad_elems_per_expert. Needs
+ * cfg.balanced; the ranks' replica gradients must be complete (signal / wait). */
+ep_status_t ep_reduce_replica_grads_peers(ep_handle_t *h, const ep_peer_table_t *replica_grads, float *owner_grad,
+                                          void *stream);
 
 /* CUDA IPC of one device buffer, for building a peer table across processes:
  * export gives a 64-byte handle of the allocation holding dev_ptr and the

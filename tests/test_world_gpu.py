@@ -265,3 +265,87 @@ def test_world_empty_batches():
         assert (flags[q] == 3).all()
         np.testing.assert_array_equal(hs[q].tensor(ep.T_RANK_OFFSET).cpu().numpy(), np.zeros(R + 1))
         hs[q].close()
+
+
+def _plan_world_ranks(idx, Tl, H, E, K, R, balanced=False, G=0):
+    dev = torch.device("cuda")
+    hs = [ep.Ep(Tl, H, E, K, R, balanced=balanced, grad_elems_per_expert=G) for _ in range(R)]
+    ids = [idx[q * Tl:(q + 1) * Tl].contiguous().to(dev) for q in range(R)]
+    counts = torch.zeros((R, E), dtype=torch.int32, device=dev)
+    for q in range(R):
+        hs[q].plan_local_counts(ids[q], counts[q])
+    for q in range(R):
+        hs[q].plan_world(counts, q)
+    return hs, ids
+
+
+@pytest.mark.parametrize("balanced", [False, True])
+def test_world_backward(balanced):
+    """The backward pass across ranks against the oracle on the concatenated
+    batch: combine backward (weighted rows stored to the owning ranks),
+    dispatch backward (rows gathered and summed in k order), and, with a plan,
+    the replica gradients reduced into each owner's rows. Two steps alternate
+    two sets of gradient buffers (double buffering), each checked."""
+    g = _gc()
+    dev = torch.device("cuda")
+    R, Tl, H, E, K = 4, 300, 256, 32, 4
+    T = R * Tl
+    G = 1024 if balanced else 0
+    idx, w = synth.routing(T, E, K, zipf_s=1.0, seed=31)
+    ref = oracle.route(idx, E=E, R=R, balanced=balanced)
+    hs, ids = _plan_world_ranks(idx, Tl, H, E, K, R, balanced, G)
+    cap = ep.world_recv_rows(hs[0].cfg)
+    roff = hs[0].tensor(ep.T_RANK_OFFSET).cpu().numpy()
+    ws = [w[q * Tl:(q + 1) * Tl].contiguous().to(dev) for q in range(R)]
+    flags = [torch.zeros(R, dtype=torch.int32, device=dev) for _ in range(R)]
+    sets = [[torch.zeros((cap, H), dtype=torch.bfloat16, device=dev) for _ in range(R)] for _ in range(2)]
+    placed = np.unique(ref.dest_row[ref.dest_row >= 0])
+    epoch = 0
+    for step in range(2):
+        bufs = sets[step % 2]
+        tab = ep.peer_table(cap, bufs, flags)
+        gout = synth.tokens_bf16(T, H, seed=40 + step)
+        gout_d = [gout[q * Tl:(q + 1) * Tl].to(dev) for q in range(R)]
+        for q in range(R):
+            hs[q].combine_backward_peers(gout_d[q], ws[q], tab)
+        epoch += 1
+        for q in range(R):
+            hs[q].signal_peers(tab, epoch)
+        for q in range(R):
+            hs[q].wait_peers(flags[q], epoch, timeout_us=2_000_000)
+        torch.cuda.synchronize()
+        want = oracle.combine_backward(gout, w, ref.dest_row, ref.recv_rows)
+        for q in range(R):
+            rows = placed[(placed >= roff[q]) & (placed < roff[q + 1])]
+            lr = torch.from_numpy((rows - roff[q]).astype(np.int64)).to(dev)
+            g.assert_bf16_close(g.bits16(bufs[q][lr]), want[rows], f"combine backward, rank {q}, step {step}")
+        # dispatch backward: each rank's gradient rows (fresh values) summed per token
+        grecv = synth.tokens_bf16(ref.recv_rows, H, seed=50 + step)
+        for q in range(R):
+            n = roff[q + 1] - roff[q]
+            bufs[q][:n] = grecv[roff[q]:roff[q + 1]].to(dev)
+        torch.cuda.synchronize()
+        gx = [torch.empty((Tl, H), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+        for q in range(R):
+            hs[q].dispatch_backward_peers(tab, gx[q])
+        torch.cuda.synchronize()
+        want2 = oracle.combine(grecv, None, ref.dest_row, T, K)
+        got2 = np.concatenate([g.bits16(o) for o in gx])
+        g.assert_bf16_close(got2, want2, f"dispatch backward, step {step}")
+    if balanced:
+        S = hs[0].S
+        gen = torch.Generator().manual_seed(61)
+        rep = torch.randn((R, S, G), generator=gen)
+        own = torch.randn((E, G), generator=gen)
+        rep_d = [rep[q].contiguous().to(dev) for q in range(R)]
+        own_d = [own[q * (E // R):(q + 1) * (E // R)].contiguous().to(dev) for q in range(R)]
+        gtab = ep.peer_table(0, rep_d, None)
+        for q in range(R):
+            hs[q].reduce_replica_grads_peers(gtab, own_d[q])
+        torch.cuda.synchronize()
+        want3 = oracle.replica_reduce(ref.plan["replica_expert"], rep.numpy(), own.numpy())
+        np.testing.assert_array_equal(torch.cat([o.cpu() for o in own_d]).numpy(), want3)
+        assert (ref.plan["replica_expert"] >= 0).any()  # the plan has replicas to reduce
+    for q in range(R):
+        assert hs[q].status() == 0
+        hs[q].close()
