@@ -317,6 +317,41 @@ __global__ void __launch_bounds__(kRedPeerThreads) k_reduce_peers(PeerGrads pg, 
     }
 }
 
+// replica weight prefetch across ranks: for each replica slot s of this rank
+// that the world plan fills with expert e, copy e's weights from its owner's
+// table entry (e's row among the owner's experts). A persistent grid over
+// (slot, 16 KB chunk) items; empty slots are skipped.
+constexpr int kCopyPeerThreads = 256, kCopyPeerUnroll = 4;
+
+__global__ void __launch_bounds__(kCopyPeerThreads) k_prefetch_peers(PeerRows pw, uint4 *__restrict__ slots,
+                                                                     const int32_t *__restrict__ replica_expert,
+                                                                     int rank, int S, int g, int64_t V) {
+    pdl_wait();
+    const int64_t chunk = (int64_t)kCopyPeerThreads * kCopyPeerUnroll;
+    const int per = (int)((V + chunk - 1) / chunk); // chunks per expert (host-checked to fit)
+    const int items = S * per;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+        const int s = it / per;
+        const int e = replica_expert[rank * S + s];
+        if (e < 0) continue; // an empty slot
+        const int o = e / g;
+        const uint4 *src = reinterpret_cast<const uint4 *>(pw.x[o]) + (int64_t)(e - o * g) * V;
+        uint4 *dst = slots + (int64_t)s * V;
+        const int64_t base = (int64_t)(it % per) * chunk + threadIdx.x;
+        uint4 v[kCopyPeerUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyPeerUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kCopyPeerThreads;
+            if (i < V) v[u] = src[i];
+        }
+#pragma unroll
+        for (int u = 0; u < kCopyPeerUnroll; ++u) {
+            const int64_t i = base + (int64_t)u * kCopyPeerThreads;
+            if (i < V) dst[i] = v[u];
+        }
+    }
+}
+
 __device__ __forceinline__ void st_release_sys(uint32_t *p, uint32_t v) {
     asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -603,6 +638,28 @@ ep_status_t ep_reduce_replica_grads_peers(ep_handle_t *h, const ep_peer_table_t 
                    (const int32_t *)h->ws.red_experts, (const int32_t *)h->ws.red_count,
                    (const int32_t *)h->ws.red_list, (const int32_t *)h->ws.red_n, d.R, d.S, h->world_rank * d.g, d.g,
                    G4);
+    return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+ep_status_t ep_prefetch_replica_weights_peers(ep_handle_t *h, const ep_peer_table_t *weights,
+                                              int64_t bytes_per_expert, void *prefetch_slots, void *stream) {
+    if (!h) return EP_ERR_INVALID_ARG;
+    if (!h->d.balanced) return EP_ERR_UNSUPPORTED;
+    if (h->planned != 2) return h->planned == 1 ? EP_ERR_UNSUPPORTED : EP_ERR_NOT_PLANNED;
+    const Dims &d = h->d;
+    ep_status_t s = check_table(h, weights, true);
+    if (s != EP_OK) return s;
+    if (bytes_per_expert <= 0 || bytes_per_expert % 16 != 0 || !prefetch_slots || !aligned_to(prefetch_slots, 16))
+        return EP_ERR_INVALID_ARG;
+    // (slot, 16 KB chunk) items are counted in 32 bits
+    if ((bytes_per_expert / 16384 + 1) * (int64_t)d.S > INT32_MAX / 2) return EP_ERR_INVALID_ARG;
+    PeerRows pw;
+    fill_rows(weights, d.R, &pw);
+    const int64_t V = bytes_per_expert / 16;
+    const int grid = num_sms() * 8;
+    const cudaError_t err =
+        launch_pdl(k_prefetch_peers, dim3(grid), dim3(kCopyPeerThreads), 0, (cudaStream_t)stream, pw,
+                   (uint4 *)prefetch_slots, (const int32_t *)h->ws.replica_expert, h->world_rank, d.S, d.g, V);
     return err == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 

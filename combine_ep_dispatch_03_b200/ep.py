@@ -97,6 +97,7 @@ SIGNATURES = {
     "ep_combine_backward_peers": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(EpPeerTable), _P]),
     "ep_dispatch_backward_peers": (ctypes.c_int, [_P, ctypes.POINTER(EpPeerTable), _P, _P]),
     "ep_reduce_replica_grads_peers": (ctypes.c_int, [_P, ctypes.POINTER(EpPeerTable), _P, _P]),
+    "ep_prefetch_replica_weights_peers": (ctypes.c_int, [_P, ctypes.POINTER(EpPeerTable), _I64, _P, _P]),
     "ep_ipc_export": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint8 * 64), ctypes.POINTER(_I64)]),
     "ep_ipc_import": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint8 * 64), _I64, ctypes.POINTER(_P),
                                      ctypes.POINTER(_P)]),
@@ -434,6 +435,15 @@ class Ep:
         _check("ep_reduce_replica_grads_peers", lib().ep_reduce_replica_grads_peers(
             self._h, ctypes.byref(replica_grads), self._p(owner_grad, torch.float32, (self.E // self.R) * self.G,
                                                           "owner_grad"), _stream(stream)))
+
+    def prefetch_replica_weights_peers(self, weights: EpPeerTable, bytes_per_expert: int, prefetch_slots,
+                                       stream=None) -> None:
+        """This rank's filled replica slots [S, bytes] receive their experts'
+        weights, read from the owners' entries of the table ([E/R, bytes] each)."""
+        if prefetch_slots.numel() * prefetch_slots.element_size() != max(self.S, 1) * bytes_per_expert:
+            raise ValueError("prefetch_slots must hold S rows of one expert's weights")
+        _check("ep_prefetch_replica_weights_peers", lib().ep_prefetch_replica_weights_peers(
+            self._h, ctypes.byref(weights), bytes_per_expert, self._p(prefetch_slots), _stream(stream)))
 
     # -- inspection
     def get_plan(self, stream=None) -> tuple[list[int], list[int]]:

@@ -413,6 +413,17 @@ ep_status_t ep_dispatch_backward_peers(ep_handle_t *h, const ep_peer_table_t *gr
 ep_status_t ep_reduce_replica_grads_peers(ep_handle_t *h, const ep_peer_table_t *replica_grads, float *owner_grad,
                                           void *stream);
 
+/* Replica weight prefetch across ranks (MoonEP article paras. 3 and 5): for
+ * each replica slot s of this rank that the world's balanced plan fills with
+ * expert e, copy e's weights from its owner o = e / (E/R):
+ *   prefetch_slots[s, :] = weights->recv_x[o][e - o*E/R, :]   (bytes_per_expert)
+ * weights: a table whose recv_x[r] holds rank r's own experts' weights
+ * [E/R, bytes_per_expert]; prefetch_slots: this rank's [S, bytes_per_expert].
+ * Both 16-byte aligned, bytes_per_expert a positive multiple of 16. Empty
+ * slots are not written. Needs cfg.balanced. */
+ep_status_t ep_prefetch_replica_weights_peers(ep_handle_t *h, const ep_peer_table_t *weights,
+                                              int64_t bytes_per_expert, void *prefetch_slots, void *stream);
+
 /* CUDA IPC of one device buffer, for building a peer table across processes:
  * export gives a 64-byte handle of the allocation holding dev_ptr and the
  * pointer's offset inside it; import maps a peer's allocation into this

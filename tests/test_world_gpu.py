@@ -349,3 +349,31 @@ def test_world_backward(balanced):
     for q in range(R):
         assert hs[q].status() == 0
         hs[q].close()
+
+
+def test_world_prefetch_from_owners():
+    """Each rank's filled replica slots receive their experts' weights from the
+    owning ranks' tables; empty slots keep their contents (the oracle's
+    prefetch on the world's plan)."""
+    dev = torch.device("cuda")
+    R, Tl, E, K, B = 4, 400, 32, 4, 4096
+    g_ = E // R
+    idx, _ = synth.routing(R * Tl, E, K, zipf_s=1.5, seed=71)
+    ref = oracle.route(idx, E=E, R=R, balanced=True)
+    hs, _ = _plan_world_ranks(idx, Tl, 128, E, K, R, balanced=True)
+    S = hs[0].S
+    rng = np.random.default_rng(72)
+    weights = rng.integers(0, 256, size=(E, B), dtype=np.uint8)
+    slots0 = rng.integers(0, 256, size=(R * S, B), dtype=np.uint8)
+    wd = [torch.from_numpy(weights[q * g_:(q + 1) * g_].copy()).to(dev) for q in range(R)]
+    sd = [torch.from_numpy(slots0[q * S:(q + 1) * S].copy()).to(dev) for q in range(R)]
+    tab = ep.peer_table(0, wd, None)
+    for q in range(R):
+        hs[q].prefetch_replica_weights_peers(tab, B, sd[q])
+    torch.cuda.synchronize()
+    want = oracle.prefetch(ref.plan["replica_expert"], weights, slots0)
+    got = np.concatenate([s_.cpu().numpy() for s_ in sd])
+    np.testing.assert_array_equal(got, want)
+    assert (ref.plan["replica_expert"] >= 0).any() and (ref.plan["replica_expert"] < 0).any()
+    for h in hs:
+        h.close()
