@@ -21,13 +21,15 @@
 //   k_route_assign  per pair: stable index j = tile base + rank in tile ->
 //                   destination row through the layout tables (each CTA
 //                   computes the plain layouts' expert offsets itself)
-// Batches up to 32768 pairs without a plan, one kernel:
+// Batches up to 32768 pairs, one kernel:
 //   k_route_cluster a thread-block cluster of 8 or 16 CTAs; each CTA counts
 //                   and ranks its share of the pairs in shared memory, stores
 //                   its per-expert totals into every CTA's shared memory
 //                   (distributed shared memory) before one cluster barrier,
-//                   and then assigns its own pairs
-// Tiny batches without a plan, one kernel:
+//                   builds the layout (or the whole balanced plan) from the
+//                   totals itself, and then assigns its own pairs; CTA 0
+//                   also writes the tables out
+// Tiny batches (with a plan, up to 1024 pairs), one kernel:
 //   k_route_small   one CTA does all of the above in shared memory
 #include <atomic>
 
@@ -123,11 +125,14 @@ __device__ __forceinline__ uint32_t block_or(uint32_t v, uint32_t *s_acc) {
     return v;
 }
 
-// Exclusive scan of a[0..n) in shared memory by the whole block; returns the
-// total. s_warp needs 32 ints. Every thread of the block must call it. Two
+// Exclusive scan of a[0..n) in shared memory by the whole block: calls
+// visit(i, prefix of i, a[i]) once for every i, then returns the total.
+// s_warp needs 32 ints. Every thread of the block must call it. Two
 // barriers: after the warps' totals are stored, every warp scans the 32
-// totals itself (instead of one warp scanning them behind a third barrier).
-__device__ int block_exscan(int32_t *a, int n, int32_t *s_warp) {
+// totals itself (instead of one warp scanning them behind a third barrier);
+// the second follows the visits.
+template <class Visit>
+__device__ int block_exscan_visit(const int32_t *a, int n, int32_t *s_warp, Visit visit) {
     const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, w = tid >> 5, nw = nth >> 5;
     const int per = (n + nth - 1) / nth;
     const int lo = min(n, tid * per), hi = min(n, lo + per);
@@ -153,11 +158,16 @@ __device__ int block_exscan(int32_t *a, int n, int32_t *s_warp) {
     int run = wbase + incl - sum;
     for (int i = lo; i < hi; ++i) {
         const int x = a[i];
-        a[i] = run;
+        visit(i, run, x);
         run += x;
     }
-    __syncthreads(); // a[] is complete, and s_warp may be reused
+    __syncthreads(); // the visits are complete, and s_warp may be reused
     return total;
+}
+
+// The same, leaving the exclusive prefixes in a[].
+__device__ int block_exscan(int32_t *a, int n, int32_t *s_warp) {
+    return block_exscan_visit(a, n, s_warp, [=](int i, int pre, int) { a[i] = pre; });
 }
 
 // One warp walks pairs [lo, hi) of s_ids in (token, k) order, 32 at a time,
@@ -208,6 +218,7 @@ __device__ int plain_tables(const Dims &d, const int32_t *s_cnt, int32_t *s_len,
     const int E = d.E, tid = threadIdx.x, nth = blockDim.x;
     const bool ll = d.mode == EP_MODE_LL;
     uint32_t fl = 0;
+    #pragma unroll 1
     for (int e = tid; e < E; e += nth) {
         const int c = s_cnt[e];
         const int kept = ll ? min(c, d.cap) : c;
@@ -228,13 +239,16 @@ __device__ void plain_outputs(const Dims &d, const Workspace &ws, const int32_t 
                               int total) {
     const int E = d.E, R = d.R, g = d.g, tid = threadIdx.x, nth = blockDim.x;
     const bool ll = d.mode == EP_MODE_LL;
+    #pragma unroll 1
     for (int e = tid; e < E; e += nth) {
         ws.len0[e] = s_len[e];
         ws.base0[e] = s_base[e];
         ws.recv_counts[e] = s_len[e];
     }
+    #pragma unroll 1
     for (int r = tid >> 5; r < R; r += nth >> 5) { // a warp per rank
         int s = 0;
+        #pragma unroll 1
         for (int i = tid & 31; i < g; i += 32) s += s_len[r * g + i];
         s = __reduce_add_sync(kFull, s);
         if ((tid & 31) == 0) {
@@ -247,6 +261,20 @@ __device__ void plain_outputs(const Dims &d, const Workspace &ws, const int32_t 
         *ws.red_count = 0;
     }
 }
+
+// A plan's assignment tables as one CTA holds them in shared memory: piece 0
+// of expert e is stable indices [0, len0[e]) at rows base0[e] + j; its extra
+// pieces are x in [pfirst[e], pfirst[e] + pn[e]), each stable indices
+// [xstart[x], xstart[x] + xlen[x]) at rows xdst[x] + (j - xstart[x]).
+struct PlanView {
+    const int32_t *len0, *base0, *pfirst, *pn, *xstart, *xlen, *xdst;
+    __device__ __forceinline__ int dest(int e, int j) const {
+        if (j < len0[e]) return base0[e] + j;
+        for (int x = pfirst[e], xe = x + pn[e]; x < xe; ++x)
+            if (j >= xstart[x] && j < xstart[x] + xlen[x]) return xdst[x] + (j - xstart[x]);
+        return -1;
+    }
+};
 
 // Balanced-replica plan (MoonEP article paras. 3 and 5). The article states
 // only the invariants; this is a deterministic greedy:
@@ -261,53 +289,72 @@ __device__ void plain_outputs(const Dims &d, const Workspace &ws, const int32_t 
 //           then replica slots in slot order.
 // Every piece of an expert covers a run of its stable indices; the owner's
 // run [0, keep) is piece 0, the others ("extra" pieces) are stored compactly.
-__device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_t *s_cnt, int32_t *sm,
-                                int32_t *s_warp, uint32_t *s_fl) {
-    const int E = d.E, R = d.R, g = d.g, S = d.S, NX = d.nx_max, tid = threadIdx.x, nth = blockDim.x;
-    int32_t *s_keep = sm;                     // [E]
-    int32_t *s_tail = s_keep + E;             // [E] rows left on the owner after the fill
-    int32_t *s_list = s_tail + E;             // [E] scratch list / flags
-    int32_t *s_spill = s_list + E;            // [E] spilled experts
-    int32_t *s_own = s_spill + E;             // [E] own lengths, then own offsets
-    int32_t *s_pfirst = s_own + E;            // [E] first extra piece of each expert (creation order)
-    int32_t *s_pn = s_pfirst + E;             // [E] extra pieces of each expert
-    int32_t *s_D = s_pn + E;                  // [R] deficits, then loads
-    int32_t *s_nrep = s_D + R;                // [R]
-    int32_t *s_recv = s_nrep + R;             // [R] receivers in visiting order
-    int32_t *s_dn = s_recv + R;               // [R] direct pieces per rank
-    int32_t *s_dsum = s_dn + R;               // [R] rows in direct pieces per rank
-    int32_t *s_dbase = s_dsum + R;            // [R] own + slot rows per rank
-    int32_t *s_slot_e = s_dbase + R;          // [R*S]
-    int32_t *s_slot_len = s_slot_e + R * S;   // [R*S]
-    int32_t *s_slot_off = s_slot_len + R * S; // [R*S]
+//
+// Every thread of the CTA calls it. With `publish` the tables go to the
+// workspace; in any case the CTA keeps, in its shared memory, what the
+// assignment of its own pairs needs (the returned view), valid after the
+// function's final barrier.
+__device__ PlanView layout_balanced(const Dims &d, const Workspace &ws, const int32_t *s_cnt, int32_t *sm,
+                                    int32_t *s_warp, uint32_t *s_fl, bool publish) {
+    const int E = d.E, R = d.R, g = d.g, S = d.S, NX = d.nx_max, RS = d.R * d.S;
+    const int tid = threadIdx.x, nth = blockDim.x;
+    int32_t *s_keep = sm;                   // [E] rows each expert keeps on its owner
+    int32_t *s_list = s_keep + E;           // [E] spill flags; then the spilled experts in fill order
+    int32_t *s_spill = s_list + E;          // [E] spilled experts in id order; then each one's first receiver
+    int32_t *s_spc = s_spill + E;           // [E] their counts; then each one's last receiver; then base0
+    int32_t *s_sps = s_spc + E;             // [E] their spilled rows
+    int32_t *s_pfirst = s_sps + E;          // [E] first extra piece of each expert (creation order)
+    int32_t *s_pn = s_pfirst + E;           // [E] extra pieces of each expert
+    int32_t *s_D = s_pn + E;                // [R] deficits
+    int32_t *s_used = s_D + R;              // [R] rows each rank keeps of its own experts
+    int32_t *s_nrep = s_used + R;           // [R] slots taken (sequential fill)
+    int32_t *s_recv = s_nrep + R;           // [R] receivers in visiting order
+    int32_t *s_dn = s_recv + R;             // [R] direct pieces per rank
+    int32_t *s_fe = s_dn + R;               // [R] expert holding each receiver's first deficit row
+    int32_t *s_inner = s_fe + R;            // [R] 1 if that row is not an expert's first spilled row
+    int32_t *s_slot_e = s_inner + R;        // [R*S] expert of each replica slot, -1 empty
     // the extra pieces (beyond each expert's own rows) in creation order,
     // which groups them by expert
-    int32_t *s_x_start = s_slot_off + R * S;  // [NX] first stable index
-    int32_t *s_x_len = s_x_start + NX;        // [NX]
-    int32_t *s_x_rank = s_x_len + NX;         // [NX] rank holding the piece
-    int32_t *s_x_slot = s_x_rank + NX;        // [NX] slot >= 0, -2 owner tail, -3 direct
-    int32_t *s_x_aux = s_x_slot + NX;         // [NX] direct: rows before it among the rank's direct rows
-    int32_t *s_A = s_x_aux + NX;              // [E+1] first spilled row of each spilled expert (fill order)
-    int32_t *s_B = s_A + E + 1;               // [R+1] first deficit row of each receiver (visiting order)
-    int32_t *s_seg = s_B + R + 1;             // [R + 2E + R*S]: the scans of the fill and of the tables
-    __shared__ int s_nrecv, s_seq;
+    int32_t *s_x_start = s_slot_e + RS;     // [NX] first stable index
+    int32_t *s_x_len = s_x_start + NX;      // [NX]
+    int32_t *s_x_rank = s_x_len + NX;       // [NX] rank holding the piece
+    int32_t *s_x_slot = s_x_rank + NX;      // [NX] slot >= 0, -2 owner tail, -3 direct
+    int32_t *s_x_aux = s_x_slot + NX;       // [NX] direct: rows before it among the rank's direct rows; then its row
+    int32_t *s_A = s_x_aux + NX;            // [E+1] first spilled row of each spilled expert (fill order)
+    int32_t *s_B = s_A + E + 1;             // [R+1] first deficit row of each receiver (visiting order)
+    // one scan's input, [own rows of each expert | rows of each slot | direct
+    // rows of each rank | extra pieces of each expert | expert has replicas |
+    // slot is filled]: its prefixes give every offset of the layout
+    int32_t *s_seg = s_B + R + 1;
+    const int o_slen = E, o_dsum = E + RS, o_x = o_dsum + R, o_rep = o_x + E, o_slot = o_rep + E;
+    const int n_seg = o_slot + RS;
+    int32_t *q_own = s_seg, *q_slen = s_seg + o_slen, *q_dsum = s_seg + o_dsum, *q_x = s_seg + o_x,
+            *q_rep = s_seg + o_rep, *q_slot = s_seg + o_slot;
+    __shared__ int s_nrecv, s_seq, s_spill_total;
     __shared__ int s_wsum[32];
 
-    if (tid == 0) s_nrecv = 0;
-    for (int i = tid; i < R * S; i += nth) {
-        s_slot_e[i] = -1;
-        s_slot_len[i] = 0;
+    // 0. clear; L = routed pairs
+    if (tid == 0) {
+        s_nrecv = 0;
+        s_seq = 0;
+        s_spill_total = 0;
     }
+    #pragma unroll 1
+    for (int i = tid; i < RS; i += nth) s_slot_e[i] = -1;
+    #pragma unroll 1
+    for (int i = tid; i < n_seg; i += nth) s_seg[i] = 0;
+    #pragma unroll 1
     for (int r = tid; r < R; r += nth) {
+        s_used[r] = 0;
         s_nrep[r] = 0;
         s_dn[r] = 0;
-        s_dsum[r] = 0;
     }
-    if (d.direct)
+    if (d.direct && publish)
+        #pragma unroll 1
         for (int i = tid; i < R * E; i += nth) ws.direct_expert[i] = -1;
     int part = 0;
+    #pragma unroll 1
     for (int e = tid; e < E; e += nth) {
-        s_tail[e] = 0;
         s_pfirst[e] = 0;
         s_pn[e] = 0;
         part += s_cnt[e];
@@ -315,78 +362,82 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
     part = __reduce_add_sync(kFull, part);
     if ((tid & 31) == 0) s_wsum[tid >> 5] = part;
     __syncthreads();
-    int L = 0;
-    for (int w = 0; w < (nth >> 5); ++w) L += s_wsum[w];
+    const int L = __reduce_add_sync(kFull, (tid & 31) < (nth >> 5) ? s_wsum[tid & 31] : 0);
     const int q = L / R, rem = L % R;
+    auto capacity = [&](int r) { return q + (r < rem ? 1 : 0); };
 
-    // keep: rows of the experts visited before e on its rank (sorted order)
+    // 1. keep: rows of the experts visited before e on its rank (sorted order)
+    int spilled = 0;
+    #pragma unroll 1
     for (int e = tid; e < E; e += nth) {
-        const int r = e / g, c = s_cnt[e];
+        const int r = e / g, c = s_cnt[e], e0 = r * g;
         int before = 0;
+#pragma unroll 8
         for (int i = 0; i < g; ++i) {
-            const int e2 = r * g + i, c2 = s_cnt[e2];
-            if (c2 < c || (c2 == c && e2 < e)) before += c2;
+            const int c2 = s_cnt[e0 + i];
+            before += (c2 < c || (c2 == c && e0 + i < e)) ? c2 : 0;
         }
-        const int cap = q + (r < rem ? 1 : 0);
-        s_keep[e] = max(0, min(c, cap - before));
+        const int keep = max(0, min(c, capacity(r) - before));
+        s_keep[e] = keep;
+        q_own[e] = keep;
+        s_list[e] = c > keep ? 1 : 0;
+        spilled += c - keep;
+        if (keep > 0) atomicAdd(&s_used[r], keep);
     }
+    spilled = __reduce_add_sync(kFull, spilled);
+    if ((tid & 31) == 0 && spilled) atomicAdd(&s_spill_total, spilled);
     __syncthreads();
-    for (int r = tid; r < R; r += nth) {
-        int used = 0;
-        for (int i = 0; i < g; ++i) used += s_keep[r * g + i];
-        s_D[r] = q + (r < rem ? 1 : 0) - used;
-    }
-    for (int e = tid; e < E; e += nth) s_list[e] = s_cnt[e] > s_keep[e] ? 1 : 0;
-    __syncthreads();
-    const int nsp = block_exscan(s_list, E, s_warp); // position among spilled, id order
-    for (int e = tid; e < E; e += nth)
-        if (s_cnt[e] > s_keep[e]) s_spill[s_list[e]] = e;
-    __syncthreads();
-    // spilled experts by (count desc, id asc): rank within the compact list
+
+    // 2. the spilled experts, compact in id order, with their counts and spilled rows
+    const int nsp = block_exscan_visit(s_list, E, s_warp, [&](int e, int pos, int flag) {
+        if (flag) {
+            s_spill[pos] = e;
+            s_spc[pos] = s_cnt[e];
+            s_sps[pos] = s_cnt[e] - s_keep[e];
+        }
+    });
+
+    // 3. fill order: each spilled expert's place by (count desc, id asc) and
+    // its first spilled row (the rows of the experts before it); each
+    // receiver's place by (deficit desc, rank asc) and its first deficit row
+    const int spill_total = s_spill_total;
+    #pragma unroll 1
     for (int i = tid; i < nsp; i += nth) {
-        const int e = s_spill[i], c = s_cnt[e];
-        int pos = 0;
+        const int e = s_spill[i], c = s_spc[i];
+        int pos = 0, a = 0;
+#pragma unroll 8
         for (int i2 = 0; i2 < nsp; ++i2) {
-            const int e2 = s_spill[i2], c2 = s_cnt[e2];
-            if (c2 > c || (c2 == c && e2 < e)) ++pos;
+            const int c2 = s_spc[i2], e2 = s_spill[i2], v = s_sps[i2];
+            const bool ahead = c2 > c || (c2 == c && e2 < e);
+            pos += ahead ? 1 : 0;
+            a += ahead ? v : 0;
         }
         s_list[pos] = e;
+        s_A[pos] = a;
     }
-    // receivers: deficit > 0, by (deficit desc, rank asc)
+    #pragma unroll 1
     for (int r = tid; r < R; r += nth) {
-        if (s_D[r] <= 0) continue;
-        int pos = 0;
-        for (int r2 = 0; r2 < R; ++r2)
-            if (s_D[r2] > 0 && (s_D[r2] > s_D[r] || (s_D[r2] == s_D[r] && r2 < r))) ++pos;
+        const int D = capacity(r) - s_used[r]; // >= 0: no rank keeps more than its capacity
+        s_D[r] = D;
+        if (D <= 0) continue;
+        int pos = 0, b = 0;
+#pragma unroll 8
+        for (int r2 = 0; r2 < R; ++r2) {
+            const int D2 = capacity(r2) - s_used[r2];
+            const bool ahead = D2 > 0 && (D2 > D || (D2 == D && r2 < r));
+            pos += ahead ? 1 : 0;
+            b += ahead ? D2 : 0;
+        }
         s_recv[pos] = r;
+        s_B[pos] = b;
         atomicAdd(&s_nrecv, 1);
     }
+    // the deficits add up to the spilled rows (the capacities add up to L)
+    if (tid == 0) s_A[nsp] = spill_total;
     __syncthreads();
+    const int nrecv = s_nrecv;
+    if (tid == 0) s_B[nrecv] = spill_total; // read after the next barrier
 
-    // fill, parallel form. Without a slot running out, the greedy walk below
-    // pairs the spilled rows (experts in fill order, one after the other) with
-    // the deficit rows (receivers in visiting order) position by position: a
-    // piece is the overlap of one expert's spilled rows with one receiver's
-    // deficit rows. Receiver p's pieces come from consecutive experts, so a
-    // piece's slot is its expert's position minus that of the expert holding
-    // p's first deficit row. If some receiver would need more than S slots
-    // (and overflow is not served directly) the walk below runs instead.
-    // one scan over [spilled rows of each spilled expert | deficits of each
-    // receiver]: the first part's prefixes are the experts' first spilled rows
-    // (and its end the spilled total); the second part, less that total, the
-    // receivers' first deficit rows
-    const int nrecv_all = s_nrecv;
-    for (int i = tid; i < nsp; i += nth) s_seg[i] = s_cnt[s_list[i]] - s_keep[s_list[i]];
-    for (int i = tid; i < nrecv_all; i += nth) s_seg[nsp + i] = s_D[s_recv[i]];
-    if (tid == 0) s_seq = 0;
-    __syncthreads();
-    block_exscan(s_seg, nsp + nrecv_all, s_warp);
-    const int spill_total = s_seg[nsp];
-    s_A = s_seg; // [nsp + 1]: s_A[nsp] is the spilled total
-    // receiver q's first deficit row, read in place; the deficits add up to
-    // the spilled rows, so the one past the last receiver is the spilled total
-    const int32_t *s_Bs = s_seg + nsp;
-    auto Bv = [&](int q) { return q < nrecv_all ? s_Bs[q] - spill_total : spill_total; };
     // the last index i in [0, n) with a[i] <= v (a ascending, a[0] <= v)
     auto last_le = [](const int32_t *a, int n, int v) {
         int lo = 0, hi = n - 1;
@@ -396,85 +447,96 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
         }
         return lo;
     };
-    // the same over the receivers' first deficit rows
-    auto last_le_B = [&](int v) {
-        int lo = 0, hi = nrecv_all - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (Bv(mid) <= v) lo = mid; else hi = mid - 1;
+    // 4. without a slot running out, the greedy walk pairs the spilled rows
+    // (experts in fill order) with the deficit rows (receivers in visiting
+    // order) position by position: a piece is the overlap of one expert's
+    // spilled rows [A_i, A_i+1) with one receiver's deficit rows [B_q, B_q+1).
+    // Receiver q's pieces come from consecutive experts, from the one holding
+    // row B_q on, so a piece's slot is its expert's place minus that one's.
+    // Per receiver: that expert, whether B_q falls inside its rows, and the
+    // check that no receiver needs more than S slots (else, without direct
+    // overflow, the walk itself runs below). Per expert: the receivers
+    // holding its first and last spilled rows.
+    #pragma unroll 1
+    for (int k = tid; k < nrecv; k += nth) {
+        const int b0 = s_B[k], b1 = k + 1 < nrecv ? s_B[k + 1] : spill_total;
+        const int fe = last_le(s_A, nsp, b0), le = last_le(s_A, nsp, b1 - 1);
+        const int npc = le - fe + 1;
+        s_fe[k] = fe;
+        s_inner[k] = s_A[fe] < b0 ? 1 : 0;
+        if (npc > S) {
+            if (!d.direct) {
+                s_seq = 1;
+            } else { // pieces past the S-th are read directly from the owner
+                const int r = s_recv[k];
+                s_dn[r] = npc - S;
+                q_dsum[r] = b1 - s_A[fe + S];
+            }
         }
-        return lo;
-    };
-    for (int i = tid; i < nsp; i += nth) { // pass 1: pieces per expert, slot check
-        const int a0 = s_A[i], a1 = s_A[i + 1];
-        int n = 0;
-        for (int q = last_le_B(a0); q < nrecv_all && Bv(q) < a1; ++q, ++n) {
-            const int slot = i - last_le(s_A, nsp, Bv(q));
-            if (slot >= S && !d.direct) s_seq = 1;
-        }
-        s_spill[i] = n; // s_spill is free again: pieces of the i-th expert in fill order
+    }
+    #pragma unroll 1
+    for (int i = tid; i < nsp; i += nth) {
+        s_spill[i] = last_le(s_B, nrecv, s_A[i]);
+        s_spc[i] = last_le(s_B, nrecv, s_A[i + 1] - 1);
     }
     __syncthreads();
-    if (!s_seq) {
-        for (int i = tid; i < nsp; i += nth) { // pass 2: write the pieces
-            const int e = s_list[i];
-            const int a0 = s_A[i], a1 = s_A[i + 1];
-            int x = 0;
-            for (int i2 = 0; i2 < i; ++i2) x += s_spill[i2]; // pieces of earlier experts
+
+    if (!s_seq) { // uniform: set before the barrier
+        // 5. the pieces. Expert i's first piece is i plus the receivers' first
+        // rows that fall strictly inside the rows of the experts before it.
+        #pragma unroll 1
+        for (int i = tid; i < nsp; i += nth) {
+            const int e = s_list[i], a0 = s_A[i], a1 = s_A[i + 1], qf = s_spill[i], ql = s_spc[i];
+            int x = i;
+#pragma unroll 8
+            for (int k = 1; k <= qf; ++k) x += s_inner[k];
             s_pfirst[e] = x;
-            s_pn[e] = s_spill[i];
-            for (int q = last_le_B(a0); q < nrecv_all && Bv(q) < a1; ++q, ++x) {
-                const int r = s_recv[q];
-                const int lo = max(a0, Bv(q)), hi = min(a1, Bv(q + 1));
-                const int fe = last_le(s_A, nsp, Bv(q));
-                const int slot = i - fe;
+            s_pn[e] = ql - qf + 1;
+            q_x[e] = ql - qf + 1;
+            int rep = 0;
+            for (int k = qf; k <= ql; ++k, ++x) {
+                const int r = s_recv[k], b0 = s_B[k], b1 = s_B[k + 1];
+                const int lo = max(a0, b0), hi = min(a1, b1);
+                const int fe = s_fe[k], slot = i - fe;
                 s_x_start[x] = s_keep[e] + (lo - a0);
                 s_x_len[x] = hi - lo;
                 s_x_rank[x] = r;
                 if (slot < S) {
                     s_x_slot[x] = slot;
                     s_slot_e[r * S + slot] = e;
-                    s_slot_len[r * S + slot] = hi - lo;
+                    q_slen[r * S + slot] = hi - lo;
+                    q_slot[r * S + slot] = 1;
+                    rep = 1;
                 } else { // direct piece slot - S of rank r
-                    const int first_direct_row = min(Bv(q + 1), s_A[fe + S]);
+                    const int first_direct_row = min(b1, s_A[fe + S]);
                     s_x_slot[x] = -3;
                     s_x_aux[x] = lo - first_direct_row;
-                    ws.direct_expert[(int64_t)r * E + slot - S] = e;
-                    ws.direct_start[(int64_t)r * E + slot - S] = s_keep[e] + (lo - a0);
-                    ws.direct_len[(int64_t)r * E + slot - S] = hi - lo;
+                    if (publish) {
+                        ws.direct_expert[(int64_t)r * E + slot - S] = e;
+                        ws.direct_start[(int64_t)r * E + slot - S] = s_keep[e] + (lo - a0);
+                        ws.direct_len[(int64_t)r * E + slot - S] = hi - lo;
+                    }
                 }
             }
+            q_rep[e] = rep;
         }
-        for (int q = tid; q < nrecv_all; q += nth) { // per receiver: slots and direct rows used
-            const int r = s_recv[q];
-            const int fe = last_le(s_A, nsp, Bv(q)), le = last_le(s_A, nsp, Bv(q + 1) - 1);
-            const int npc = le - fe + 1;
-            s_nrep[r] = min(S, npc);
-            s_dn[r] = max(0, npc - S);
-            s_dsum[r] = npc > S ? Bv(q + 1) - s_A[fe + S] : 0;
-            s_D[r] = 0;
-        }
-    }
-    __syncthreads();
-
-    // fill, sequential form: one thread, one step per piece (receivers that
-    // ran out of deficit or slots never qualify again, so one cursor over them
-    // suffices; with direct overflow a receiver out of slots still qualifies
-    // and takes the rows as a direct piece). Pieces go to shared memory in
-    // creation order.
-    if (s_seq) { // uniform: set in pass 1, read after its barrier
+    } else {
+        // 5'. the walk itself: one thread, one step per piece (receivers that
+        // ran out of deficit or slots never qualify again, so one cursor over
+        // them suffices; with direct overflow a receiver out of slots still
+        // qualifies and takes the rows as a direct piece). Pieces go to shared
+        // memory in creation order.
         if (tid == 0) {
-            const int nrecv = s_nrecv;
             int p = 0, nx = 0;
             uint32_t fl = 0;
             for (int i = 0; i < nsp; ++i) {
                 const int e = s_list[i], owner = e / g;
-                int left = s_cnt[e] - s_keep[e], next = s_keep[e];
+                int left = s_cnt[e] - s_keep[e], next = s_keep[e], rep = 0;
                 s_pfirst[e] = nx;
                 while (left > 0) {
                     while (p < nrecv && (s_D[s_recv[p]] == 0 || (!d.direct && s_nrep[s_recv[p]] >= S))) ++p;
-                    if (p == nrecv) {
-                        s_tail[e] = left;
+                    if (p == nrecv) { // the owner keeps the rest
+                        q_own[e] += left;
                         s_x_start[nx] = next;
                         s_x_len[nx] = left;
                         s_x_rank[nx] = owner;
@@ -491,16 +553,20 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
                     if (s_nrep[r] < S) {
                         const int sl = s_nrep[r]++;
                         s_slot_e[r * S + sl] = e;
-                        s_slot_len[r * S + sl] = give;
+                        q_slen[r * S + sl] = give;
+                        q_slot[r * S + sl] = 1;
                         s_x_slot[nx] = sl;
+                        rep = 1;
                     } else { // a direct piece (direct overflow only)
                         const int di = s_dn[r]++;
-                        ws.direct_expert[(int64_t)r * E + di] = e;
-                        ws.direct_start[(int64_t)r * E + di] = next;
-                        ws.direct_len[(int64_t)r * E + di] = give;
+                        if (publish) {
+                            ws.direct_expert[(int64_t)r * E + di] = e;
+                            ws.direct_start[(int64_t)r * E + di] = next;
+                            ws.direct_len[(int64_t)r * E + di] = give;
+                        }
                         s_x_slot[nx] = -3;
-                        s_x_aux[nx] = s_dsum[r];
-                        s_dsum[r] += give;
+                        s_x_aux[nx] = q_dsum[r];
+                        q_dsum[r] += give;
                     }
                     ++nx;
                     s_D[r] -= give;
@@ -508,99 +574,98 @@ __device__ void layout_balanced(const Dims &d, const Workspace &ws, const int32_
                     next += give;
                 }
                 s_pn[e] = nx - s_pfirst[e];
+                q_x[e] = nx - s_pfirst[e];
+                q_rep[e] = rep;
             }
             if (fl) atomicOr(s_fl, fl);
         }
-        __syncthreads();
     }
-
-    // layout inside each rank region (a thread per rank): own experts, replica
-    // slots, direct pieces; and, for the one scan that follows, each expert's
-    // extra pieces, whether it has replicas, and which slots are filled
-    int32_t *q_roff = s_seg, *q_x = s_seg + R, *q_rep = q_x + E, *q_slot = q_rep + E;
-    for (int r = tid; r < R; r += nth) {
-        int run = 0;
-        int32_t *rc = ws.recv_counts + (int64_t)r * (g + S);
-        for (int i = 0; i < g; ++i) {
-            const int e = r * g + i, v = s_keep[e] + s_tail[e];
-            rc[i] = v;
-            s_own[e] = run;
-            run += v;
-        }
-        for (int sl = 0; sl < S; ++sl) {
-            const int v = s_slot_len[r * S + sl];
-            rc[g + sl] = v;
-            s_slot_off[r * S + sl] = run;
-            run += v;
-        }
-        s_dbase[r] = run;
-        run += s_dsum[r];
-        if (d.direct) ws.direct_n[r] = s_dn[r];
-        q_roff[r] = run;
-        ws.rank_load[r] = run;
-    }
-    for (int e = tid; e < E; e += nth) {
-        const int f = s_pfirst[e], n = s_pn[e];
-        int nrep = 0;
-        for (int i = 0; i < n; ++i) nrep += s_x_slot[f + i] >= 0 ? 1 : 0;
-        q_x[e] = n;
-        q_rep[e] = nrep > 0 ? 1 : 0;
-    }
-    for (int i = tid; i < R * S; i += nth) q_slot[i] = s_slot_e[i] >= 0 ? 1 : 0;
     __syncthreads();
-    // one scan over [rank loads | extra pieces | has replicas | filled slots];
-    // each part's prefixes are then relative to its first element's
-    const int grand = block_exscan(s_seg, R + 2 * E + R * S, s_warp);
-    const int rows_total = q_x[0], xb = q_x[0], rb = q_rep[0], sb = q_slot[0];
-    for (int r = tid; r < R; r += nth) ws.rank_off[r] = q_roff[r];
-    if (tid == 0) {
-        ws.rank_off[R] = rows_total;
-        ws.xoff[E] = rb - xb;
-        *ws.red_count = sb - rb;
-        *ws.slot_count = grand - sb;
+
+    // 6. one scan; then, with P the prefixes (each part's relative to its
+    // first element) and v(i) = P(i+1) - P(i) the scanned values:
+    //   rank r's region starts at own(r*g) + slots(r*S) + direct(r) and holds
+    //   its own experts (offsets own(e) - own(r*g)), then its slots, then its
+    //   direct rows
+    const int grand = block_exscan(s_seg, n_seg, s_warp);
+    const int32_t *P = s_seg;
+    auto own_total = [&](int r) { return P[(r + 1) * g] - P[r * g]; };
+    auto slot_total = [&](int r) { return P[o_slen + (r + 1) * S] - P[o_slen + r * S]; };
+    auto rank_off = [&](int r) { return P[r * g] + (P[o_slen + r * S] - P[o_slen]) + (P[o_dsum + r] - P[o_dsum]); };
+    if (publish) {
+        #pragma unroll 1
+        for (int e = tid; e < E; e += nth) // own rows of each own expert
+            ws.recv_counts[(int64_t)(e / g) * (g + S) + e % g] = P[e + 1] - P[e];
+        #pragma unroll 1
+        for (int i = tid; i < RS; i += nth) { // rows of each slot; the filled slots, ascending
+            ws.recv_counts[(int64_t)(i / S) * (g + S) + g + i % S] = P[o_slen + i + 1] - P[o_slen + i];
+            ws.replica_expert[i] = s_slot_e[i];
+            if (s_slot_e[i] >= 0) ws.slot_list[P[o_slot + i] - P[o_slot]] = i;
+        }
+        #pragma unroll 1
+        for (int r = tid; r < R; r += nth) {
+            const int dsum = P[o_dsum + r + 1] - P[o_dsum + r];
+            ws.rank_load[r] = own_total(r) + slot_total(r) + dsum;
+            ws.rank_off[r] = rank_off(r);
+            if (d.direct) ws.direct_n[r] = s_dn[r];
+        }
+        if (tid == 0) {
+            ws.rank_off[R] = P[o_x];
+            ws.xoff[E] = P[o_rep] - P[o_x];
+            *ws.red_count = P[o_slot] - P[o_rep];
+            *ws.slot_count = grand - P[o_slot];
+        }
     }
-    // the filled replica slots, ascending (the prefetch copies only these)
-    for (int i = tid; i < R * S; i += nth) {
-        ws.replica_expert[i] = s_slot_e[i];
-        if (s_slot_e[i] >= 0) ws.slot_list[q_slot[i] - sb] = i;
-    }
-    // piece 0, the compact extra pieces, and the per-expert replica lists
-    // (slots r*S+s in ascending order: each entry's place is the number of
-    // the expert's slot pieces with a smaller key)
+    // piece 0, the extra pieces' rows, and the per-expert replica lists (slots
+    // r*S+s in ascending order: each entry's place is the number of the
+    // expert's slot pieces with a smaller key)
+    #pragma unroll 1
     for (int e = tid; e < E; e += nth) {
         const int owner = e / g;
-        const int own_base = q_roff[owner] + s_own[e];
-        const int xo = q_x[e] - xb;
-        ws.base0[e] = own_base;
-        ws.len0[e] = s_keep[e];
-        ws.xoff[e] = xo;
+        const int own_base = rank_off(owner) + P[e] - P[owner * g];
+        const int xo = P[o_x + e] - P[o_x];
+        s_spc[e] = own_base;
+        if (publish) {
+            ws.base0[e] = own_base;
+            ws.len0[e] = s_keep[e];
+            ws.xoff[e] = xo;
+        }
         const int f = s_pfirst[e], n = s_pn[e];
         int nrep = 0;
         for (int i = 0; i < n; ++i) {
             const int x = f + i, r = s_x_rank[x], sl = s_x_slot[x];
-            const int o = xo + i;
-            ws.xstart[o] = s_x_start[x];
-            ws.xlen[o] = s_x_len[x];
+            int dst;
             if (sl == -2) {
-                ws.xdst[o] = own_base + s_keep[e];
+                dst = own_base + s_keep[e];
             } else if (sl == -3) { // direct piece: no slot, no gradient to reduce
-                ws.xdst[o] = q_roff[r] + s_dbase[r] + s_x_aux[x];
+                dst = rank_off(r) + own_total(r) + slot_total(r) + s_x_aux[x];
             } else {
-                ws.xdst[o] = q_roff[r] + s_slot_off[r * S + sl];
-                const int key = r * S + sl;
-                int pos = 0;
-                for (int i2 = 0; i2 < n; ++i2) {
-                    const int sl2 = s_x_slot[f + i2];
-                    if (sl2 >= 0 && s_x_rank[f + i2] * S + sl2 < key) ++pos;
+                dst = rank_off(r) + own_total(r) + P[o_slen + r * S + sl] - P[o_slen + r * S];
+                if (publish) {
+                    const int key = r * S + sl;
+                    int pos = 0;
+                    for (int i2 = 0; i2 < n; ++i2) {
+                        const int sl2 = s_x_slot[f + i2];
+                        if (sl2 >= 0 && s_x_rank[f + i2] * S + sl2 < key) ++pos;
+                    }
+                    ws.red_list[(int64_t)e * R + pos] = key;
                 }
-                ws.red_list[(int64_t)e * R + pos] = key;
                 ++nrep;
             }
+            s_x_aux[x] = dst;
+            if (publish) {
+                ws.xstart[xo + i] = s_x_start[x];
+                ws.xlen[xo + i] = s_x_len[x];
+                ws.xdst[xo + i] = dst;
+            }
         }
-        ws.red_n[e] = nrep;
-        if (nrep > 0) ws.red_experts[q_rep[e] - rb] = e;
+        if (publish) {
+            ws.red_n[e] = nrep;
+            if (nrep > 0) ws.red_experts[P[o_rep + e] - P[o_rep]] = e;
+        }
     }
     __syncthreads();
+    return PlanView{s_keep, s_spc, s_pfirst, s_pn, s_x_start, s_x_len, s_x_aux};
 }
 
 // ---------------------------------------------------------------------------
@@ -679,6 +744,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const int32_t *__r
     // the scan kernel's ticket starts every plan at 0, whatever an earlier
     // launch left there (the scan waits for this grid to complete)
     if (d.balanced && blockIdx.x == 0 && threadIdx.x == 0) *ws.ticket = 0ull;
+    #pragma unroll 1
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
         for (int ww = 0; ww < ntile; ++ww) {
@@ -755,7 +821,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_route_scan(Dims d, Workspace w
     for (int b = tid; b < d.nhist; b += nth) fl |= __ldcg(ws.tile_flags + b);
     block_or(fl, &s_fl);
     __syncthreads();
-    layout_balanced(d, ws, s_cnt, sm + d.E, s_warp, &s_fl);
+    layout_balanced(d, ws, s_cnt, sm + d.E, s_warp, &s_fl, true);
     if (tid == 0) *ws.flags = s_fl;
 }
 
@@ -779,6 +845,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspac
     int32_t *s_jb = s_xd + d.nx_max; // [E] world: this rank's first stable index per expert
     if (tid == 0) s_fl = 0;
     if (d.balanced || d.world) {
+        #pragma unroll 1
         for (int i = tid; i < E; i += nth) {
             s_base[i] = ws.base0[i];
             s_len[i] = ws.len0[i];
@@ -866,6 +933,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_route_world(Dims d, Workspace 
     uint32_t fl = 0; // this rank's id checks, from its histogram CTAs
     for (int b = tid; b < d.nhist; b += nth) fl |= ws.tile_flags[b];
     block_or(fl, &s_fl);
+    #pragma unroll 1
     for (int e = tid; e < E; e += nth) {
         int all = 0, before = 0;
         for (int r = 0; r < R; ++r) {
@@ -881,7 +949,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_route_world(Dims d, Workspace 
     if (tid == 0) ws.xoff[E] = 0;
     __syncthreads();
     if (d.balanced) {
-        layout_balanced(d, ws, s_cnt, s_plan, s_warp, &s_fl);
+        layout_balanced(d, ws, s_cnt, s_plan, s_warp, &s_fl, true);
     } else {
         const int total = plain_tables(d, s_cnt, s_len, s_base, s_warp, &s_fl);
         plain_outputs(d, ws, s_len, s_base, total);
@@ -967,6 +1035,7 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     __syncthreads();
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); // every CTA has started
     if (tid < C) *cluster.map_shared_rank(&s_flq[r], tid) = s_fl;
+    #pragma unroll 1
     for (int e = tid; e < E; e += blockDim.x) { // per-warp bases; the CTA's totals go to every CTA
         int run = 0;
         for (int w0 = 0; w0 < NW; w0 += 8) {
@@ -987,6 +1056,7 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     cluster.sync();
 
     // 2. totals of the whole batch and of the lower-ranked CTAs, all local now
+    #pragma unroll 1
     for (int e = tid; e < E; e += blockDim.x) {
         int before = 0, all = 0;
 #pragma unroll 8
@@ -1010,10 +1080,12 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
         const int total = plain_tables(d, s_cnt, s_len, s_off, s_warp, &s_fl);
         if (r == 0) {
             plain_outputs(d, ws, s_len, s_off, total);
+            #pragma unroll 1
             for (int e = tid; e < E; e += blockDim.x) ws.cnt[e] = s_cnt[e];
             __syncthreads();
             if (tid == 0) *ws.flags = s_fl;
         }
+        #pragma unroll 1
         for (int i = lo + lane; i < hi; i += 32) {
             const int pk = s_pk[i];
             const int e = pk & 0xffff;
@@ -1027,40 +1099,20 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
         }
         return;
     }
-    // 3'. balanced plan: CTA 0 builds it from the totals every CTA now holds and
-    // writes its tables to the workspace; the cluster barrier (release /
-    // acquire at cluster scope) makes them visible to every CTA, which then
-    // assigns its own pairs through them
+    // 3'. balanced plan: every CTA builds it from the totals it now holds, in
+    // its own shared memory (CTA 0 also publishes the tables), and assigns its
+    // own pairs through its copy
+    const PlanView pv = layout_balanced(d, ws, s_cnt, s_pk + ppc, s_warp, &s_fl, r == 0); // scratch: after the pair arrays
     if (r == 0) {
-        layout_balanced(d, ws, s_cnt, s_pk + ppc, s_warp, &s_fl); // scratch: after the pair arrays
+        #pragma unroll 1
         for (int e = tid; e < E; e += blockDim.x) ws.cnt[e] = s_cnt[e];
-        __syncthreads();
-        if (tid == 0) *ws.flags = s_fl;
+        if (tid == 0) *ws.flags = s_fl; // final: the planner's last barrier follows its last flag
     }
-    cluster.sync();
-    for (int e = tid; e < E; e += blockDim.x) {
-        s_len[e] = __ldcg(ws.len0 + e);
-        s_off[e] = __ldcg(ws.base0 + e);
-    }
-    __syncthreads();
+    #pragma unroll 1
     for (int i = lo + lane; i < hi; i += 32) {
         const int pk = s_pk[i];
         const int e = pk & 0xffff;
-        int dest = -1;
-        if (e != 0xffff) {
-            const int j = s_cta[e] + my[e] + (pk >> 16);
-            if (j < s_len[e]) {
-                dest = s_off[e] + j;
-            } else {
-                for (int x = __ldcg(ws.xoff + e), xe = __ldcg(ws.xoff + e + 1); x < xe; ++x) {
-                    const int xs = __ldcg(ws.xstart + x), xl = __ldcg(ws.xlen + x);
-                    if (j >= xs && j < xs + xl) {
-                        dest = __ldcg(ws.xdst + x) + (j - xs);
-                        break;
-                    }
-                }
-            }
-        }
+        const int dest = e != 0xffff ? pv.dest(e, s_cta[e] + my[e] + (pk >> 16)) : -1;
         ws.dest_row[c0 + i] = dest;
         if (dest >= 0 && ws.src_row) ws.src_row[dest] = (int32_t)(c0 + i);
     }
@@ -1097,6 +1149,7 @@ __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__
     warp_count(s_ids, lo, hi, K, E, my, fl);
     block_or(fl, &s_fl);
     __syncthreads();
+    #pragma unroll 1
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
         for (int ww = 0; ww < kSmallWarps; ++ww) {
@@ -1114,22 +1167,10 @@ __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__
         warp_assign(s_ids, lo, hi, K, E, my, ws.dest_row, ws.src_row,
                     [&](int e, int j) { return j < s_len[e] ? s_base[e] + j : -1; });
     } else {
-        // The plan's tables go to the workspace; this CTA's own writes are
-        // visible to it after the barrier. Piece 0 of each expert is kept in
-        // shared memory, the few extra pieces are read from the workspace.
-        layout_balanced(d, ws, s_cnt, s_plan, s_warp, &s_fl);
-        for (int e = threadIdx.x; e < E; e += blockDim.x) {
-            s_len[e] = ws.len0[e];
-            s_base[e] = ws.base0[e];
-        }
-        __syncthreads();
-        const int32_t *xoff = ws.xoff, *xs = ws.xstart, *xl = ws.xlen, *xd = ws.xdst;
-        warp_assign(s_ids, lo, hi, K, E, my, ws.dest_row, ws.src_row, [&](int e, int j) {
-            if (j < s_len[e]) return s_base[e] + j;
-            for (int x = xoff[e]; x < xoff[e + 1]; ++x)
-                if (j >= xs[x] && j < xs[x] + xl[x]) return xd[x] + (j - xs[x]);
-            return -1;
-        });
+        // the plan's tables go to the workspace; this CTA assigns its pairs
+        // through its own copy in shared memory
+        const PlanView pv = layout_balanced(d, ws, s_cnt, s_plan, s_warp, &s_fl, true);
+        warp_assign(s_ids, lo, hi, K, E, my, ws.dest_row, ws.src_row, [&](int e, int j) { return pv.dest(e, j); });
     }
     __syncthreads();
     if (threadIdx.x == 0) *ws.flags = s_fl;
@@ -1139,10 +1180,10 @@ __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__
 
 size_t route_smem_layout(const Dims &d) {
     if (!d.balanced) return 0;
-    const size_t E = d.E, R = d.R, S = d.S, NX = d.nx_max;
-    // s_cnt (callers), 7 E-arrays, 6 R-arrays, 3 slot arrays, 5 piece arrays,
-    // s_A, s_B, and the scans' buffer
-    return sizeof(int32_t) * (E + 7 * E + 6 * R + 3 * R * S + 5 * NX + E + 1 + R + 1 + (R + 2 * E + R * S));
+    const size_t E = d.E, R = d.R, RS = (size_t)d.R * d.S, NX = d.nx_max;
+    // s_cnt (callers), 7 E-arrays, 7 R-arrays, the slot experts, 5 piece
+    // arrays, s_A, s_B, and the scan's input (3 E-parts, 2 slot parts, R)
+    return sizeof(int32_t) * (E + 7 * E + 7 * R + RS + 5 * NX + E + 1 + R + 1 + (3 * E + 2 * RS + R));
 }
 
 size_t route_smem_assign(const Dims &d) {
@@ -1162,7 +1203,7 @@ size_t route_smem_small(const Dims &d) {
 }
 
 size_t route_smem_cluster(const Dims &d) {
-    // with a plan, the planner's scratch follows the pair arrays (CTA 0 uses it)
+    // with a plan, the planner's scratch follows the pair arrays (every CTA plans)
     return sizeof(int32_t) * ((size_t)(d.cl_warps + 4 + d.cl_size) * d.E + 2 * (size_t)d.cl_ppw * d.cl_warps) +
            route_smem_layout(d);
 }
