@@ -66,7 +66,11 @@ def workload_config(name: str, wl: dict, world: int, l2_note: str) -> dict:
             "parallelism": f"{world} independent EP worlds (one per GPU), R logical ranks each"}
 
 
-def l2_note_for(step_bytes: int, l2: int, flushed: bool) -> str:
+def l2_note_for(step_bytes: int, l2: int, flushed) -> str:
+    if flushed == "clean":
+        return (f"flushed, clean: before every timed step a {2 * l2 / 2**20:.0f} MiB buffer is written and then a "
+                "second one read, so the step finds none of its data in L2 and no dirty lines of the flush to write "
+                "back (the write alone leaves up to an L2 of them)")
     if flushed:
         return (f"flushed: each step moves {step_bytes / 1e6:.1f} MB, at most 4x L2 ({l2 / 2**20:.0f} MiB), so "
                 f"a {2 * l2 / 2**20:.0f} MiB buffer is written before every timed step and the steps are "
@@ -628,7 +632,8 @@ def timed(step: Step, steps, warmup, stream, breakdown_steps=None, graph=True, f
     With a `flush` buffer (larger than L2), every timed step, and every step
     of the per-call loop, follows a write of that buffer outside its events:
     the step is timed alone (a replay of a one-step graph, with `graph`), on
-    cold L2, and the step time is the sum of the steps' own times."""
+    cold L2, and the step time is the sum of the steps' own times. A pair of
+    buffers (written, then read) leaves L2 cold and clean."""
     import torch
 
     if flush is not None:
@@ -684,6 +689,15 @@ def timed(step: Step, steps, warmup, stream, breakdown_steps=None, graph=True, f
     return total, per
 
 
+def _flush_l2(flush, i):
+    """Write the flush buffer (and read the second one of a pair)."""
+    if isinstance(flush, tuple):
+        flush[0].fill_(i & 0x7F)
+        flush[1].sum()
+    else:
+        flush.fill_(i & 0x7F)
+
+
 def _timed_flushed(step: Step, steps, warmup, stream, breakdown_steps, graph, flush):
     import torch
 
@@ -703,7 +717,7 @@ def _timed_flushed(step: Step, steps, warmup, stream, breakdown_steps, graph, fl
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     with torch.cuda.stream(stream):
         for i in range(steps):
-            flush.fill_(i & 0x7F)
+            _flush_l2(flush, i)
             ev[i][0].record(stream)
             if g is not None:
                 g.replay()
@@ -718,7 +732,7 @@ def _timed_flushed(step: Step, steps, warmup, stream, breakdown_steps, graph, fl
     pev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(nb)]
     with torch.cuda.stream(stream):
         for s in range(nb):
-            flush.fill_(s & 0x7F)
+            _flush_l2(flush, s)
             pev[s][0].record(stream)
             for i, (_, f) in enumerate(step.calls):
                 f(stream)
@@ -992,11 +1006,12 @@ def run_sweep(dev, stream, seed, peak, steps=10, warmup=3):
     return rows
 
 
-def side_record(name: str, dev, stream, seed, peak, world, no_graph, steps, warmup, flushed: bool):
+def side_record(name: str, dev, stream, seed, peak, world, no_graph, steps, warmup, flushed):
     """One workload timed as the headline is (CUDA-graph replays, CUDA events
     on the launching stream, max over ranks), with or without an L2 flush
-    before every step: step time, GB/s of algorithmic bytes, fraction of the
-    measured copy bandwidth, per-call split and the clocks seen."""
+    before every step (flushed: True, False or "clean"): step time, GB/s of
+    algorithmic bytes, fraction of the measured copy bandwidth, per-call split
+    and the clocks seen."""
     import torch
 
     from combine_ep_dispatch_03_b200 import ep
@@ -1007,6 +1022,8 @@ def side_record(name: str, dev, stream, seed, peak, world, no_graph, steps, warm
     step_bytes = sum(nb.values())
     l2 = l2_bytes(dev)
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev) if flushed else None
+    if flushed == "clean":
+        flush = (flush, torch.zeros(2 * l2, dtype=torch.uint8, device=dev))
     torch.cuda.synchronize()
     t0 = time.time()
     total, per = timed(step, steps, warmup, stream, min(steps, 20), graph=not no_graph, flush=flush)
@@ -1050,6 +1067,8 @@ def run_side_workloads(dev, stream, seed, peak, world, no_graph):
         if small:
             rec["flushed"] = side_record(name, dev, stream, seed, peak, world, no_graph, steps, warmup, True)
             if name in ("ll_decode", "inference_decode", "ht_decode"):
+                rec["flushed_clean"] = side_record(name, dev, stream, seed, peak, world, no_graph, steps, warmup,
+                                                   "clean")
                 rec["back_to_back"] = side_record(name, dev, stream, seed, peak, world, no_graph, steps, warmup,
                                                   False)
         else:
@@ -1057,7 +1076,7 @@ def run_side_workloads(dev, stream, seed, peak, world, no_graph):
         out[name] = rec
     out["clocks"] = sampler.stop()  # every sample of the side workloads together
     for rec in out.values():
-        for mode in ("flushed", "back_to_back"):
+        for mode in ("flushed", "flushed_clean", "back_to_back"):
             if isinstance(rec, dict) and mode in rec:
                 rec[mode]["clocks"] = sampler.window(*rec[mode].pop("timed_host_interval"))
     if "inference_decode" in out and "ht_decode" in out:

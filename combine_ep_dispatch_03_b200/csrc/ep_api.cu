@@ -74,8 +74,8 @@ ep_status_t derive_dims(const ep_config_t *c, Dims *d) {
     const int64_t per_cta = (int64_t)kRouteThreads * kAssignPer; // pairs per assignment CTA
     d->nassign = (int)(L > 0 ? (L + per_cta - 1) / per_cta : 1);
     // cluster routing: at most kClusterMaxPairs pairs (measured faster than
-    // the three-kernel path there, slower beyond); with a balanced plan, CTA 0
-    // of the cluster runs the planner between two cluster barriers. The
+    // the three-kernel path there, slower beyond); with a balanced plan, every
+    // CTA of the cluster runs the planner after the cluster barrier. The
     // cluster shape keeps each warp near 64 pairs with as few warps per SM as
     // that allows, since the warp votes of the first pass issue slowly when
     // every warp of an SM votes. Step times measured per shape: 8192 pairs,

@@ -80,6 +80,31 @@ def test_l2_flush_decision():
     b = bench.algorithmic_bytes(wl["T"], wl["H"], wl["K"], wl["T"] * wl["K"], fp8=False)
     assert bench.needs_l2_flush(sum(b.values()), l2)
     assert bench.needs_l2_flush(4 * 32768 * 256 + 8 * 32768 * 8, l2)
+    # the three notes name what was done before each timed step
+    assert bench.l2_note_for(264568832, l2, True).startswith("flushed: ")
+    assert bench.l2_note_for(264568832, l2, "clean").startswith("flushed, clean: ")
+    assert "read" in bench.l2_note_for(264568832, l2, "clean")
+    assert bench.l2_note_for(264568832, l2, False).startswith("not flushed")
+
+
+class _Buf:
+    def __init__(self):
+        self.calls = []
+
+    def fill_(self, v):
+        self.calls.append(("fill", v))
+
+    def sum(self):
+        self.calls.append(("sum",))
+
+
+def test_flush_writes_then_reads_for_a_clean_l2():
+    w, r = _Buf(), _Buf()
+    bench._flush_l2((w, r), 130)
+    assert w.calls == [("fill", 130 & 0x7F)] and r.calls == [("sum",)]
+    one = _Buf()
+    bench._flush_l2(one, 3)
+    assert one.calls == [("fill", 3)]
 
 
 def test_modelled_exchange_stays_flat_under_the_balanced_plan():
