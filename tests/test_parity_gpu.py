@@ -168,8 +168,8 @@ def test_routing_shape_boundaries(T, K):
                                              (4097, 8, 128, 8, True)])
 def test_balanced_plan_shape_boundaries(T, K, E, R, direct):
     """The balanced plan is built inside the one-CTA routing kernel up to
-    1024 pairs, by CTA 0 of the one-launch routing cluster up to 32768 pairs
-    (between two cluster barriers), and by the three-kernel path beyond: both
+    1024 pairs, by every CTA of the one-launch routing cluster up to 32768
+    pairs (CTA 0 writes the tables out), and by the three-kernel path beyond: both
     sides of each switch, with skewed routing, training and inference plans
     (two slots a rank for the inference plan), forward and backward with the
     replica reduce."""
@@ -278,14 +278,18 @@ def test_hand_worked_plans():
         assert r["flags"] == c["flags"][0]
 
 
-def test_balanced_plan_slot_overflow_keeps_rows_on_owner():
+@pytest.mark.parametrize("T", [2048, 8192, 16384])
+def test_balanced_plan_slot_overflow_keeps_rows_on_owner(T):
     """Replica slots limited to 1 per rank under heavy skew: the plan runs out
-    of slots, raises PLAN_SLOTS and keeps the leftover rows on the owner; the
-    layout stays a permutation and matches the oracle."""
+    of slots (the planner's one-thread walk), raises PLAN_SLOTS and keeps the
+    leftover rows on the owner; the layout stays a permutation and matches the
+    oracle. 8192 pairs route in a cluster of 8 CTAs, 32768 in one of 16, and
+    65536 in three kernels."""
     g = _gc()
-    r = g.run_forward(2048, 256, 32, 4, 8, balanced=True, slots=1, zipf_s=2.0, seed=6, G=128)
+    r = g.run_forward(T, 256, 32, 4, 8, balanced=True, slots=1, zipf_s=2.0, seed=6, G=128)
+    assert ep.plan_launches(r["h"]) == (1 if T * 4 <= 32768 else 3)
     assert r["flags"] & oracle.FLAG_PLAN_SLOTS
-    assert sorted(r["ref"].dest_row.tolist()) == list(range(2048 * 4))
+    assert sorted(r["ref"].dest_row.tolist()) == list(range(T * 4))
     g.run_backward(r, seed=6)
 
 
