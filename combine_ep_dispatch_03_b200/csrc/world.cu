@@ -13,7 +13,7 @@
 // g - rank_off[r], and every row moves with plain 16-byte stores (dispatch)
 // or loads (combine) through the peer table: over NVLink when the table holds
 // other GPUs' mapped buffers, within one HBM when it holds local ones. No bulk
-// or multicast copy touches a peer's memory.
+// copy engine or cluster-wide broadcast load touches a peer's memory.
 #include <string.h>
 
 #include "bulk.cuh"

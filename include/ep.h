@@ -306,7 +306,8 @@ ep_status_t ep_get_tensor(const ep_handle_t *h, ep_tensor_t which, const void **
  *   - backward: the same two movements with roles swapped, and the replica
  *              gradients reduced into their owners across ranks.
  * Remote rows move with plain 16-byte stores and loads in the library's own
- * kernels (no bulk or multicast copies touch another GPU's memory).
+ * kernels (no bulk copy or cluster-wide broadcast load touches another GPU's
+ * memory).
  *
  * A handle for this mode is created with cfg.num_tokens = this rank's tokens
  * (the same on every rank) and cfg.num_ranks = R, the number of GPUs; global
