@@ -218,7 +218,7 @@ __device__ int plain_tables(const Dims &d, const int32_t *s_cnt, int32_t *s_len,
     const int E = d.E, tid = threadIdx.x, nth = blockDim.x;
     const bool ll = d.mode == EP_MODE_LL;
     uint32_t fl = 0;
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nth) {
         const int c = s_cnt[e];
         const int kept = ll ? min(c, d.cap) : c;
@@ -239,16 +239,16 @@ __device__ void plain_outputs(const Dims &d, const Workspace &ws, const int32_t 
                               int total) {
     const int E = d.E, R = d.R, g = d.g, tid = threadIdx.x, nth = blockDim.x;
     const bool ll = d.mode == EP_MODE_LL;
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nth) {
         ws.len0[e] = s_len[e];
         ws.base0[e] = s_base[e];
         ws.recv_counts[e] = s_len[e];
     }
-    #pragma unroll 1
+#pragma unroll 1
     for (int r = tid >> 5; r < R; r += nth >> 5) { // a warp per rank
         int s = 0;
-        #pragma unroll 1
+#pragma unroll 1
         for (int i = tid & 31; i < g; i += 32) s += s_len[r * g + i];
         s = __reduce_add_sync(kFull, s);
         if ((tid & 31) == 0) {
@@ -339,21 +339,22 @@ __device__ PlanView layout_balanced(const Dims &d, const Workspace &ws, const in
         s_seq = 0;
         s_spill_total = 0;
     }
-    #pragma unroll 1
+#pragma unroll 1
     for (int i = tid; i < RS; i += nth) s_slot_e[i] = -1;
-    #pragma unroll 1
+#pragma unroll 1
     for (int i = tid; i < n_seg; i += nth) s_seg[i] = 0;
-    #pragma unroll 1
+#pragma unroll 1
     for (int r = tid; r < R; r += nth) {
         s_used[r] = 0;
         s_nrep[r] = 0;
         s_dn[r] = 0;
     }
-    if (d.direct && publish)
-        #pragma unroll 1
+    if (d.direct && publish) {
+#pragma unroll 1
         for (int i = tid; i < R * E; i += nth) ws.direct_expert[i] = -1;
+    }
     int part = 0;
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nth) {
         s_pfirst[e] = 0;
         s_pn[e] = 0;
@@ -368,7 +369,7 @@ __device__ PlanView layout_balanced(const Dims &d, const Workspace &ws, const in
 
     // 1. keep: rows of the experts visited before e on its rank (sorted order)
     int spilled = 0;
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nth) {
         const int r = e / g, c = s_cnt[e], e0 = r * g;
         int before = 0;
@@ -401,7 +402,7 @@ __device__ PlanView layout_balanced(const Dims &d, const Workspace &ws, const in
     // its first spilled row (the rows of the experts before it); each
     // receiver's place by (deficit desc, rank asc) and its first deficit row
     const int spill_total = s_spill_total;
-    #pragma unroll 1
+#pragma unroll 1
     for (int i = tid; i < nsp; i += nth) {
         const int e = s_spill[i], c = s_spc[i];
         int pos = 0, a = 0;
@@ -415,7 +416,7 @@ __device__ PlanView layout_balanced(const Dims &d, const Workspace &ws, const in
         s_list[pos] = e;
         s_A[pos] = a;
     }
-    #pragma unroll 1
+#pragma unroll 1
     for (int r = tid; r < R; r += nth) {
         const int D = capacity(r) - s_used[r]; // >= 0: no rank keeps more than its capacity
         s_D[r] = D;
@@ -457,7 +458,7 @@ __device__ PlanView layout_balanced(const Dims &d, const Workspace &ws, const in
     // check that no receiver needs more than S slots (else, without direct
     // overflow, the walk itself runs below). Per expert: the receivers
     // holding its first and last spilled rows.
-    #pragma unroll 1
+#pragma unroll 1
     for (int k = tid; k < nrecv; k += nth) {
         const int b0 = s_B[k], b1 = k + 1 < nrecv ? s_B[k + 1] : spill_total;
         const int fe = last_le(s_A, nsp, b0), le = last_le(s_A, nsp, b1 - 1);
@@ -474,7 +475,7 @@ __device__ PlanView layout_balanced(const Dims &d, const Workspace &ws, const in
             }
         }
     }
-    #pragma unroll 1
+#pragma unroll 1
     for (int i = tid; i < nsp; i += nth) {
         s_spill[i] = last_le(s_B, nrecv, s_A[i]);
         s_spc[i] = last_le(s_B, nrecv, s_A[i + 1] - 1);
@@ -484,7 +485,7 @@ __device__ PlanView layout_balanced(const Dims &d, const Workspace &ws, const in
     if (!s_seq) { // uniform: set before the barrier
         // 5. the pieces. Expert i's first piece is i plus the receivers' first
         // rows that fall strictly inside the rows of the experts before it.
-        #pragma unroll 1
+#pragma unroll 1
         for (int i = tid; i < nsp; i += nth) {
             const int e = s_list[i], a0 = s_A[i], a1 = s_A[i + 1], qf = s_spill[i], ql = s_spc[i];
             int x = i;
@@ -593,16 +594,16 @@ __device__ PlanView layout_balanced(const Dims &d, const Workspace &ws, const in
     auto slot_total = [&](int r) { return P[o_slen + (r + 1) * S] - P[o_slen + r * S]; };
     auto rank_off = [&](int r) { return P[r * g] + (P[o_slen + r * S] - P[o_slen]) + (P[o_dsum + r] - P[o_dsum]); };
     if (publish) {
-        #pragma unroll 1
+#pragma unroll 1
         for (int e = tid; e < E; e += nth) // own rows of each own expert
             ws.recv_counts[(int64_t)(e / g) * (g + S) + e % g] = P[e + 1] - P[e];
-        #pragma unroll 1
+#pragma unroll 1
         for (int i = tid; i < RS; i += nth) { // rows of each slot; the filled slots, ascending
             ws.recv_counts[(int64_t)(i / S) * (g + S) + g + i % S] = P[o_slen + i + 1] - P[o_slen + i];
             ws.replica_expert[i] = s_slot_e[i];
             if (s_slot_e[i] >= 0) ws.slot_list[P[o_slot + i] - P[o_slot]] = i;
         }
-        #pragma unroll 1
+#pragma unroll 1
         for (int r = tid; r < R; r += nth) {
             const int dsum = P[o_dsum + r + 1] - P[o_dsum + r];
             ws.rank_load[r] = own_total(r) + slot_total(r) + dsum;
@@ -619,7 +620,7 @@ __device__ PlanView layout_balanced(const Dims &d, const Workspace &ws, const in
     // piece 0, the extra pieces' rows, and the per-expert replica lists (slots
     // r*S+s in ascending order: each entry's place is the number of the
     // expert's slot pieces with a smaller key)
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nth) {
         const int owner = e / g;
         const int own_base = rank_off(owner) + P[e] - P[owner * g];
@@ -744,7 +745,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_hist(const int32_t *__r
     // the scan kernel's ticket starts every plan at 0, whatever an earlier
     // launch left there (the scan waits for this grid to complete)
     if (d.balanced && blockIdx.x == 0 && threadIdx.x == 0) *ws.ticket = 0ull;
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
         for (int ww = 0; ww < ntile; ++ww) {
@@ -845,7 +846,7 @@ __global__ void __launch_bounds__(kRouteThreads) k_route_assign(Dims d, Workspac
     int32_t *s_jb = s_xd + d.nx_max; // [E] world: this rank's first stable index per expert
     if (tid == 0) s_fl = 0;
     if (d.balanced || d.world) {
-        #pragma unroll 1
+#pragma unroll 1
         for (int i = tid; i < E; i += nth) {
             s_base[i] = ws.base0[i];
             s_len[i] = ws.len0[i];
@@ -933,7 +934,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_route_world(Dims d, Workspace 
     uint32_t fl = 0; // this rank's id checks, from its histogram CTAs
     for (int b = tid; b < d.nhist; b += nth) fl |= ws.tile_flags[b];
     block_or(fl, &s_fl);
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += nth) {
         int all = 0, before = 0;
         for (int r = 0; r < R; ++r) {
@@ -1035,7 +1036,7 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     __syncthreads();
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); // every CTA has started
     if (tid < C) *cluster.map_shared_rank(&s_flq[r], tid) = s_fl;
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += blockDim.x) { // per-warp bases; the CTA's totals go to every CTA
         int run = 0;
         for (int w0 = 0; w0 < NW; w0 += 8) {
@@ -1056,7 +1057,7 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     cluster.sync();
 
     // 2. totals of the whole batch and of the lower-ranked CTAs, all local now
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = tid; e < E; e += blockDim.x) {
         int before = 0, all = 0;
 #pragma unroll 8
@@ -1080,12 +1081,12 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
         const int total = plain_tables(d, s_cnt, s_len, s_off, s_warp, &s_fl);
         if (r == 0) {
             plain_outputs(d, ws, s_len, s_off, total);
-            #pragma unroll 1
+#pragma unroll 1
             for (int e = tid; e < E; e += blockDim.x) ws.cnt[e] = s_cnt[e];
             __syncthreads();
             if (tid == 0) *ws.flags = s_fl;
         }
-        #pragma unroll 1
+#pragma unroll 1
         for (int i = lo + lane; i < hi; i += 32) {
             const int pk = s_pk[i];
             const int e = pk & 0xffff;
@@ -1104,11 +1105,11 @@ __global__ void __launch_bounds__(kClusterThreads) k_route_cluster(const int32_t
     // own pairs through its copy
     const PlanView pv = layout_balanced(d, ws, s_cnt, s_pk + ppc, s_warp, &s_fl, r == 0); // scratch: after the pair arrays
     if (r == 0) {
-        #pragma unroll 1
+#pragma unroll 1
         for (int e = tid; e < E; e += blockDim.x) ws.cnt[e] = s_cnt[e];
         if (tid == 0) *ws.flags = s_fl; // final: the planner's last barrier follows its last flag
     }
-    #pragma unroll 1
+#pragma unroll 1
     for (int i = lo + lane; i < hi; i += 32) {
         const int pk = s_pk[i];
         const int e = pk & 0xffff;
@@ -1149,7 +1150,7 @@ __global__ void __launch_bounds__(kSmallThreads) k_route_small(const int32_t *__
     warp_count(s_ids, lo, hi, K, E, my, fl);
     block_or(fl, &s_fl);
     __syncthreads();
-    #pragma unroll 1
+#pragma unroll 1
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
         for (int ww = 0; ww < kSmallWarps; ++ww) {
