@@ -88,6 +88,44 @@ def test_router_topk_near_ties(T, E, K):
     _check_router((base.view(torch.int32) ^ low).view(torch.float32).contiguous(), K)
 
 
+def _fuzz_case(i):
+    rng = np.random.default_rng(11000 + i)
+    if i % 2 == 0:  # four lanes a token: K <= 8, E a multiple of 16
+        E = int(rng.choice([16, 32, 48, 64, 128, 256, 384, 512, 1024]))
+        K = int(rng.integers(1, min(E, 8) + 1))
+    else:  # a warp a token
+        E = int(rng.integers(1, 1025))
+        K = int(rng.integers(1, min(E, 32) + 1))
+    T = int(rng.choice([1, 7, 8, 9, 63, 64, 65, 500, 2049]))
+    kind = ["normal", "ties", "near", "signed_zero", "wide"][i % 5]
+    return T, E, K, kind, 11000 + i
+
+
+@pytest.mark.parametrize("T,E,K,kind,seed", [_fuzz_case(i) for i in range(60)])
+def test_router_topk_random(T, E, K, kind, seed):
+    """Random sizes on both router kernels and logits that stress the
+    selection: exact ties (values on a coarse grid), near-ties (all but the
+    low mantissa bits equal), signed zeros among them, and a wide range of
+    magnitudes and signs. Ids bit-exact; weights within the derived bound."""
+    g = torch.Generator().manual_seed(seed)
+    if kind == "normal":
+        lg = torch.randn(T, E, generator=g)
+    elif kind == "ties":
+        lg = torch.randint(-3, 4, (T, E), generator=g).to(torch.float32) * 0.5
+    elif kind == "near":
+        base = torch.randn(T, 1, generator=g).expand(T, E).contiguous()
+        low = torch.randint(0, 1 << 9, (T, E), generator=g, dtype=torch.int32)
+        lg = (base.view(torch.int32) ^ low).view(torch.float32)
+    elif kind == "signed_zero":
+        lg = torch.randint(-1, 2, (T, E), generator=g).to(torch.float32) * 1e-3
+        zero = torch.rand(T, E, generator=g) < 0.5
+        lg[zero] = torch.where(torch.rand(int(zero.sum()), generator=g) < 0.5, torch.tensor(0.0),
+                               torch.tensor(-0.0))
+    else:
+        lg = torch.randn(T, E, generator=g) * torch.exp(torch.randn(T, E, generator=g) * 8)
+    _check_router(lg.contiguous(), K)
+
+
 def test_router_feeds_plan_dispatch_combine():
     """Router -> plan -> dispatch -> combine on the GPU equals the oracle chain."""
     import gpu_cases
