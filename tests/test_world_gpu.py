@@ -377,3 +377,30 @@ def test_world_prefetch_from_owners():
     assert (ref.plan["replica_expert"] >= 0).any() and (ref.plan["replica_expert"] < 0).any()
     for h in hs:
         h.close()
+
+
+def _world_case(i):
+    rng = np.random.default_rng(13000 + i)
+    R = int(rng.choice([2, 4, 8]))
+    E = R * int(rng.choice([1, 2, 4, 8, 16, 32]))
+    K = int(rng.integers(1, min(E, 8) + 1))
+    Tl = int(rng.choice([1, 3, 64, 129, 300, 700, 2000]))
+    H = int(rng.choice([128, 256]))
+    mode = "ll" if rng.random() < 0.3 else "ht"
+    cap = int(rng.integers(1, max(2, 2 * Tl * R * K // E) + 1)) if mode == "ll" else 0
+    fp8 = bool(mode == "ht" and rng.random() < 0.3)
+    balanced = bool(mode == "ht" and rng.random() < 0.4)
+    slots = int(rng.integers(0, E // R + 1)) if balanced else 0
+    direct = bool(balanced and slots > 0 and rng.random() < 0.4)
+    s = float(rng.choice([0.0, 1.0, 2.0]))
+    return Tl, H, E, K, R, mode, cap, fp8, balanced, slots, direct, s, 13000 + i
+
+
+@pytest.mark.parametrize("Tl,H,E,K,R,mode,cap,fp8,balanced,slots,direct,s,seed",
+                         [_world_case(i) for i in range(40)])
+def test_world_random(Tl, H, E, K, R, mode, cap, fp8, balanced, slots, direct, s, seed):
+    """Seeded random worlds: ranks, experts, top-K, tokens a rank, HT or LL
+    (random capacities), FP8, and balanced plans with slots and direct
+    overflow, each against the oracle's routing of the concatenated batch."""
+    _world(Tl, H, E, K, R, mode=mode, cap=cap, fp8=fp8, balanced=balanced, slots=slots, direct=direct, zipf_s=s,
+           seed=seed)
