@@ -106,7 +106,9 @@ typedef struct ep_config {
     int32_t ll_capacity;           /* LL: rows per expert (>= 1); ignored in HT */
     int32_t fp8;                   /* 1: dispatch casts to FP8 e4m3 + fp32 scales */
     int32_t balanced;              /* 1: balanced-replica plan (HT only; its tables must
-                                      fit one CTA's shared memory, about E <= 2048) */
+                                      fit one CTA's shared memory: E up to about 1700
+                                      with the default E/R slots a rank, about 2200 with
+                                      two; ep_validate_config decides) */
     int32_t replica_slots;         /* S in [1, E/R] with balanced; 0 = E/R */
     int64_t grad_elems_per_expert; /* G for ep_reduce_replica_grads; 0 if unused */
     int32_t direct_overflow;       /* 1 (with balanced): inference plan, see ep_plan */
