@@ -108,7 +108,8 @@ typedef struct ep_config {
     int32_t balanced;              /* 1: balanced-replica plan (HT only; its tables must
                                       fit one CTA's shared memory: E up to about 1700
                                       with the default E/R slots a rank, about 2200 with
-                                      two; ep_validate_config decides) */
+                                      two; beyond it ep_validate_config returns
+                                      EP_ERR_UNSUPPORTED) */
     int32_t replica_slots;         /* S in [1, E/R] with balanced; 0 = E/R */
     int64_t grad_elems_per_expert; /* G for ep_reduce_replica_grads; 0 if unused */
     int32_t direct_overflow;       /* 1 (with balanced): inference plan, see ep_plan */

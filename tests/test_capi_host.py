@@ -70,7 +70,7 @@ def _cfg(**kw):
     (dict(T=-1), 1),
     # a balanced plan's tables fit one CTA's shared memory (the limit ep.h states)
     (dict(E=1696, R=8, K=8, balanced=True), 0),
-    (dict(E=2048, R=8, K=8, balanced=True), 1),
+    (dict(E=2048, R=8, K=8, balanced=True), 3),  # unsupported, not malformed
     (dict(E=2048, R=8, K=8, balanced=True, replica_slots=2), 0),
     (dict(E=2048, R=8, K=8), 0),      # no plan: no such limit
 ])
