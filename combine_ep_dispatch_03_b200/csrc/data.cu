@@ -314,9 +314,13 @@ __global__ void __launch_bounds__(kRedThreads) k_replica_reduce(const float4 *__
 
 // ---------------------------------------------------------------------------
 // replica weight prefetch: slots[r*S+s] = weights[replica_expert[r*S+s]] for
-// every filled slot; a persistent grid over (slot, chunk) items
+// every filled slot. The grid strides over (slot, chunk) items of 8 KB, with
+// twice the CTAs an SM holds: the CTAs that start late fill the SMs that
+// finish early. Measured on the large step's plan (1.03 GB copied), 318 us
+// against 331 us for 16 KB items on a grid that fits at once, and 325 us for
+// 4 KB items.
 // ---------------------------------------------------------------------------
-constexpr int kCopyThreads = 256, kCopyUnroll = 4;
+constexpr int kCopyThreads = 256, kCopyUnroll = 2, kCopyCtasPerSm = 16;
 
 __global__ void __launch_bounds__(kCopyThreads) k_prefetch(const uint4 *__restrict__ weights,
                                                            uint4 *__restrict__ slots,
@@ -476,7 +480,7 @@ cudaError_t launch_prefetch(const Dims &d, const Workspace &ws, const void *weig
                             void *slots, cudaStream_t st) {
     const int64_t V = bytes_per_expert / 16;
     if (V == 0 || d.R * d.S == 0) return cudaSuccess;
-    const int grid = num_sms() * 8;
+    const int grid = num_sms() * kCopyCtasPerSm;
     return launch_pdl(k_prefetch, dim3(grid), dim3(kCopyThreads), 0, st, (const uint4 *)weights, (uint4 *)slots,
                       (const int32_t *)ws.replica_expert, (const int32_t *)ws.slot_list,
                       (const int32_t *)ws.slot_count, V);

@@ -363,8 +363,8 @@ ep_status_t ep_prefetch_replica_weights(ep_handle_t *h, const void *expert_weigh
     if (bytes_per_expert <= 0 || bytes_per_expert % 16 != 0 || !expert_weights || !prefetch_slots ||
         !aligned(expert_weights, 16) || !aligned(prefetch_slots, 16))
         return EP_ERR_INVALID_ARG;
-    // (slot, 16 KB chunk) items are counted in 32 bits
-    if ((bytes_per_expert / 16384 + 1) * (int64_t)h->d.R * h->d.S > INT32_MAX / 2) return EP_ERR_INVALID_ARG;
+    // (slot, 8 KB chunk) items are counted in 32 bits
+    if ((bytes_per_expert / 8192 + 1) * (int64_t)h->d.R * h->d.S > INT32_MAX / 2) return EP_ERR_INVALID_ARG;
     if (launch_prefetch(h->d, h->ws, expert_weights, bytes_per_expert, prefetch_slots, as_stream(stream)) !=
         cudaSuccess)
         return EP_ERR_CUDA;

@@ -265,8 +265,10 @@ ep_status_t ep_reduce_replica_grads(ep_handle_t *h, const float *replica_grad, f
  *   prefetch_slots[r, s, :] = expert_weights[e, :]   (bytes_per_expert bytes)
  * Empty slots are not written. expert_weights: device [E, bytes_per_expert];
  * prefetch_slots: device [R, S, bytes_per_expert]; both 16-byte aligned and
- * bytes_per_expert a positive multiple of 16. Reads the plan on the device:
- * no host sync. Needs cfg.balanced. */
+ * bytes_per_expert a positive multiple of 16, with R*S*(bytes_per_expert/8192
+ * + 1) at most 2^30 (the copy's 8 KB items are counted in 32 bits), else
+ * EP_ERR_INVALID_ARG. Reads the plan on the device: no host sync. Needs
+ * cfg.balanced. */
 ep_status_t ep_prefetch_replica_weights(ep_handle_t *h, const void *expert_weights, int64_t bytes_per_expert,
                                         void *prefetch_slots, void *stream);
 
