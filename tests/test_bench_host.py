@@ -132,3 +132,13 @@ def test_modelled_exchange_stays_flat_under_the_balanced_plan():
     assert flat == [flat[0]] * 4
     assert abs(flat[0] - 2 * (L // R) * 2 * H / 770e9 * 1e3) < 1e-9
     assert np.all(np.diff(plain) > 0) and plain[-1] > 5 * flat[0]
+
+
+def test_clock_records_that_reject_a_number():
+    ok = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.clocks_rejected(ok) is None
+    assert bench.clocks_rejected(dict(ok, reasons=["sw_power_cap"], sm_mhz=1500.0)) is None  # kept, noted
+    assert "hw_thermal_slowdown" in bench.clocks_rejected(dict(ok, reasons=["hw_thermal_slowdown"]))
+    assert "sw_thermal_slowdown" in bench.clocks_rejected(dict(ok, reasons=["sw_power_cap", "sw_thermal_slowdown"]))
+    assert "no reason" in bench.clocks_rejected(dict(ok, sm_mhz=1000.0))  # a leftover clock lock
+    assert bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": []}) is None
